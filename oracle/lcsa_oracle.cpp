@@ -1,0 +1,356 @@
+// LCSA CPU oracle: a plain, slow fp64 restatement of locality-constrained
+// sparse attention (LCSA) as used by FlashVSR's streaming video DiT.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing in the library path may call this code:
+// it is loaded by the tests, by the smoke check and by the CPU-baseline leg of
+// the benchmark, and by nothing else. It shares no code, header, table or
+// constant generator with the CUDA library.
+//
+// Sources of each step (page title, section):
+//  * "Add FlashVSR contrib model ... on Neuron" (aws-neuron NxDI PR), Model
+//    Information: 12 heads, head_dim 128, factored 3D RoPE, QK-norm done with
+//    DistributedRMSNorm; Additional Information: that norm all-reduces across
+//    tensor-parallel (head-sharded) ranks, so it spans all heads of a token.
+//  * "FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408", What Was Actually Slow
+//    and Rebuild sparse attention for Hopper: the attention glue is pooling,
+//    mask selection and RoPE; the sparse mask is turned into a CSR list.
+//  * "FlashVSR Inference" skill, Non-Negotiable Streaming Contract: kv_ratio
+//    3.0, local_range 11 or 9, topk_ratio = sparse_ratio*768*1280/(H*W).
+//  * "FlashVSR - Real-Time Diffusion-Based Video Super-Resolution" summary,
+//    How it works: attention limited to spatially local patches.
+//
+// Readings taken where the pages are silent:
+//  * norm scope: over the whole heads*head_dim token vector (token scope); a
+//    per-head scope is offered as well; eps = 1e-6.
+//  * 3D RoPE: the pairs (2i, 2i+1) of a head are rotated; the first
+//    d - 4*(d/6) dims follow the frame index, the next 2*(d/6) the token row,
+//    the last 2*(d/6) the token column; within an axis of n dims pair j turns
+//    by pos * 10000^(-2j/n). Parity of this schedule is unpinned against the
+//    pages (they only say "factored 3D RoPE").
+//  * block score: raw dot product of the block means of the normalised,
+//    rotated q and k (no scale).
+//  * window: odd local_range is a centred diameter in blocks, r = (lr-1)/2,
+//    Chebyshev distance over (block row, block column), clipped at the frame
+//    edge, the same in every frame of the KV window; 0 means unbounded.
+//  * budget: k = floor(topk_ratio * blocks per latent frame), H = 16 H',
+//    W = 16 W' (VAE 8x and 2x2 patchify), unless an explicit k is given.
+//  * query frames are the last q_frames of the KV window.
+//  * ties between equal scores go to the lower KV block index.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+struct Geom {
+  int batch, heads, head_dim;
+  int q_frames, kv_frames, grid_h, grid_w;
+  int block_t, block_h, block_w;
+  int local_range;   // 0 = unbounded
+  int topk;          // resolved budget in blocks, > 0
+  int kv_frame_offset;
+  int norm_scope;    // 0 = token (heads*d), 1 = head (d)
+  int threads;       // 0 = all hardware threads
+  double rms_eps;
+  double softmax_scale;
+};
+
+// ---- small helpers -------------------------------------------------------
+
+double bf16_to_double(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return static_cast<double>(f);
+}
+
+int n_threads(const Geom& g) {
+  int t = g.threads > 0 ? g.threads : static_cast<int>(std::thread::hardware_concurrency());
+  return t > 0 ? t : 1;
+}
+
+template <class F>
+void parallel_for(const Geom& g, int64_t n, F fn) {
+  int nt = static_cast<int>(std::min<int64_t>(n_threads(g), std::max<int64_t>(n, 1)));
+  std::atomic<int64_t> next(0);
+  auto worker = [&]() {
+    for (;;) {
+      int64_t i = next.fetch_add(1);
+      if (i >= n) return;
+      fn(i);
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 1; t < nt; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
+}
+
+struct Derived {
+  int64_t tokens_per_frame, Lq, Lkv, C, nb, nHb, nWb, bpf, nQB, nKB;
+};
+
+Derived derive(const Geom& g) {
+  Derived d{};
+  d.tokens_per_frame = int64_t(g.grid_h) * g.grid_w;
+  d.Lq = g.q_frames * d.tokens_per_frame;
+  d.Lkv = g.kv_frames * d.tokens_per_frame;
+  d.C = int64_t(g.heads) * g.head_dim;
+  d.nb = int64_t(g.block_t) * g.block_h * g.block_w;
+  d.nHb = g.grid_h / g.block_h;
+  d.nWb = g.grid_w / g.block_w;
+  d.bpf = d.nHb * d.nWb;
+  d.nQB = (g.q_frames / g.block_t) * d.bpf;
+  d.nKB = (g.kv_frames / g.block_t) * d.bpf;
+  return d;
+}
+
+// Raster token index of token i (0 .. nb-1) of block `blk`. Blocks are
+// numbered frame-group major, then block row, then block column; tokens of a
+// block are numbered frame, row, column.
+int64_t block_token(const Geom& g, const Derived& d, int64_t blk, int64_t i) {
+  int64_t tb = blk / d.bpf, rem = blk % d.bpf;
+  int64_t hb = rem / d.nWb, wb = rem % d.nWb;
+  int64_t tt = i / (int64_t(g.block_h) * g.block_w);
+  int64_t yy = (i / g.block_w) % g.block_h;
+  int64_t xx = i % g.block_w;
+  int64_t t = tb * g.block_t + tt, y = hb * g.block_h + yy, x = wb * g.block_w + xx;
+  return (t * g.grid_h + y) * g.grid_w + x;
+}
+
+// RMSNorm over the chosen scope, gain, then the factored 3D rotation. `x` is
+// the token's heads*d bf16 vector; `out` receives heads*d doubles.
+void norm_rope_token(const Geom& g, const Derived& d, const uint16_t* x, const float* gamma,
+                     bool is_q, int64_t tok, double* out) {
+  const int D = g.head_dim;
+  for (int64_t c = 0; c < d.C; ++c) out[c] = bf16_to_double(x[c]);
+  if (g.norm_scope == 0) {
+    double ss = 0.0;
+    for (int64_t c = 0; c < d.C; ++c) ss += out[c] * out[c];
+    double inv = 1.0 / std::sqrt(ss / double(d.C) + g.rms_eps);
+    for (int64_t c = 0; c < d.C; ++c) out[c] = out[c] * inv * double(gamma[c]);
+  } else {
+    for (int h = 0; h < g.heads; ++h) {
+      double ss = 0.0;
+      for (int e = 0; e < D; ++e) ss += out[h * D + e] * out[h * D + e];
+      double inv = 1.0 / std::sqrt(ss / double(D) + g.rms_eps);
+      for (int e = 0; e < D; ++e) out[h * D + e] = out[h * D + e] * inv * double(gamma[h * D + e]);
+    }
+  }
+  // position of the token on the (frame, row, column) grid
+  int64_t t_local = tok / d.tokens_per_frame;
+  int64_t y = (tok / g.grid_w) % g.grid_h;
+  int64_t xcol = tok % g.grid_w;
+  double t_abs = double(g.kv_frame_offset) + double(is_q ? (g.kv_frames - g.q_frames) : 0) + double(t_local);
+  const int dims_h = 2 * (D / 6), dims_w = 2 * (D / 6), dims_t = D - dims_h - dims_w;
+  const int pairs_t = dims_t / 2, pairs_h = dims_h / 2;
+  std::vector<double> cs(D / 2), sn(D / 2);
+  for (int j = 0; j < D / 2; ++j) {
+    double pos, expo;
+    if (j < pairs_t) {
+      pos = t_abs;
+      expo = 2.0 * j / dims_t;
+    } else if (j < pairs_t + pairs_h) {
+      pos = double(y);
+      expo = 2.0 * (j - pairs_t) / dims_h;
+    } else {
+      pos = double(xcol);
+      expo = 2.0 * (j - pairs_t - pairs_h) / dims_w;
+    }
+    double ang = pos * std::pow(10000.0, -expo);
+    cs[j] = std::cos(ang);
+    sn[j] = std::sin(ang);
+  }
+  for (int h = 0; h < g.heads; ++h) {
+    for (int j = 0; j < D / 2; ++j) {
+      double a = out[h * D + 2 * j], b = out[h * D + 2 * j + 1];
+      out[h * D + 2 * j] = a * cs[j] - b * sn[j];
+      out[h * D + 2 * j + 1] = a * sn[j] + b * cs[j];
+    }
+  }
+}
+
+bool admissible(const Geom& g, const Derived& d, int64_t qb, int64_t kb) {
+  if (g.local_range <= 0) return true;
+  int64_t r = (g.local_range - 1) / 2;
+  int64_t qrem = qb % d.bpf, krem = kb % d.bpf;
+  int64_t dh = qrem / d.nWb - krem / d.nWb, dw = qrem % d.nWb - krem % d.nWb;
+  return std::llabs(dh) <= r && std::llabs(dw) <= r;
+}
+
+}  // namespace
+
+extern "C" {
+
+typedef Geom ora_geom;
+
+// Budget in blocks from the pages' topk_ratio rule:
+// topk_ratio = sparse_ratio*768*1280/(H*W), H = 16*grid_h, W = 16*grid_w,
+// k = floor(topk_ratio * blocks per latent frame). All factors are integers
+// except sparse_ratio, so the product is formed before the one division.
+int ora_resolve_topk(double sparse_ratio, int grid_h, int grid_w, int block_t, int block_h, int block_w) {
+  double H = 16.0 * grid_h, W = 16.0 * grid_w;
+  double blocks_per_frame = double(grid_h / block_h) * double(grid_w / block_w);
+  (void)block_t;
+  double num = sparse_ratio * 768.0 * 1280.0 * blocks_per_frame;
+  double k = std::floor(num / (H * W));
+  return static_cast<int>(k);
+}
+
+// Normalised, rotated vectors (all heads) of chosen tokens. `tokens` holds
+// b*L + raster index per entry; out is [ntok][heads*d].
+void ora_norm_rope(const ora_geom* gp, const uint16_t* x, const float* gamma, int is_q,
+                   const int64_t* tokens, int64_t ntok, double* out) {
+  const Geom& g = *gp;
+  Derived d = derive(g);
+  int64_t L = is_q ? d.Lq : d.Lkv;
+  parallel_for(g, ntok, [&](int64_t n) {
+    int64_t bt = tokens[n];
+    int64_t tok = bt % L;
+    norm_rope_token(g, d, x + bt * d.C, gamma, is_q != 0, tok, out + n * d.C);
+  });
+}
+
+// Block means of the normalised, rotated vectors: pooled[b][h][blk][d].
+void ora_pool(const ora_geom* gp, const uint16_t* x, const float* gamma, int is_q, double* pooled) {
+  const Geom& g = *gp;
+  Derived d = derive(g);
+  int64_t L = is_q ? d.Lq : d.Lkv;
+  int64_t nblk = is_q ? d.nQB : d.nKB;
+  const int D = g.head_dim;
+  parallel_for(g, int64_t(g.batch) * nblk, [&](int64_t job) {
+    int64_t b = job / nblk, blk = job % nblk;
+    std::vector<double> acc(d.C, 0.0), v(d.C);
+    for (int64_t i = 0; i < d.nb; ++i) {
+      int64_t tok = block_token(g, d, blk, i);
+      norm_rope_token(g, d, x + (b * L + tok) * d.C, gamma, is_q != 0, tok, v.data());
+      for (int64_t c = 0; c < d.C; ++c) acc[c] += v[c];
+    }
+    for (int h = 0; h < g.heads; ++h)
+      for (int e = 0; e < D; ++e)
+        pooled[((b * g.heads + h) * nblk + blk) * D + e] = acc[h * D + e] / double(d.nb);
+  });
+}
+
+// Admissible-set size of every query block (depends on geometry only).
+void ora_window_sizes(const ora_geom* gp, int32_t* sizes) {
+  const Geom& g = *gp;
+  Derived d = derive(g);
+  for (int64_t qb = 0; qb < d.nQB; ++qb) {
+    int32_t n = 0;
+    for (int64_t kb = 0; kb < d.nKB; ++kb) n += admissible(g, d, qb, kb) ? 1 : 0;
+    sizes[qb] = n;
+  }
+}
+
+// Scores, window, top-k. Rows are (b, h, qb) in that nesting. For each row:
+// row_len = min(k, |A|), cols[row][0..row_len) ascending, gap = score of the
+// k-th best minus the (k+1)-th best admissible block (+inf when all of A is
+// kept), kth = score of the k-th best. `scores` (nullable) receives the full
+// [rows][nKB] score matrix with non-admissible entries set to -inf.
+void ora_select(const ora_geom* gp, const double* pq, const double* pk, int32_t* row_len,
+                int32_t* cols, int cap, double* gap, double* scores) {
+  const Geom& g = *gp;
+  Derived d = derive(g);
+  const int D = g.head_dim;
+  int64_t rows = int64_t(g.batch) * g.heads * d.nQB;
+  parallel_for(g, rows, [&](int64_t row) {
+    int64_t bh = row / d.nQB, qb = row % d.nQB;
+    const double* q = pq + row * D;
+    std::vector<std::pair<double, int64_t>> cand;
+    for (int64_t kb = 0; kb < d.nKB; ++kb) {
+      double s = 0.0;
+      const double* kk = pk + (bh * d.nKB + kb) * D;
+      for (int e = 0; e < D; ++e) s += q[e] * kk[e];
+      bool ok = admissible(g, d, qb, kb);
+      if (scores) scores[row * d.nKB + kb] = ok ? s : -std::numeric_limits<double>::infinity();
+      if (ok) cand.emplace_back(s, kb);
+    }
+    std::sort(cand.begin(), cand.end(), [](const std::pair<double, int64_t>& a, const std::pair<double, int64_t>& b) {
+      if (a.first != b.first) return a.first > b.first;
+      return a.second < b.second;
+    });
+    int64_t keff = std::min<int64_t>(g.topk, int64_t(cand.size()));
+    row_len[row] = int32_t(keff);
+    gap[row] = keff < int64_t(cand.size()) ? cand[keff - 1].first - cand[keff].first
+                                           : std::numeric_limits<double>::infinity();
+    std::vector<int64_t> sel;
+    for (int64_t i = 0; i < keff; ++i) sel.push_back(cand[i].second);
+    std::sort(sel.begin(), sel.end());
+    for (int64_t i = 0; i < keff && i < cap; ++i) cols[row * cap + i] = int32_t(sel[i]);
+  });
+}
+
+// Exact softmax attention of the requested rows over the tokens of their
+// selected blocks. rows[n] is a (b, h, qb) row number; its block list is
+// cols[row][0 .. row_len[row]). out is [nrows][nb][d] (fp64, before any
+// rounding), wsum [nrows][nb] the sum of the normalised weights.
+void ora_attention(const ora_geom* gp, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const float* gamma_q, const float* gamma_k, const int32_t* row_len,
+                   const int32_t* cols, int cap, const int64_t* rows, int64_t nrows, double* out,
+                   double* wsum) {
+  const Geom& g = *gp;
+  Derived d = derive(g);
+  const int D = g.head_dim;
+  parallel_for(g, nrows, [&](int64_t n) {
+    int64_t row = rows[n];
+    int64_t bh = row / d.nQB, qb = row % d.nQB;
+    int64_t b = bh / g.heads, h = bh % g.heads;
+    int64_t nsel = row_len[row];
+    std::vector<double> tokvec(d.C);
+    // normalised, rotated query rows of this block (head h)
+    std::vector<double> qh(d.nb * D);
+    for (int64_t i = 0; i < d.nb; ++i) {
+      int64_t tok = block_token(g, d, qb, i);
+      norm_rope_token(g, d, q + (b * d.Lq + tok) * d.C, gamma_q, true, tok, tokvec.data());
+      for (int e = 0; e < D; ++e) qh[i * D + e] = tokvec[h * D + e];
+    }
+    // keys and values of the selected blocks (head h)
+    int64_t nkey = nsel * d.nb;
+    std::vector<double> kh(nkey * D), vh(nkey * D);
+    for (int64_t s = 0; s < nsel; ++s) {
+      int64_t kb = cols[row * cap + s];
+      for (int64_t i = 0; i < d.nb; ++i) {
+        int64_t tok = block_token(g, d, kb, i);
+        norm_rope_token(g, d, k + (b * d.Lkv + tok) * d.C, gamma_k, false, tok, tokvec.data());
+        for (int e = 0; e < D; ++e) {
+          kh[(s * d.nb + i) * D + e] = tokvec[h * D + e];
+          vh[(s * d.nb + i) * D + e] = bf16_to_double(v[(b * d.Lkv + tok) * d.C + h * D + e]);
+        }
+      }
+    }
+    std::vector<double> logit(nkey);
+    for (int64_t i = 0; i < d.nb; ++i) {
+      double mx = -std::numeric_limits<double>::infinity();
+      for (int64_t j = 0; j < nkey; ++j) {
+        double s = 0.0;
+        for (int e = 0; e < D; ++e) s += qh[i * D + e] * kh[j * D + e];
+        logit[j] = s * g.softmax_scale;
+        mx = std::max(mx, logit[j]);
+      }
+      double l = 0.0;
+      for (int64_t j = 0; j < nkey; ++j) {
+        logit[j] = std::exp(logit[j] - mx);
+        l += logit[j];
+      }
+      double* o = out + (n * d.nb + i) * D;
+      for (int e = 0; e < D; ++e) o[e] = 0.0;
+      double ws = 0.0;
+      for (int64_t j = 0; j < nkey; ++j) {
+        double p = logit[j] / l;
+        ws += p;
+        for (int e = 0; e < D; ++e) o[e] += p * vh[j * D + e];
+      }
+      if (wsum) wsum[n * d.nb + i] = ws;
+    }
+  });
+}
+
+int ora_hardware_threads(void) { return static_cast<int>(std::thread::hardware_concurrency()); }
+
+}  // extern "C"
