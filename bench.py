@@ -1,0 +1,362 @@
+"""LCSA benchmark: ms per call and effective TFLOP/s (kept blocks only).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one whole LCSA call (prologue, block selection, block-sparse
+attention) on one stream chunk of synthetic inputs already resident in HBM.
+The default workload is the 768x1280 stream chunk: 2 query frames of 48x80
+tokens, a 6-frame KV window, 12 heads, head_dim 128, 1x8x16 blocks,
+local_range 11, sparse_ratio 2.0 (k = 60 blocks).
+
+Timing: W untimed warm-up calls, then exactly K timed calls, each between
+its own pair of CUDA events on the launching stream; a 256 MiB buffer is
+written before every timed call so each call starts with a cold L2. The
+timed region is bracketed by a barrier and a device synchronise; the
+reported time is the maximum over ranks. Under torchrun every rank runs its
+own independent chunk (weak scaling, no collective on the data path).
+
+--impl reference times the fp64 CPU oracle (the independent checker) on the
+host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LCSA ms/call and effective TFLOP/s (selected blocks) at 768×1280 stream chunk"
+UNIT = "TFLOP/s"
+FLUSH_BYTES = 256 << 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="stream_768x1280")
+    ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def _kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_video_lcsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(kernel_tag, files):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (same hash); else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = _kernel_source_hash(files)
+    with open(path) as f:
+        for line in f:
+            m = re.match(r"\s*(\w+)\s+src=(\w+)\s+workload=(\S+)\s+dram_bytes_per_launch=([0-9.eE+]+)", line)
+            if m and m.group(1) == kernel_tag and m.group(2) == want:
+                return float(m.group(4))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _oracle_sample(wl, inp, target_s=12.0):
+    """Time the fp64 oracle on a bounded sample: pooled values and selection
+    for the whole chunk, attention for a sample of rows; the full-call time is
+    extrapolated by the row count."""
+    import numpy as np
+    import oracle
+
+    og = oracle.Geometry.from_workload(wl)
+    threads = oracle.hardware_threads()
+    t0 = time.perf_counter()
+    pq = oracle.pool(og, inp.q, inp.gamma_q, True)
+    pk = oracle.pool(og, inp.k, inp.gamma_k, False)
+    sel = oracle.select(og, pq, pk)
+    t_pre = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    n = min(og.rows, max(threads, 4))
+    rows = np.sort(rng.choice(og.rows, size=n, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attention(og, inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, sel, rows)
+    t_probe = time.perf_counter() - t0
+    # grow the sample to about target_s of attention work
+    n2 = int(min(og.rows, max(n, n * max(1.0, (target_s - t_pre) / max(t_probe, 1e-3)))))
+    if n2 > n:
+        rows = np.sort(rng.choice(og.rows, size=n2, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(og, inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, sel, rows)
+        t_attn = time.perf_counter() - t0
+    else:
+        n2, t_attn = n, t_probe
+    full_s = t_pre + t_attn * og.rows / n2
+    flops = float(np.minimum(oracle.window_sizes(og), og.topk).sum()) * og.batch * og.heads * 4.0 * og.nb ** 2 * \
+        og.head_dim
+    return {"value": flops / full_s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "ms_per_call": full_s * 1e3,
+            "sample": "fp64 oracle: pooling + selection of the whole chunk (%.2f s), attention of %d of %d rows "
+                      "(%.2f s), call time extrapolated by rows" % (t_pre, n2, og.rows, t_attn)}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    from block_sparse_video_lcsa_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl)
+    samples = []
+    for i in range(args.warmup + args.steps):
+        r = _oracle_sample(wl, inp, target_s=2.0)
+        if i >= args.warmup:
+            samples.append(r)
+    ms = statistics.mean(s["ms_per_call"] for s in samples)
+    value = statistics.mean(s["value"] for s in samples)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[-1]["cores"], "kind": "oracle",
+                             "sample": samples[-1]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_lcsa(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_video_lcsa_b200 as lcsa
+    from block_sparse_video_lcsa_b200 import synth
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload].replace(seed=rank)
+    inp = synth.make_inputs(wl)
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+
+    q, k, v = bf(inp.q), bf(inp.k), bf(inp.v)
+    gq, gk = torch.from_numpy(inp.gamma_q).to(dev), torch.from_numpy(inp.gamma_k).to(dev)
+    out = torch.empty_like(q)
+    plan = lcsa.lcsa_plan_create(lcsa.config_from_workload(wl, host_io=1), local)
+    geo = plan.geometry
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        plan.lcsa_forward(q, k, v, gq, gk, out, stream)
+    plan.lcsa_check_device_error(stream)
+
+    plan.lcsa_plan_set_timing(args.steps)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    try:
+        gpu_id = "GPU-%s" % torch.cuda.get_device_properties(dev).uuid
+    except Exception:  # noqa: BLE001 - fall back to the index
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            plan.lcsa_forward(q, k, v, gq, gk, out, stream)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    plan.lcsa_check_device_error(stream)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kms, kcount = plan.lcsa_get_kernel_times()
+    plan.lcsa_plan_set_timing(0)
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end: pinned host buffers through lcsa_forward_host (copies inside)
+    hq = torch.from_numpy(inp.q).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(inp.k).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(inp.v).view(torch.bfloat16).pin_memory()
+    hgq = torch.from_numpy(inp.gamma_q).pin_memory()
+    hgk = torch.from_numpy(inp.gamma_k).pin_memory()
+    hout = torch.empty(tuple(q.shape), dtype=torch.bfloat16).pin_memory()
+    plan.lcsa_forward_host(hq, hk, hv, hgq, hgk, hout, stream)
+    e2e_steps = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        plan.lcsa_forward_host(hq, hk, hv, hgq, hgk, hout, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+    plan.destroy()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks = _peaks()
+    flops = geo.selected_flops
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    k3_tflops = flops / (kms[2] * 1e-3) / 1e12
+    k1_gbs = geo.prologue_bytes / (kms[0] * 1e-3) / 1e9
+    traffic = _profiled_traffic("k3", ["k3_attention_mma.cu", "lcsa_internal.h"])
+    roofline = {"bound": "tensor", "kernel": "attention (K3)", "achieved": k3_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": k3_tflops / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": peaks["source"] + " burst bf16",
+                "algorithmic_flops_per_launch": flops}
+    h2d = (inp.q.nbytes + inp.k.nbytes + inp.v.nbytes + inp.gamma_q.nbytes + inp.gamma_k.nbytes)
+    d2h = inp.q.nbytes
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "q_tokens": geo.q_tokens, "kv_tokens": geo.kv_tokens,
+                       "heads": wl.heads, "head_dim": wl.head_dim,
+                       "block": "%dx%dx%d" % (wl.block_t, wl.block_h, wl.block_w), "local_range": wl.local_range,
+                       "sparse_ratio": wl.sparse_ratio, "topk": geo.topk, "kept_blocks": geo.nnz,
+                       "l2": "256 MiB buffer written before every timed call", "parallelism": "replicas%d" % world},
+            "roofline": roofline,
+            "kernels": {"prologue_ms": kms[0], "select_ms": kms[1], "attention_ms": kms[2], "timed_calls": kcount,
+                        "prologue_gbs": k1_gbs, "prologue_hbm_frac": k1_gbs / peaks["hbm_gbs"],
+                        "prologue_bytes": geo.prologue_bytes, "hbm_peak_gbs": peaks["hbm_gbs"]},
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary()}
+    if world == 1 and not args.no_cpu_baseline:
+        cb = _oracle_sample(wl, inp)
+        cb.pop("ms_per_call")
+        line["cpu_baseline"] = cb
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_lcsa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,276 @@
-"""B200-native LCSA (locality-constrained sparse attention) library binding."""
+"""B200-native LCSA (locality-constrained sparse attention) library binding.
+
+A thin ctypes face of ``liblcsa.so`` (declared in include/lcsa.h): the same
+entry-point names, argument marshalling only. Every step of the call runs in
+the library's CUDA kernels; there is no Python or CPU fallback, and using the
+binding without the built library raises ``LcsaLibraryMissing``.
+
+Tensors are passed as torch CUDA tensors (bf16 q, k, v, out; fp32 gains) or
+as raw device addresses (int).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcsa.so")
+
+LCSA_OK = 0
+LCSA_ERR_INVALID_ARG = 1
+LCSA_ERR_SHAPE = 2
+LCSA_ERR_ALIGNMENT = 3
+LCSA_ERR_UNSUPPORTED = 4
+LCSA_ERR_OOM = 5
+LCSA_ERR_CUDA = 6
+LCSA_ERR_DEVICE_TIMEOUT = 7
+LCSA_ERR_DEVICE_BOUNDS = 8
+LCSA_UNBOUNDED = 0
+LCSA_NORM_TOKEN = 0
+LCSA_NORM_HEAD = 1
+
+
+class LcsaLibraryMissing(ImportError):
+    pass
+
+
+class LcsaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (where, _status_name(status), detail))
+
+
+class lcsa_config_t(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("q_frames", ctypes.c_int), ("kv_frames", ctypes.c_int),
+        ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+        ("block_t", ctypes.c_int), ("block_h", ctypes.c_int), ("block_w", ctypes.c_int),
+        ("local_range", ctypes.c_int), ("topk", ctypes.c_int), ("sparse_ratio", ctypes.c_float),
+        ("kv_frame_offset", ctypes.c_int), ("norm_scope", ctypes.c_int),
+        ("rms_eps", ctypes.c_float), ("softmax_scale", ctypes.c_float), ("host_io", ctypes.c_int),
+    ]
+
+
+class lcsa_geometry_t(ctypes.Structure):
+    _fields_ = [
+        ("q_tokens", ctypes.c_int64), ("kv_tokens", ctypes.c_int64), ("channels", ctypes.c_int64),
+        ("block_tokens", ctypes.c_int64), ("blocks_per_frame", ctypes.c_int64),
+        ("q_blocks", ctypes.c_int64), ("kv_blocks", ctypes.c_int64), ("rows", ctypes.c_int64),
+        ("nnz", ctypes.c_int64), ("topk", ctypes.c_int), ("window_radius", ctypes.c_int),
+        ("min_window", ctypes.c_int), ("max_window", ctypes.c_int),
+        ("selected_flops", ctypes.c_double), ("prologue_bytes", ctypes.c_double),
+        ("attention_min_bytes", ctypes.c_double), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+# (name, restype, argtypes) of every entry point in include/lcsa.h
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_PLAN = ctypes.c_void_p
+SIGNATURES = [
+    ("lcsa_config_default", None, [ctypes.POINTER(lcsa_config_t)]),
+    ("lcsa_config_resolve", _I, [ctypes.POINTER(lcsa_config_t), ctypes.POINTER(lcsa_geometry_t)]),
+    ("lcsa_plan_create", _I, [ctypes.POINTER(lcsa_config_t), _I, ctypes.POINTER(_PLAN)]),
+    ("lcsa_plan_destroy", None, [_PLAN]),
+    ("lcsa_forward", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_forward_host", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_plan_geometry", _I, [_PLAN, ctypes.POINTER(lcsa_geometry_t)]),
+    ("lcsa_plan_topk", _I, [_PLAN, ctypes.POINTER(_I)]),
+    ("lcsa_get_selection", _I, [_PLAN, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t]),
+    ("lcsa_get_intermediates", _I, [_PLAN, _VP, _VP, _VP, _VP]),
+    ("lcsa_check_device_error", _I, [_PLAN, _VP]),
+    ("lcsa_plan_set_timing", _I, [_PLAN, _I]),
+    ("lcsa_get_kernel_times", _I, [_PLAN, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I)]),
+    ("lcsa_status_string", ctypes.c_char_p, [_I]),
+    ("lcsa_last_error_message", ctypes.c_char_p, []),
+    ("lcsa_abi_version", _I, []),
+]
+
+_lib = None
+
+
+def lib():
+    """The loaded liblcsa.so (raises LcsaLibraryMissing if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise LcsaLibraryMissing(
+                "liblcsa.so is not built (python -m block_sparse_video_lcsa_b200.build); "
+                "there is no fallback implementation")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _status_name(st: int) -> str:
+    try:
+        return lib().lcsa_status_string(st).decode()
+    except Exception:  # noqa: BLE001 - only used to format an error
+        return "status %d" % st
+
+
+def _check(st: int, where: str):
+    if st != LCSA_OK:
+        raise LcsaError(st, where, lib().lcsa_last_error_message().decode())
+
+
+def _addr(x) -> int:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ---- entry points, same names as the C ABI --------------------------------
+
+def lcsa_config_default() -> lcsa_config_t:
+    c = lcsa_config_t()
+    lib().lcsa_config_default(ctypes.byref(c))
+    return c
+
+
+def lcsa_config_resolve(cfg: lcsa_config_t) -> lcsa_geometry_t:
+    g = lcsa_geometry_t()
+    _check(lib().lcsa_config_resolve(ctypes.byref(cfg), ctypes.byref(g)), "lcsa_config_resolve")
+    return g
+
+
+def lcsa_plan_create(cfg: lcsa_config_t, device: int = 0) -> "Plan":
+    h = _PLAN()
+    _check(lib().lcsa_plan_create(ctypes.byref(cfg), int(device), ctypes.byref(h)), "lcsa_plan_create")
+    return Plan(h, cfg)
+
+
+def config_from_workload(wl, **over) -> lcsa_config_t:
+    """lcsa_config_t of a named workload (synth.WORKLOADS entry)."""
+    c = lcsa_config_default()
+    for name in ("batch", "heads", "head_dim", "q_frames", "kv_frames", "grid_h", "grid_w", "block_t", "block_h",
+                 "block_w", "local_range", "topk", "sparse_ratio", "kv_frame_offset"):
+        setattr(c, name, getattr(wl, name))
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+class Plan:
+    """Owner of an lcsa_plan_t; every method maps to one C entry point."""
+
+    def __init__(self, handle, cfg):
+        self._h = handle
+        self.cfg = cfg
+        g = lcsa_geometry_t()
+        _check(lib().lcsa_plan_geometry(self._h, ctypes.byref(g)), "lcsa_plan_geometry")
+        self.geometry = g
+
+    @property
+    def handle(self):
+        return self._h
+
+    def destroy(self):
+        if self._h is not None and self._h.value:
+            lib().lcsa_plan_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+    def _expect(self, t, dtype, shape, name):
+        if isinstance(t, int):
+            return
+        import torch
+        if t.dtype != dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+            raise ValueError("%s: want contiguous CUDA %s %s, got %s %s %s" % (
+                name, dtype, tuple(shape), t.dtype, tuple(t.shape), t.device))
+        _ = torch  # the check above needs torch only for real tensors
+
+    def lcsa_forward(self, q, k, v, gamma_q, gamma_k, out, stream=None):
+        import torch
+        c, g = self.cfg, self.geometry
+        self._expect(q, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "q")
+        self._expect(k, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "k")
+        self._expect(v, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "v")
+        self._expect(out, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "out")
+        self._expect(gamma_q, torch.float32, (g.channels,), "gamma_q")
+        self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k")
+        _check(lib().lcsa_forward(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
+                                  _addr(out), _stream(stream)), "lcsa_forward")
+        return out
+
+    forward = lcsa_forward
+
+    def lcsa_forward_host(self, q, k, v, gamma_q, gamma_k, out, stream=None):
+        """Host (preferably pinned) tensors in and out; copies are inside the call."""
+        _check(lib().lcsa_forward_host(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
+                                       _addr(out), _stream(stream)), "lcsa_forward_host")
+        return out
+
+    def lcsa_plan_topk(self) -> int:
+        k = ctypes.c_int()
+        _check(lib().lcsa_plan_topk(self._h, ctypes.byref(k)), "lcsa_plan_topk")
+        return k.value
+
+    def lcsa_get_selection(self):
+        import numpy as np
+        g = self.geometry
+        rp = np.empty(g.rows + 1, dtype=np.int32)
+        ci = np.empty(max(1, g.nnz), dtype=np.int32)
+        _check(lib().lcsa_get_selection(self._h, rp.ctypes.data, rp.size, ci.ctypes.data, ci.size),
+               "lcsa_get_selection")
+        return rp, ci[: g.nnz]
+
+    def lcsa_get_intermediates(self):
+        """(q^, k^ as uint16 bf16 bits, pooled q, pooled k) in the plan's layouts."""
+        import numpy as np
+        c, g = self.cfg, self.geometry
+        qh = np.empty((c.batch, c.heads, g.q_blocks, g.block_tokens, c.head_dim), dtype=np.uint16)
+        kh = np.empty((c.batch, c.heads, g.kv_blocks, g.block_tokens, c.head_dim), dtype=np.uint16)
+        pq = np.empty((c.batch, c.heads, g.q_blocks, c.head_dim), dtype=np.float32)
+        pk = np.empty((c.batch, c.heads, g.kv_blocks, c.head_dim), dtype=np.float32)
+        _check(lib().lcsa_get_intermediates(self._h, qh.ctypes.data, kh.ctypes.data, pq.ctypes.data,
+                                            pk.ctypes.data), "lcsa_get_intermediates")
+        return qh, kh, pq, pk
+
+    def lcsa_check_device_error(self, stream=None):
+        _check(lib().lcsa_check_device_error(self._h, _stream(stream)), "lcsa_check_device_error")
+
+    def lcsa_plan_set_timing(self, capacity: int):
+        _check(lib().lcsa_plan_set_timing(self._h, int(capacity)), "lcsa_plan_set_timing")
+
+    def lcsa_get_kernel_times(self):
+        """(mean ms of prologue, select, attention; number of calls averaged)."""
+        ms = (ctypes.c_float * 3)()
+        n = ctypes.c_int()
+        _check(lib().lcsa_get_kernel_times(self._h, ms, ctypes.byref(n)), "lcsa_get_kernel_times")
+        return list(ms), n.value
+
+
+def lcsa_status_string(status: int) -> str:
+    return lib().lcsa_status_string(int(status)).decode()
+
+
+def lcsa_last_error_message() -> str:
+    return lib().lcsa_last_error_message().decode()
+
+
+def lcsa_abi_version() -> int:
+    return int(lib().lcsa_abi_version())

@@ -1,0 +1,152 @@
+// K2: LCSA block selection. For every (batch, head, query block) row: score
+// each KV block inside the local window by the dot product of the pooled q
+// and pooled k vectors, keep the k best (equal scores: lower block index
+// first) and write the kept block indices in ascending order into the row's
+// CSR slot.
+//
+// Pages: "FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408", What Was Actually
+// Slow (mask selection as glue) and Rebuild sparse attention for Hopper (fused
+// CSR construction); "FlashVSR Inference" skill, Non-Negotiable Streaming
+// Contract (local_range, topk_ratio); "FlashVSR - Real-Time Diffusion-Based
+// Video Super-Resolution", How it works (attention limited to local patches).
+//
+// Determinism: a score is the fp32 sum of four products per lane followed by
+// a butterfly over the warp; every lane ends with the same bits, and the order
+// never depends on timing. The sort key is (order-preserving score bits << 32)
+// | (~block index), so one descending sort of unique keys gives the k best
+// with ties broken toward the lower index. The CSR row offsets depend only on
+// the geometry and are computed once when the plan is made.
+#include "lcsa_internal.h"
+
+namespace lcsa {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kCandPerIter = 4;  // candidates in flight per warp
+
+__device__ __forceinline__ unsigned order_bits(float s) {
+  const unsigned u = __float_as_uint(s + 0.0f);  // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
+  extern __shared__ unsigned long long keys[];  // [sort_n], then flags [sort_n] bytes
+  unsigned char* flag = reinterpret_cast<unsigned char*>(keys + p.sort_n);
+  __shared__ int warp_sum[kWarps];
+  const Grid& g = p.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rr = blockIdx.x;
+  const int bh = rr / g.nQB, qb = rr % g.nQB;
+  const int rem = qb % g.bpf, hb = rem / g.nWb, wb = rem % g.nWb;
+  int h0 = 0, h1 = g.nHb - 1, w0 = 0, w1 = g.nWb - 1;
+  if (p.radius >= 0) {
+    h0 = max(hb - p.radius, 0);
+    h1 = min(hb + p.radius, g.nHb - 1);
+    w0 = max(wb - p.radius, 0);
+    w1 = min(wb + p.radius, g.nWb - 1);
+  }
+  const int nh = h1 - h0 + 1, nw = w1 - w0 + 1, per = nh * nw;
+  const int nc = (g.nKB / g.bpf) * per;  // admissible blocks, ascending index order
+
+  const float4 qv = reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * kHeadDim)[lane];
+  const float4* pk = reinterpret_cast<const float4*>(p.pooled_k + int64_t(bh) * g.nKB * kHeadDim);
+
+  for (int c = threadIdx.x; c < p.sort_n; c += kThreads) flag[c] = 0;
+  for (int c0 = warp * kCandPerIter; c0 < p.sort_n; c0 += kWarps * kCandPerIter) {
+    float4 kv[kCandPerIter];
+    int kb[kCandPerIter];
+#pragma unroll
+    for (int u = 0; u < kCandPerIter; ++u) {
+      const int c = c0 + u;
+      kb[u] = -1;
+      kv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < nc) {
+        const int tk = c / per, r2 = c % per;
+        kb[u] = tk * g.bpf + (h0 + r2 / nw) * g.nWb + (w0 + r2 % nw);
+        kv[u] = pk[int64_t(kb[u]) * (kHeadDim / 4) + lane];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCandPerIter; ++u) {
+      float s = qv.x * kv[u].x;
+      s = fmaf(qv.y, kv[u].y, s);
+      s = fmaf(qv.z, kv[u].z, s);
+      s = fmaf(qv.w, kv[u].w, s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const int c = c0 + u;
+      if (lane == 0 && c < p.sort_n)
+        keys[c] = kb[u] >= 0 ? ((unsigned long long)order_bits(s) << 32) | (0xFFFFFFFFu - unsigned(kb[u]))
+                             : 0ull;
+    }
+  }
+  __syncthreads();
+
+  // bitonic sort, descending
+  const int n = p.sort_n;
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += kThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], bk = keys[ixj];
+          const bool desc = (i & k) == 0;
+          if (desc ? (a < bk) : (a > bk)) {
+            keys[i] = bk;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // mark the kept candidates, then compact them in ascending block order
+  const int keff = min(p.topk, nc);
+  for (int i = threadIdx.x; i < keff; i += kThreads) {
+    const int kbi = int(0xFFFFFFFFu - unsigned(keys[i] & 0xFFFFFFFFull));
+    const int tk = kbi / g.bpf, r2 = kbi % g.bpf;
+    const int c = (tk * nh + (r2 / g.nWb - h0)) * nw + (r2 % g.nWb - w0);
+    flag[c] = 1;
+  }
+  __syncthreads();
+  const int span = (nc + kThreads - 1) / kThreads;
+  const int c_beg = threadIdx.x * span, c_end = min(c_beg + span, nc);
+  int cnt = 0;
+  for (int c = c_beg; c < c_end; ++c) cnt += flag[c];
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_sum[w];
+  int pos = p.row_ptr[rr] + base + incl - cnt;
+  for (int c = c_beg; c < c_end; ++c) {
+    if (flag[c]) {
+      const int tk = c / per, r2 = c % per;
+      p.col_idx[pos++] = tk * g.bpf + (h0 + r2 / nw) * g.nWb + (w0 + r2 % nw);
+    }
+  }
+}
+
+}  // namespace
+
+size_t select_smem_bytes(int sort_n) { return size_t(sort_n) * (sizeof(unsigned long long) + 1); }
+
+cudaError_t launch_select(const K2Params& p, cudaStream_t s) {
+  const size_t smem = select_smem_bytes(p.sort_n);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int rows = p.g.B * p.g.Hn * p.g.nQB;
+  select_kernel<<<rows, kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace lcsa

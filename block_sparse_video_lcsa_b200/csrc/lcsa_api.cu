@@ -1,0 +1,547 @@
+// Host side of liblcsa: configuration checks, plan (workspace) management and
+// the three-kernel forward call. Every entry point returns a status code; no
+// path aborts, throws across the ABI or substitutes another implementation.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <array>
+#include <vector>
+
+#include "lcsa.h"
+#include "lcsa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+lcsa_status_t fail(lcsa_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+lcsa_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(LCSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct Resolved {
+  lcsa_geometry_t geo;
+  lcsa::Grid grid;
+  int radius;          // -1: unbounded
+  int sort_n;
+  std::vector<int32_t> row_ptr;
+  float scale;
+};
+
+// Budget in blocks: topk_ratio = sparse_ratio * 768 * 1280 / (H * W) with the
+// pixel size H = 16 grid_h, W = 16 grid_w ("FlashVSR Inference" skill,
+// Non-Negotiable Streaming Contract), times the blocks of one latent frame.
+int budget_from_ratio(double sparse_ratio, int gh, int gw, int64_t blocks_per_frame) {
+  const double pixels = (16.0 * gh) * (16.0 * gw);
+  return int(std::floor(sparse_ratio * 983040.0 * double(blocks_per_frame) / pixels));
+}
+
+lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
+  if (!c) return fail(LCSA_ERR_INVALID_ARG, "config is null");
+  if (c->batch < 1 || c->heads < 1 || c->head_dim < 1 || c->q_frames < 1 || c->kv_frames < 1 || c->grid_h < 1 ||
+      c->grid_w < 1 || c->block_t < 1 || c->block_h < 1 || c->block_w < 1)
+    return fail(LCSA_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (c->local_range < 0 || (c->local_range != LCSA_UNBOUNDED && c->local_range % 2 == 0))
+    return fail(LCSA_ERR_INVALID_ARG, "local_range %d must be odd (a centred window diameter) or 0 (unbounded)",
+                c->local_range);
+  if (c->topk < 0) return fail(LCSA_ERR_INVALID_ARG, "topk %d < 0", c->topk);
+  if (c->topk == 0 && !(c->sparse_ratio > 0.f))
+    return fail(LCSA_ERR_INVALID_ARG, "topk = 0 needs sparse_ratio > 0");
+  if (c->norm_scope != LCSA_NORM_TOKEN && c->norm_scope != LCSA_NORM_HEAD)
+    return fail(LCSA_ERR_INVALID_ARG, "norm_scope %d", c->norm_scope);
+  if (!(c->rms_eps > 0.f)) return fail(LCSA_ERR_INVALID_ARG, "rms_eps must be > 0");
+  if (!(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale))
+    return fail(LCSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (c->kv_frame_offset < 0) return fail(LCSA_ERR_INVALID_ARG, "kv_frame_offset < 0");
+  if (c->kv_frames < c->q_frames)
+    return fail(LCSA_ERR_SHAPE, "kv_frames %d < q_frames %d (queries are the last frames of the KV window)",
+                c->kv_frames, c->q_frames);
+  if (c->grid_h % c->block_h || c->grid_w % c->block_w || c->q_frames % c->block_t || c->kv_frames % c->block_t)
+    return fail(LCSA_ERR_SHAPE, "token grid %dx%dx%d (q %d) not divisible by block %dx%dx%d", c->kv_frames,
+                c->grid_h, c->grid_w, c->q_frames, c->block_t, c->block_h, c->block_w);
+  if (c->head_dim != lcsa::kHeadDim) return fail(LCSA_ERR_UNSUPPORTED, "head_dim %d (only 128)", c->head_dim);
+  if (c->heads > lcsa::kMaxHeads) return fail(LCSA_ERR_UNSUPPORTED, "heads %d > %d", c->heads, lcsa::kMaxHeads);
+  const int nb = c->block_t * c->block_h * c->block_w;
+  if (nb != 64 && nb != 128) return fail(LCSA_ERR_UNSUPPORTED, "block of %d tokens (64 or 128)", nb);
+  if (c->block_t * c->block_h > 8)
+    return fail(LCSA_ERR_UNSUPPORTED, "block_t*block_h = %d > 8 token rows", c->block_t * c->block_h);
+
+  lcsa::Grid& g = r->grid;
+  g.B = c->batch;
+  g.Hn = c->heads;
+  g.Tq = c->q_frames;
+  g.Tkv = c->kv_frames;
+  g.gh = c->grid_h;
+  g.gw = c->grid_w;
+  g.bt = c->block_t;
+  g.bh = c->block_h;
+  g.bw = c->block_w;
+  g.nb = nb;
+  g.nHb = c->grid_h / c->block_h;
+  g.nWb = c->grid_w / c->block_w;
+  g.bpf = g.nHb * g.nWb;
+  g.nQB = (c->q_frames / c->block_t) * g.bpf;
+  g.nKB = (c->kv_frames / c->block_t) * g.bpf;
+  g.Lq = int64_t(c->q_frames) * c->grid_h * c->grid_w;
+  g.Lkv = int64_t(c->kv_frames) * c->grid_h * c->grid_w;
+  g.C = c->heads * c->head_dim;
+
+  const int64_t elems = int64_t(c->batch) * g.Lkv * g.C;
+  if (elems > (int64_t(1) << 40)) return fail(LCSA_ERR_UNSUPPORTED, "tensor of %lld elements", (long long)elems);
+  const int64_t rows = int64_t(g.B) * g.Hn * g.nQB;
+  if (rows > (int64_t(1) << 30)) return fail(LCSA_ERR_UNSUPPORTED, "%lld rows", (long long)rows);
+
+  int topk = c->topk;
+  if (topk == 0) {
+    topk = budget_from_ratio(double(c->sparse_ratio), c->grid_h, c->grid_w, g.bpf);
+    if (topk < 1)
+      return fail(LCSA_ERR_INVALID_ARG, "sparse_ratio %g gives a budget of %d blocks", double(c->sparse_ratio), topk);
+  }
+  r->radius = c->local_range == LCSA_UNBOUNDED ? -1 : (c->local_range - 1) / 2;
+
+  // admissible-set size per query block: frame groups x clipped window
+  const int groups = g.nKB / g.bpf;
+  auto span = [](int center, int rad, int n) {
+    if (rad < 0) return n;
+    const int lo = center - rad < 0 ? 0 : center - rad;
+    const int hi = center + rad > n - 1 ? n - 1 : center + rad;
+    return hi - lo + 1;
+  };
+  int wmin = 1 << 30, wmax = 0;
+  int64_t nnz_per_head = 0;
+  std::vector<int32_t> keff(g.nQB);
+  for (int qb = 0; qb < g.nQB; ++qb) {
+    const int rem = qb % g.bpf;
+    const int a = groups * span(rem / g.nWb, r->radius, g.nHb) * span(rem % g.nWb, r->radius, g.nWb);
+    wmin = a < wmin ? a : wmin;
+    wmax = a > wmax ? a : wmax;
+    keff[qb] = topk < a ? topk : a;
+    nnz_per_head += keff[qb];
+  }
+  if (wmax > lcsa::kMaxCandidates)
+    return fail(LCSA_ERR_UNSUPPORTED, "window holds %d blocks (> %d)", wmax, lcsa::kMaxCandidates);
+  int sort_n = 32;
+  while (sort_n < wmax) sort_n <<= 1;
+  r->sort_n = sort_n;
+
+  const int64_t nnz = nnz_per_head * g.B * g.Hn;
+  if (nnz > (int64_t(1) << 31) - 1) return fail(LCSA_ERR_UNSUPPORTED, "%lld kept blocks", (long long)nnz);
+  if (want_rows) {
+    r->row_ptr.assign(size_t(rows) + 1, 0);
+    int64_t acc = 0;
+    for (int64_t row = 0; row < rows; ++row) {
+      r->row_ptr[size_t(row)] = int32_t(acc);
+      acc += keff[size_t(row % g.nQB)];
+    }
+    r->row_ptr[size_t(rows)] = int32_t(acc);
+  }
+  r->scale = c->softmax_scale > 0.f ? c->softmax_scale : float(1.0 / std::sqrt(double(c->head_dim)));
+
+  lcsa_geometry_t& o = r->geo;
+  std::memset(&o, 0, sizeof(o));
+  o.q_tokens = g.Lq;
+  o.kv_tokens = g.Lkv;
+  o.channels = g.C;
+  o.block_tokens = nb;
+  o.blocks_per_frame = g.bpf;
+  o.q_blocks = g.nQB;
+  o.kv_blocks = g.nKB;
+  o.rows = rows;
+  o.nnz = nnz;
+  o.topk = topk;
+  o.window_radius = r->radius;
+  o.min_window = wmin;
+  o.max_window = wmax;
+  o.selected_flops = double(nnz) * 4.0 * double(nb) * double(nb) * double(c->head_dim);
+  const double act = 2.0 * double(g.C);  // bytes of one bf16 token vector
+  o.prologue_bytes = 2.0 * act * double(g.B) * double(g.Lq + g.Lkv);
+  // q^ read once, out written once, each (b, h, kept-anywhere) K/V block once
+  o.attention_min_bytes = act * double(g.B) * double(2 * g.Lq + 2 * g.Lkv);
+  const lcsa::RopeSplit rs = lcsa::rope_split(c->head_dim);
+  const size_t rope_n = size_t(g.Tkv) * rs.pairs_t + size_t(g.gh) * rs.pairs_h + size_t(g.gw) * rs.pairs_w;
+  size_t ws = 0;
+  ws += size_t(g.B) * g.Lq * g.C * 2 + size_t(g.B) * g.Lkv * g.C * 2;            // q^, k^
+  ws += size_t(g.B) * g.Hn * (g.nQB + g.nKB) * size_t(c->head_dim) * 4;         // pooled
+  ws += (size_t(rows) + 1) * 4 + size_t(nnz) * 4;                                // CSR
+  ws += rope_n * sizeof(float2) + 256;
+  if (c->host_io)
+    ws += size_t(g.B) * (2 * g.Lq + 2 * g.Lkv) * g.C * 2 + size_t(2) * g.C * 4;
+  o.workspace_bytes = ws;
+  return LCSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct lcsa_plan {
+  lcsa_config_t cfg;
+  Resolved res;
+  int device = 0;
+  __nv_bfloat16* qhat = nullptr;
+  __nv_bfloat16* khat = nullptr;
+  float* pooled_q = nullptr;
+  float* pooled_k = nullptr;
+  int32_t* row_ptr = nullptr;
+  int32_t* col_idx = nullptr;
+  float2* rope = nullptr;
+  int rope_h_off = 0, rope_w_off = 0;
+  unsigned* err = nullptr;
+  // host-IO staging
+  void* st_q = nullptr;
+  void* st_k = nullptr;
+  void* st_v = nullptr;
+  void* st_out = nullptr;
+  float* st_gq = nullptr;
+  float* st_gk = nullptr;
+  std::vector<std::array<cudaEvent_t, 4>> evsets;  // timing ring
+  int64_t timed = 0;                                // forwards recorded
+};
+
+namespace {
+
+void release(lcsa_plan* p) {
+  void* ptrs[] = {p->qhat, p->khat, p->pooled_q, p->pooled_k, p->row_ptr, p->col_idx, p->rope, p->err,
+                  p->st_q, p->st_k, p->st_v, p->st_out, p->st_gq, p->st_gk};
+  for (void* q : ptrs)
+    if (q) cudaFree(q);
+  for (auto& set : p->evsets)
+    for (auto e : set)
+      if (e) cudaEventDestroy(e);
+  p->evsets.clear();
+}
+
+template <class T>
+lcsa_status_t dev_alloc(T** ptr, size_t bytes, const char* what) {
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(ptr), bytes < 16 ? 16 : bytes);
+  if (e != cudaSuccess) {
+    *ptr = nullptr;
+    cudaGetLastError();
+    return fail(e == cudaErrorMemoryAllocation ? LCSA_ERR_OOM : LCSA_ERR_CUDA, "cudaMalloc(%s, %zu bytes): %s", what,
+                bytes, cudaGetErrorString(e));
+  }
+  return LCSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void lcsa_config_default(lcsa_config_t* c) {
+  if (!c) return;
+  std::memset(c, 0, sizeof(*c));
+  c->batch = 1;
+  c->heads = 12;
+  c->head_dim = 128;
+  c->q_frames = 2;
+  c->kv_frames = 6;
+  c->grid_h = 48;
+  c->grid_w = 80;
+  c->block_t = 1;
+  c->block_h = 8;
+  c->block_w = 16;
+  c->local_range = 11;
+  c->topk = 0;
+  c->sparse_ratio = 2.0f;
+  c->kv_frame_offset = 0;
+  c->norm_scope = LCSA_NORM_TOKEN;
+  c->rms_eps = 1e-6f;
+  c->softmax_scale = 0.f;
+  c->host_io = 0;
+}
+
+lcsa_status_t lcsa_config_resolve(const lcsa_config_t* cfg, lcsa_geometry_t* out) {
+  if (!out) return fail(LCSA_ERR_INVALID_ARG, "geometry output is null");
+  Resolved r;
+  lcsa_status_t st = resolve(cfg, &r, false);
+  if (st == LCSA_OK) *out = r.geo;
+  return st;
+}
+
+lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out) {
+  if (!out) return fail(LCSA_ERR_INVALID_ARG, "plan output is null");
+  *out = nullptr;
+  lcsa_plan* p = new (std::nothrow) lcsa_plan();
+  if (!p) return fail(LCSA_ERR_OOM, "host allocation of the plan");
+  lcsa_status_t st = resolve(cfg, &p->res, true);
+  if (st != LCSA_OK) {
+    delete p;
+    return st;
+  }
+  p->cfg = *cfg;
+  p->device = cuda_device;
+  cudaError_t e = cudaSetDevice(cuda_device);
+  if (e != cudaSuccess) {
+    delete p;
+    cudaGetLastError();
+    return cuda_fail(e, "cudaSetDevice");
+  }
+  const lcsa::Grid& g = p->res.grid;
+  const lcsa::RopeSplit rs = lcsa::rope_split(cfg->head_dim);
+  const size_t rope_n = size_t(g.Tkv) * rs.pairs_t + size_t(g.gh) * rs.pairs_h + size_t(g.gw) * rs.pairs_w;
+  p->rope_h_off = g.Tkv * rs.pairs_t;
+  p->rope_w_off = p->rope_h_off + g.gh * rs.pairs_h;
+  const size_t rows = size_t(p->res.geo.rows), nnz = size_t(p->res.geo.nnz);
+  const size_t D = size_t(cfg->head_dim);
+  if ((st = dev_alloc(&p->qhat, size_t(g.B) * g.Lq * g.C * 2, "q^")) ||
+      (st = dev_alloc(&p->khat, size_t(g.B) * g.Lkv * g.C * 2, "k^")) ||
+      (st = dev_alloc(&p->pooled_q, size_t(g.B) * g.Hn * g.nQB * D * 4, "pooled q")) ||
+      (st = dev_alloc(&p->pooled_k, size_t(g.B) * g.Hn * g.nKB * D * 4, "pooled k")) ||
+      (st = dev_alloc(&p->row_ptr, (rows + 1) * 4, "row_ptr")) ||
+      (st = dev_alloc(&p->col_idx, nnz * 4, "col_idx")) ||
+      (st = dev_alloc(&p->rope, rope_n * sizeof(float2), "rope table")) ||
+      (st = dev_alloc(&p->err, 256, "error word"))) {
+    release(p);
+    delete p;
+    return st;
+  }
+  if (cfg->host_io) {
+    if ((st = dev_alloc(&p->st_q, size_t(g.B) * g.Lq * g.C * 2, "staging q")) ||
+        (st = dev_alloc(&p->st_k, size_t(g.B) * g.Lkv * g.C * 2, "staging k")) ||
+        (st = dev_alloc(&p->st_v, size_t(g.B) * g.Lkv * g.C * 2, "staging v")) ||
+        (st = dev_alloc(&p->st_out, size_t(g.B) * g.Lq * g.C * 2, "staging out")) ||
+        (st = dev_alloc(&p->st_gq, size_t(g.C) * 4, "staging gamma q")) ||
+        (st = dev_alloc(&p->st_gk, size_t(g.C) * 4, "staging gamma k"))) {
+      release(p);
+      delete p;
+      return st;
+    }
+  }
+  if ((e = cudaMemcpy(p->row_ptr, p->res.row_ptr.data(), (rows + 1) * 4, cudaMemcpyHostToDevice)) != cudaSuccess ||
+      (e = cudaMemset(p->err, 0, 256)) != cudaSuccess ||
+      (e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, cfg->head_dim, 0)) !=
+          cudaSuccess ||
+      (e = cudaDeviceSynchronize()) != cudaSuccess) {
+    release(p);
+    delete p;
+    return cuda_fail(e, "plan set-up");
+  }
+  *out = p;
+  return LCSA_OK;
+}
+
+void lcsa_plan_destroy(lcsa_plan_t p) {
+  if (!p) return;
+  cudaSetDevice(p->device);
+  cudaDeviceSynchronize();
+  release(p);
+  delete p;
+}
+
+lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                           const float* gamma_k, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(gamma_q) ||
+      !aligned16(gamma_k))
+    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  const lcsa::Grid& g = p->res.grid;
+
+  lcsa::K1Params k1;
+  k1.g = g;
+  k1.q = static_cast<const __nv_bfloat16*>(q);
+  k1.k = static_cast<const __nv_bfloat16*>(k);
+  k1.gamma_q = gamma_q;
+  k1.gamma_k = gamma_k;
+  k1.qhat = p->qhat;
+  k1.khat = p->khat;
+  k1.pooled_q = p->pooled_q;
+  k1.pooled_k = p->pooled_k;
+  k1.rope = p->rope;
+  k1.rope_h_off = p->rope_h_off;
+  k1.rope_w_off = p->rope_w_off;
+  k1.norm_scope = p->cfg.norm_scope;
+  k1.eps = p->cfg.rms_eps;
+
+  lcsa::K2Params k2;
+  k2.g = g;
+  k2.pooled_q = p->pooled_q;
+  k2.pooled_k = p->pooled_k;
+  k2.row_ptr = p->row_ptr;
+  k2.col_idx = p->col_idx;
+  k2.radius = p->res.radius;
+  k2.topk = p->res.geo.topk;
+  k2.sort_n = p->res.sort_n;
+
+  lcsa::K3Params k3;
+  k3.g = g;
+  k3.qhat = p->qhat;
+  k3.khat = p->khat;
+  k3.v = static_cast<const __nv_bfloat16*>(v);
+  k3.out = static_cast<__nv_bfloat16*>(out);
+  k3.row_ptr = p->row_ptr;
+  k3.col_idx = p->col_idx;
+  k3.scale_log2 = p->res.scale * 1.4426950408889634f;
+  k3.err = p->err;
+
+  cudaEvent_t* ev = nullptr;
+  if (!p->evsets.empty()) ev = p->evsets[size_t(p->timed % int64_t(p->evsets.size()))].data();
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
+  if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
+  if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
+  if ((e = lcsa::launch_attention_mma(k3, s)) != cudaSuccess) return cuda_fail(e, "attention launch");
+  if (ev) {
+    if ((e = cudaEventRecord(ev[3], s)) != cudaSuccess) return cuda_fail(e, "event");
+    ++p->timed;
+  }
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                                const float* gamma_k, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (!p->cfg.host_io) return fail(LCSA_ERR_INVALID_ARG, "plan was created without host_io");
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null host pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  const lcsa::Grid& g = p->res.grid;
+  const size_t qb = size_t(g.B) * g.Lq * g.C * 2, kb = size_t(g.B) * g.Lkv * g.C * 2, gb = size_t(g.C) * 4;
+  if ((e = cudaMemcpyAsync(p->st_q, q, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_k, k, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_gq, gamma_q, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_gk, gamma_k, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e, "host-to-device copy");
+  lcsa_status_t st = lcsa_forward(p, p->st_q, p->st_k, p->st_v, p->st_gq, p->st_gk, p->st_out, stream);
+  if (st != LCSA_OK) return st;
+  if ((e = cudaMemcpyAsync(out, p->st_out, qb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_fail(e, "device-to-host copy");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_plan_geometry(lcsa_plan_t p, lcsa_geometry_t* out) {
+  if (!p || !out) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  *out = p->res.geo;
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_plan_topk(lcsa_plan_t p, int* k_out) {
+  if (!p || !k_out) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  *k_out = p->res.geo.topk;
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_get_selection(lcsa_plan_t p, int32_t* row_ptr, size_t row_ptr_cap, int32_t* col_idx,
+                                 size_t col_idx_cap) {
+  if (!p || !row_ptr || !col_idx) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  const size_t rows = size_t(p->res.geo.rows), nnz = size_t(p->res.geo.nnz);
+  if (row_ptr_cap < rows + 1 || col_idx_cap < nnz)
+    return fail(LCSA_ERR_INVALID_ARG, "capacity %zu/%zu < %zu/%zu", row_ptr_cap, col_idx_cap, rows + 1, nnz);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(row_ptr, p->row_ptr, (rows + 1) * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(col_idx, p->col_idx, nnz * 4, cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? LCSA_OK : cuda_fail(e, "copy selection");
+}
+
+lcsa_status_t lcsa_get_intermediates(lcsa_plan_t p, void* qhat, void* khat, float* pooled_q, float* pooled_k) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  const lcsa::Grid& g = p->res.grid;
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess && qhat) e = cudaMemcpy(qhat, p->qhat, size_t(g.B) * g.Lq * g.C * 2, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && khat) e = cudaMemcpy(khat, p->khat, size_t(g.B) * g.Lkv * g.C * 2, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && pooled_q)
+    e = cudaMemcpy(pooled_q, p->pooled_q, size_t(g.B) * g.Hn * g.nQB * lcsa::kHeadDim * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && pooled_k)
+    e = cudaMemcpy(pooled_k, p->pooled_k, size_t(g.B) * g.Hn * g.nKB * lcsa::kHeadDim * 4, cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? LCSA_OK : cuda_fail(e, "copy intermediates");
+}
+
+lcsa_status_t lcsa_check_device_error(lcsa_plan_t p, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
+  unsigned word[4] = {0, 0, 0, 0};
+  if ((e = cudaMemcpy(word, p->err, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read error word");
+  if (word[0] == lcsa::kDevErrNone) return LCSA_OK;
+  cudaMemset(p->err, 0, 256);
+  if (word[0] == lcsa::kDevErrTimeout)
+    return fail(LCSA_ERR_DEVICE_TIMEOUT, "kernel gave up a bounded wait (site %u, block %u)", word[1], word[2]);
+  return fail(LCSA_ERR_DEVICE_BOUNDS, "kernel index check failed (site %u, value %u)", word[1], word[2]);
+}
+
+lcsa_status_t lcsa_plan_set_timing(lcsa_plan_t p, int capacity) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (capacity < 0 || capacity > (1 << 16)) return fail(LCSA_ERR_INVALID_ARG, "timing capacity %d", capacity);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  for (auto& set : p->evsets)
+    for (auto ev : set) cudaEventDestroy(ev);
+  p->evsets.clear();
+  p->timed = 0;
+  for (int i = 0; i < capacity; ++i) {
+    std::array<cudaEvent_t, 4> set{};
+    for (auto& ev : set) {
+      if ((e = cudaEventCreate(&ev)) != cudaSuccess) {
+        p->evsets.push_back(set);
+        return cuda_fail(e, "cudaEventCreate");
+      }
+    }
+    p->evsets.push_back(set);
+  }
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_get_kernel_times(lcsa_plan_t p, float ms[3], int* count) {
+  if (!p || !ms) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  if (p->evsets.empty() || p->timed == 0) return fail(LCSA_ERR_INVALID_ARG, "no timed forward recorded");
+  const int64_t cap = int64_t(p->evsets.size());
+  const int64_t n = p->timed < cap ? p->timed : cap;
+  cudaError_t e = cudaEventSynchronize(p->evsets[size_t((p->timed - 1) % cap)][3]);
+  double acc[3] = {0, 0, 0};
+  for (int64_t i = 0; i < n && e == cudaSuccess; ++i) {
+    const auto& set = p->evsets[size_t((p->timed - 1 - i) % cap)];
+    for (int k = 0; k < 3 && e == cudaSuccess; ++k) {
+      float t = 0.f;
+      e = cudaEventElapsedTime(&t, set[k], set[k + 1]);
+      acc[k] += t;
+    }
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "event timing");
+  for (int k = 0; k < 3; ++k) ms[k] = float(acc[k] / double(n));
+  if (count) *count = int(n);
+  return LCSA_OK;
+}
+
+const char* lcsa_status_string(lcsa_status_t s) {
+  switch (s) {
+    case LCSA_OK: return "LCSA_OK";
+    case LCSA_ERR_INVALID_ARG: return "LCSA_ERR_INVALID_ARG";
+    case LCSA_ERR_SHAPE: return "LCSA_ERR_SHAPE";
+    case LCSA_ERR_ALIGNMENT: return "LCSA_ERR_ALIGNMENT";
+    case LCSA_ERR_UNSUPPORTED: return "LCSA_ERR_UNSUPPORTED";
+    case LCSA_ERR_OOM: return "LCSA_ERR_OOM";
+    case LCSA_ERR_CUDA: return "LCSA_ERR_CUDA";
+    case LCSA_ERR_DEVICE_TIMEOUT: return "LCSA_ERR_DEVICE_TIMEOUT";
+    case LCSA_ERR_DEVICE_BOUNDS: return "LCSA_ERR_DEVICE_BOUNDS";
+  }
+  return "LCSA_ERR_UNKNOWN";
+}
+
+const char* lcsa_last_error_message(void) { return g_last_error.c_str(); }
+
+int lcsa_abi_version(void) { return LCSA_ABI_VERSION; }
+
+}  // extern "C"

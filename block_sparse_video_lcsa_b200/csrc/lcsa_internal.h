@@ -1,0 +1,96 @@
+// Internal interface between the host side of liblcsa (plan, validation,
+// launches) and the three kernels. Not installed; the public ABI is lcsa.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lcsa {
+
+constexpr int kHeadDim = 128;        // the only head size the kernels implement
+constexpr int kMaxHeads = 16;
+constexpr int kMaxCandidates = 4096; // admissible blocks per query block (K2 sort)
+
+// Device error word codes (first word of the plan's error buffer).
+constexpr unsigned kDevErrNone = 0;
+constexpr unsigned kDevErrTimeout = 1;
+constexpr unsigned kDevErrBounds = 2;
+
+// Factored 3D RoPE split of a head: pairs [0, pairs_t) follow the frame,
+// [pairs_t, pairs_t + pairs_h) the token row, the rest the token column.
+struct RopeSplit {
+  int pairs_t, pairs_h, pairs_w;
+  int dims_t, dims_h, dims_w;
+};
+inline RopeSplit rope_split(int d) {
+  RopeSplit s;
+  s.dims_h = 2 * (d / 6);
+  s.dims_w = 2 * (d / 6);
+  s.dims_t = d - s.dims_h - s.dims_w;
+  s.pairs_t = s.dims_t / 2;
+  s.pairs_h = s.dims_h / 2;
+  s.pairs_w = s.dims_w / 2;
+  return s;
+}
+
+// Geometry shared by all kernels (token grid, blocks, window).
+struct Grid {
+  int B, Hn;            // batch, heads
+  int Tq, Tkv;          // query / KV frames
+  int gh, gw;           // token grid per frame
+  int bt, bh, bw;       // block shape
+  int nb;               // tokens per block
+  int nHb, nWb, bpf;    // block rows / columns / blocks per frame group
+  int nQB, nKB;         // blocks per (batch, head)
+  int64_t Lq, Lkv;      // tokens per batch element
+  int C;                // heads * head_dim
+};
+
+struct K1Params {
+  Grid g;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const float* gamma_q;
+  const float* gamma_k;
+  __nv_bfloat16* qhat;  // [B][Hn][nQB][nb][d]
+  __nv_bfloat16* khat;  // [B][Hn][nKB][nb][d]
+  float* pooled_q;      // [B][Hn][nQB][d]
+  float* pooled_k;      // [B][Hn][nKB][d]
+  const float2* rope;   // cos/sin: [Tkv][pairs_t], [gh][pairs_h], [gw][pairs_w]
+  int rope_h_off, rope_w_off;  // float2 offsets of the row and column tables
+  int norm_scope;       // 0 token, 1 head
+  float eps;
+};
+
+struct K2Params {
+  Grid g;
+  const float* pooled_q;
+  const float* pooled_k;
+  const int* row_ptr;   // [rows + 1]
+  int* col_idx;         // [nnz]
+  int radius;           // window radius in blocks, < 0 when unbounded
+  int topk;
+  int sort_n;           // power of two >= the largest admissible set
+};
+
+struct K3Params {
+  Grid g;
+  const __nv_bfloat16* qhat;
+  const __nv_bfloat16* khat;
+  const __nv_bfloat16* v;   // raster [B][Lkv][C]
+  __nv_bfloat16* out;       // raster [B][Lq][C]
+  const int* row_ptr;
+  const int* col_idx;
+  float scale_log2;         // softmax scale * log2(e)
+  unsigned* err;
+};
+
+// Launchers (return the launch's cudaError_t).
+cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, int d, cudaStream_t s);
+cudaError_t launch_prologue(const K1Params& p, cudaStream_t s);
+size_t select_smem_bytes(int sort_n);
+cudaError_t launch_select(const K2Params& p, cudaStream_t s);
+cudaError_t launch_attention_mma(const K3Params& p, cudaStream_t s);
+
+}  // namespace lcsa

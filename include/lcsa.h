@@ -1,0 +1,209 @@
+/*
+ * lcsa.h - C ABI of liblcsa.so, a B200 (sm_100a) implementation of the
+ * locality-constrained sparse attention (LCSA) call of FlashVSR's streaming
+ * video DiT.
+ *
+ * What one call computes (sources are page title + section):
+ *   For every batch b, head h and query block qb of a T x H' x W' latent token
+ *   grid (12 heads, head_dim 128, QK-norm with a norm that spans the heads of a
+ *   token, factored 3D RoPE: "Add FlashVSR contrib model ... on Neuron", Model
+ *   Information and Additional Information):
+ *     1. q^, k^ = RoPE3D(RMSNorm(x) * gamma)               (prologue)
+ *     2. pooled block means of q^ and k^                     (prologue)
+ *     3. score = pooled_q . pooled_k, restricted to the KV blocks inside the
+ *        local window, keep the best k blocks, ties to the lower block index,
+ *        emitted as a CSR list ("FlashVSR: From 17.2 FPS to 57.3 FPS at
+ *        768x1408", What Was Actually Slow and Rebuild sparse attention for
+ *        Hopper: pooling, mask selection, fused CSR construction)
+ *     4. out = softmax(q^ k^T * scale) v over the tokens of the kept blocks
+ *        (block-sparse flash attention, same section).
+ *   Parameters follow the "FlashVSR Inference" skill, Non-Negotiable Streaming
+ *   Contract: local_range 11 or 9, KV window = kv_ratio (3.0) x query frames,
+ *   topk_ratio = sparse_ratio * 768 * 1280 / (H * W), sizes divisible by 128,
+ *   bf16 tensors; and "FlashVSR - Real-Time Diffusion-Based Video
+ *   Super-Resolution", How it works: attention limited to local patches.
+ *
+ * Readings where the pages are silent: the RMSNorm spans heads*head_dim
+ * (LCSA_NORM_TOKEN; LCSA_NORM_HEAD is offered), eps 1e-6; RoPE rotates pairs
+ * (2i, 2i+1), first d-4*(d/6) dims by frame, next 2*(d/6) by token row, last
+ * 2*(d/6) by token column, pair j of an n-dim axis turning by
+ * pos * 10000^(-2j/n); the block score is the raw dot product of block means;
+ * local_range is an odd window diameter in blocks applied as a Chebyshev
+ * distance over (block row, block column), clipped at the frame edge and the
+ * same in every frame of the KV window; the budget in blocks is
+ * k = floor(topk_ratio * blocks per latent frame) with H = 16 H', W = 16 W';
+ * query frames are the last q_frames of the KV window.
+ *
+ * Layouts (all row-major, no padding):
+ *   q    bf16 [batch][q_frames*grid_h*grid_w][heads*head_dim]   (device)
+ *   k, v bf16 [batch][kv_frames*grid_h*grid_w][heads*head_dim]  (device)
+ *   out  bf16 [batch][q_frames*grid_h*grid_w][heads*head_dim]   (device)
+ *   gamma_q, gamma_k fp32 [heads*head_dim]                      (device)
+ *   Token index inside a frame group is raster: (t*grid_h + y)*grid_w + x.
+ *   Blocks are numbered (frame group, block row, block column); tokens in a
+ *   block (frame, row, column). CSR rows are numbered (b, h, qb), qb fastest.
+ *
+ * Ownership: the caller owns q, k, v, gains and out. The plan owns every
+ * intermediate (normalised q^/k^, pooled values, CSR, RoPE table, error word,
+ * optional host-IO staging), all allocated in lcsa_plan_create and freed in
+ * lcsa_plan_destroy. lcsa_forward allocates nothing, is asynchronous on the
+ * given stream and must not run concurrently with another call on the same
+ * plan (the intermediates are shared).
+ *
+ * Errors: every entry point returns a status; none aborts, throws or falls
+ * back to another implementation. lcsa_last_error_message() gives a one-line
+ * detail for the calling thread. Failures inside a kernel set the plan's
+ * device error word, read by lcsa_check_device_error.
+ */
+#ifndef LCSA_H
+#define LCSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCSA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define LCSA_API __attribute__((visibility("default")))
+#else
+#define LCSA_API
+#endif
+
+typedef enum {
+  LCSA_OK = 0,
+  LCSA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, even local_range ... */
+  LCSA_ERR_SHAPE = 2,           /* grid not divisible by the block, kv_frames < q_frames ... */
+  LCSA_ERR_ALIGNMENT = 3,       /* a tensor pointer is not 16-byte aligned */
+  LCSA_ERR_UNSUPPORTED = 4,     /* valid but outside what the kernels implement */
+  LCSA_ERR_OOM = 5,             /* device allocation failed in lcsa_plan_create */
+  LCSA_ERR_CUDA = 6,            /* a CUDA runtime call failed (no device, launch error) */
+  LCSA_ERR_DEVICE_TIMEOUT = 7,  /* a kernel gave up a bounded wait */
+  LCSA_ERR_DEVICE_BOUNDS = 8    /* a kernel found an index outside its buffers */
+} lcsa_status_t;
+
+#define LCSA_UNBOUNDED 0        /* local_range value that disables the window */
+#define LCSA_NORM_TOKEN 0       /* RMSNorm over heads*head_dim of a token */
+#define LCSA_NORM_HEAD 1        /* RMSNorm over head_dim of each head */
+
+typedef struct lcsa_config {
+  int batch;            /* >= 1 */
+  int heads;            /* 1 .. 16 */
+  int head_dim;         /* 128 */
+  int q_frames;         /* >= 1; the last q_frames of the KV window */
+  int kv_frames;        /* >= q_frames (equal: self-attention over the chunk) */
+  int grid_h, grid_w;   /* latent token grid per frame (H' = H/16, W' = W/16) */
+  int block_t, block_h, block_w;  /* block shape; tokens per block must be 64 or 128,
+                                     block_t*block_h <= 8 */
+  int local_range;      /* odd window diameter in blocks, or LCSA_UNBOUNDED */
+  int topk;             /* > 0: budget in blocks; 0: derive from sparse_ratio */
+  float sparse_ratio;   /* used when topk == 0 (1.5 or 2.0 on the pages) */
+  int kv_frame_offset;  /* absolute latent frame index of KV frame 0 (RoPE) */
+  int norm_scope;       /* LCSA_NORM_TOKEN or LCSA_NORM_HEAD */
+  float rms_eps;        /* > 0 */
+  float softmax_scale;  /* 0: 1/sqrt(head_dim) */
+  int host_io;          /* 1: also allocate device staging for lcsa_forward_host */
+} lcsa_config_t;
+
+/* Sizes derived from a configuration (host-side, no device needed). */
+typedef struct lcsa_geometry {
+  int64_t q_tokens, kv_tokens;       /* per batch element */
+  int64_t channels;                  /* heads*head_dim */
+  int64_t block_tokens;              /* n_b */
+  int64_t blocks_per_frame;          /* per frame group */
+  int64_t q_blocks, kv_blocks;       /* per batch and head */
+  int64_t rows;                      /* batch*heads*q_blocks */
+  int64_t nnz;                       /* total kept blocks over all rows */
+  int topk;                          /* resolved budget in blocks */
+  int window_radius;                 /* r = (local_range-1)/2, -1 when unbounded */
+  int min_window, max_window;        /* smallest / largest admissible-set size */
+  double selected_flops;             /* sum over rows of kept * 4 * n_b^2 * head_dim */
+  double prologue_bytes;             /* bytes the prologue must move (q,k in; q^,k^ out) */
+  double attention_min_bytes;        /* q^ + out + each touched k^/v block once */
+  size_t workspace_bytes;            /* device bytes the plan allocates */
+} lcsa_geometry_t;
+
+typedef struct lcsa_plan* lcsa_plan_t;
+
+/* Fill *cfg with the stream-chunk defaults (12 heads, d 128, 2 of 6 frames,
+   48x80 grid, 1x8x16 blocks, local_range 11, sparse_ratio 2.0, eps 1e-6). */
+LCSA_API void lcsa_config_default(lcsa_config_t* cfg);
+
+/* Validate *cfg and derive its sizes. Host only: touches no device.
+   Returns LCSA_ERR_INVALID_ARG / SHAPE / UNSUPPORTED on a bad config. */
+LCSA_API lcsa_status_t lcsa_config_resolve(const lcsa_config_t* cfg, lcsa_geometry_t* out);
+
+/* Validate, then allocate every intermediate on `cuda_device` and build the
+   constant tables. *out is set only on LCSA_OK. */
+LCSA_API lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out);
+
+/* Free everything the plan owns (synchronises the device). Null is a no-op. */
+LCSA_API void lcsa_plan_destroy(lcsa_plan_t plan);
+
+/* One LCSA call: prologue, block selection and block-sparse attention,
+   launched on `stream` (a cudaStream_t; null = legacy default stream).
+   q, k, v, out: device bf16 as laid out above, 16-byte aligned. gamma_q,
+   gamma_k: device fp32 [heads*head_dim], 16-byte aligned. Asynchronous. */
+LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void* k, const void* v,
+                           const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
+/* Same call from HOST buffers: copies q, k, v and the gains into plan-owned
+   device staging, runs lcsa_forward and copies out back, all on `stream`.
+   Needs a plan created with host_io = 1. Host buffers should be pinned for
+   asynchronous copies; the call returns once `out` holds the result. */
+LCSA_API lcsa_status_t lcsa_forward_host(lcsa_plan_t plan, const void* q, const void* k, const void* v,
+                                const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
+/* Resolved geometry of a plan. */
+LCSA_API lcsa_status_t lcsa_plan_geometry(lcsa_plan_t plan, lcsa_geometry_t* out);
+
+/* Resolved budget k in blocks. */
+LCSA_API lcsa_status_t lcsa_plan_topk(lcsa_plan_t plan, int* k_out);
+
+/* Copy the last call's CSR to host: row_ptr [rows+1], col_idx [nnz]. The
+   capacities are element counts; too small -> LCSA_ERR_INVALID_ARG.
+   Synchronises the device. */
+LCSA_API lcsa_status_t lcsa_get_selection(lcsa_plan_t plan, int32_t* row_ptr, size_t row_ptr_cap,
+                                 int32_t* col_idx, size_t col_idx_cap);
+
+/* Copy the last call's prologue outputs to host (any pointer may be null):
+   qhat bf16 [batch][heads][q_blocks][n_b][head_dim], khat likewise with
+   kv_blocks, pooled_q fp32 [batch][heads][q_blocks][head_dim], pooled_k
+   likewise. Synchronises the device. */
+LCSA_API lcsa_status_t lcsa_get_intermediates(lcsa_plan_t plan, void* qhat, void* khat, float* pooled_q,
+                                     float* pooled_k);
+
+/* Synchronise `stream`, then read and clear the plan's device error word:
+   LCSA_OK, LCSA_ERR_DEVICE_TIMEOUT or LCSA_ERR_DEVICE_BOUNDS (or
+   LCSA_ERR_CUDA if the stream itself failed). */
+LCSA_API lcsa_status_t lcsa_check_device_error(lcsa_plan_t plan, void* stream);
+
+/* Kernel timing. capacity > 0: create `capacity` sets of CUDA events and,
+   from now on, record one set around the three kernels of every lcsa_forward
+   (the ring wraps after `capacity` calls); capacity = 0: stop recording and
+   free the events. Any call resets what was recorded so far. */
+LCSA_API lcsa_status_t lcsa_plan_set_timing(lcsa_plan_t plan, int capacity);
+
+/* Mean device milliseconds of the three kernels (ms[0] prologue, ms[1]
+   select, ms[2] attention) over the forwards recorded since the last
+   lcsa_plan_set_timing (at most `capacity` most recent); *count receives how
+   many were averaged. Synchronises on the newest recorded event. */
+LCSA_API lcsa_status_t lcsa_get_kernel_times(lcsa_plan_t plan, float ms[3], int* count);
+
+/* Static text of a status code. */
+LCSA_API const char* lcsa_status_string(lcsa_status_t status);
+
+/* Detail of the last failure on the calling thread ("" if none). */
+LCSA_API const char* lcsa_last_error_message(void);
+
+/* LCSA_ABI_VERSION of the loaded library. */
+LCSA_API int lcsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCSA_H */

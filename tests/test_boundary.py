@@ -1,0 +1,143 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, resolves the measured workloads to the geometry the oracle
+derives independently, and maps every bad configuration to its status code
+without aborting."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_video_lcsa_b200 as L
+import oracle
+from block_sparse_video_lcsa_b200 import build as lcsa_build
+from block_sparse_video_lcsa_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    lcsa_build.build()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(lcsa_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = declared_functions()
+    assert len(names) >= 15
+    raw = ctypes.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    bound = {s[0] for s in L.SIGNATURES}
+    assert bound == set(names)
+
+
+def test_abi_version_and_status_strings():
+    assert L.lcsa_abi_version() == 1
+    for code in range(9):
+        assert L.lcsa_status_string(code).startswith("LCSA_")
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_resolved_geometry_matches_the_oracle(name):
+    wl = synth.WORKLOADS[name]
+    geo = L.lcsa_config_resolve(L.config_from_workload(wl))
+    og = oracle.Geometry.from_workload(wl)
+    sizes = oracle.window_sizes(og)
+    assert geo.topk == og.topk
+    assert geo.q_blocks == og.nQB and geo.kv_blocks == og.nKB
+    assert geo.rows == og.rows
+    assert geo.nnz == og.batch * og.heads * int(np.minimum(sizes, og.topk).sum())
+    assert geo.min_window == sizes.min() and geo.max_window == sizes.max()
+    assert geo.selected_flops == geo.nnz * 4 * og.nb * og.nb * og.head_dim
+
+
+def test_stream_chunk_numbers():
+    geo = L.lcsa_config_resolve(L.config_from_workload(synth.WORKLOADS["stream_768x1280"]))
+    assert (geo.q_tokens, geo.kv_tokens, geo.q_blocks, geo.kv_blocks, geo.topk) == (7680, 23040, 60, 180, 60)
+    assert geo.selected_flops == pytest.approx(362.4e9, rel=1e-3)
+
+
+def _cfg(**over):
+    c = L.config_from_workload(synth.WORKLOADS["tiny"])
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(batch=0), L.LCSA_ERR_INVALID_ARG),
+    (dict(heads=-1), L.LCSA_ERR_INVALID_ARG),
+    (dict(local_range=4), L.LCSA_ERR_INVALID_ARG),
+    (dict(local_range=-3), L.LCSA_ERR_INVALID_ARG),
+    (dict(topk=-1), L.LCSA_ERR_INVALID_ARG),
+    (dict(topk=0, sparse_ratio=0.0), L.LCSA_ERR_INVALID_ARG),
+    (dict(topk=0, sparse_ratio=0.001), L.LCSA_ERR_INVALID_ARG),   # budget floors to 0 blocks
+    (dict(norm_scope=2), L.LCSA_ERR_INVALID_ARG),
+    (dict(rms_eps=0.0), L.LCSA_ERR_INVALID_ARG),
+    (dict(softmax_scale=-1.0), L.LCSA_ERR_INVALID_ARG),
+    (dict(kv_frame_offset=-1), L.LCSA_ERR_INVALID_ARG),
+    (dict(q_frames=3), L.LCSA_ERR_SHAPE),                          # more query than KV frames
+    (dict(grid_w=20), L.LCSA_ERR_SHAPE),                           # ragged block column
+    (dict(grid_h=12), L.LCSA_ERR_SHAPE),                           # ragged block row
+    (dict(block_t=2, q_frames=1, kv_frames=2), L.LCSA_ERR_SHAPE),
+    (dict(head_dim=64), L.LCSA_ERR_UNSUPPORTED),
+    (dict(heads=17), L.LCSA_ERR_UNSUPPORTED),
+    (dict(block_w=4), L.LCSA_ERR_UNSUPPORTED),                     # 32-token blocks
+    (dict(block_h=16, block_w=8, grid_h=32), L.LCSA_ERR_UNSUPPORTED),  # 16 token rows per block
+])
+def test_bad_configs_return_their_status(over, code):
+    cfg = _cfg(**over)
+    g = L.lcsa_geometry_t()
+    st = L.lib().lcsa_config_resolve(ctypes.byref(cfg), ctypes.byref(g))
+    assert st == code, L.lcsa_last_error_message()
+    assert L.lcsa_last_error_message() != ""
+    h = ctypes.c_void_p()
+    assert L.lib().lcsa_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == code
+    assert h.value is None
+
+
+def test_window_too_large_for_the_selection_sort():
+    cfg = _cfg(grid_h=8 * 40, grid_w=8 * 40, q_frames=1, kv_frames=3, local_range=0, topk=4)
+    g = L.lcsa_geometry_t()
+    assert L.lib().lcsa_config_resolve(ctypes.byref(cfg), ctypes.byref(g)) == L.LCSA_ERR_UNSUPPORTED
+
+
+def test_null_arguments_never_crash():
+    lib = L.lib()
+    assert lib.lcsa_config_resolve(None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_plan_create(None, 0, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_forward(None, None, None, None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_forward_host(None, None, None, None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_check_device_error(None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_get_selection(None, None, 0, None, 0) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_get_intermediates(None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_plan_set_timing(None, 1) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_get_kernel_times(None, None, None) == L.LCSA_ERR_INVALID_ARG
+    lib.lcsa_plan_destroy(None)
+
+
+def test_default_config_is_the_stream_chunk():
+    c = L.lcsa_config_default()
+    wl = synth.WORKLOADS["stream_768x1280"]
+    for name in ("heads", "head_dim", "q_frames", "kv_frames", "grid_h", "grid_w", "block_t", "block_h", "block_w",
+                 "local_range"):
+        assert getattr(c, name) == getattr(wl, name), name
+    assert c.sparse_ratio == 2.0 and c.topk == 0
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "liblcsa.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(L.LcsaLibraryMissing):
+        L.lib()
