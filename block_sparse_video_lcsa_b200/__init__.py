@@ -77,6 +77,7 @@ SIGNATURES = [
     ("lcsa_plan_destroy", None, [_PLAN]),
     ("lcsa_forward", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_forward_host", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_forward_noalloc", _I, [ctypes.POINTER(lcsa_config_t), _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_plan_geometry", _I, [_PLAN, ctypes.POINTER(lcsa_geometry_t)]),
     ("lcsa_plan_topk", _I, [_PLAN, ctypes.POINTER(_I)]),
     ("lcsa_get_selection", _I, [_PLAN, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t]),
@@ -156,6 +157,17 @@ def lcsa_plan_create(cfg: lcsa_config_t, device: int = 0) -> "Plan":
     h = _PLAN()
     _check(lib().lcsa_plan_create(ctypes.byref(cfg), int(device), ctypes.byref(h)), "lcsa_plan_create")
     return Plan(h, cfg)
+
+
+LCSA_NOALLOC_WORKSPACE_BYTES = 32 << 20
+
+
+def lcsa_forward_noalloc(cfg: lcsa_config_t, q, k, v, gamma_q, gamma_k, out, stream=None) -> int:
+    """Plan-free call for callers that may not allocate device memory: every
+    intermediate lives in the library's static device workspace. Returns the
+    status code (LCSA_ERR_UNSUPPORTED when the problem does not fit)."""
+    return int(lib().lcsa_forward_noalloc(ctypes.byref(cfg), _addr(q), _addr(k), _addr(v), _addr(gamma_q),
+                                          _addr(gamma_k), _addr(out), _stream(stream)))
 
 
 def config_from_workload(wl, **over) -> lcsa_config_t:

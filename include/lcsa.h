@@ -157,6 +157,29 @@ LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void*
 LCSA_API lcsa_status_t lcsa_forward_host(lcsa_plan_t plan, const void* q, const void* k, const void* v,
                                 const float* gamma_q, const float* gamma_k, void* out, void* stream);
 
+/* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
+   Every GPU that loads the library holds this array until the process exits. */
+#define LCSA_NOALLOC_WORKSPACE_BYTES (32u << 20)
+
+/* The LCSA call without a plan and without any allocation, for callers that
+   may not allocate device memory once running (for instance a real-time
+   video pipeline or a plugin whose device memory is fully reserved at start-up,
+   where cudaMalloc/cudaFree would synchronise the device and stall the other
+   streams, or could fail). This entry point has no counterpart in the paper.
+   Arguments are those of lcsa_forward, with the configuration passed directly
+   (host_io must be 0). All intermediates live in one file-scope static device
+   array of LCSA_NOALLOC_WORKSPACE_BYTES; the first call on a device looks up
+   that array's address on the current device, so make the first call before
+   any stream capture. All calls share the array and it keeps the last call's
+   contents: calls that overlap on the GPU race and must be serialised by the
+   caller. Returns LCSA_ERR_UNSUPPORTED when the problem's intermediates do not
+   fit in the array (create a plan instead), and the codes of
+   lcsa_config_resolve for a bad configuration; no detail message is set. No
+   device or host memory is allocated and no allocating library routine is
+   called. Asynchronous on `stream`. */
+LCSA_API lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const void* q, const void* k, const void* v,
+                                            const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
 /* Resolved geometry of a plan. */
 LCSA_API lcsa_status_t lcsa_plan_geometry(lcsa_plan_t plan, lcsa_geometry_t* out);
 

@@ -141,3 +141,12 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(L.LcsaLibraryMissing):
         L.lib()
+
+
+def test_noalloc_entry_point_rejects_before_touching_a_device():
+    big = L.config_from_workload(synth.WORKLOADS["stream_768x1280"])
+    fake = 1 << 20   # never dereferenced: the size check comes first
+    assert L.lcsa_forward_noalloc(big, fake, fake, fake, fake, fake, fake, 0) == L.LCSA_ERR_UNSUPPORTED
+    assert L.lcsa_forward_noalloc(_cfg(local_range=2), fake, fake, fake, fake, fake, fake, 0) == \
+        L.LCSA_ERR_INVALID_ARG
+    assert L.lcsa_forward_noalloc(_cfg(grid_w=20), fake, fake, fake, fake, fake, fake, 0) == L.LCSA_ERR_SHAPE
