@@ -1,0 +1,528 @@
+// K3 (tcgen05 form): block-sparse flash attention over the CSR list with the
+// 5th-generation tensor cores, tensor memory and TMA, for 128-token blocks.
+//
+// Pages: "FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408", Rebuild sparse
+// attention for Hopper: a warp-specialised producer/consumer path with TMA
+// loads, block-sparse attention over a fused CSR list, FFMA-form softmax math,
+// strided IO and zero-copy raster V. This kernel keeps those ideas and maps
+// them onto sm_100a: accumulators live in tensor memory instead of registers,
+// one thread issues the MMAs, and P goes back to tensor memory as the A
+// operand of the P.V product.
+//
+// Persistent: one CTA per SM walks rows (batch, head, query block) r =
+// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (192 threads):
+//   warp 0  TMA producer: Q tile of the row, then K^ / V blocks of its CSR list
+//           (K^ from the block-major prologue output, V straight from the
+//           raster input through a 5-D tensor map: d, head, x, y, frame).
+//   warp 1  MMA issuer (one lane): S = Q K^T into one of two TMEM S buffers,
+//           O += P V with P read from TMEM; also owns the TMEM allocation.
+//   warps 2-5 softmax: thread = query row = TMEM lane. Reads its S row,
+//           online softmax in the exp2 domain (scale folded into log2 e),
+//           writes P as bf16 pairs to TMEM, rescales its O row only when the
+//           running max grew by more than 2^8 (exact: O and the row sum use
+//           the same stale max), and finally normalises and stores O.
+// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,512).
+// Shared memory: Q 32 KB, K^ ring 3 x 32 KB, V ring 2 x 32 KB, all in the
+// 128-byte swizzled layout that TMA writes and the MMA descriptors read.
+//
+// Every wait on an mbarrier is bounded (wall-clock limit); a wait that runs
+// out records LCSA device error "timeout", raises a CTA-wide abort flag and
+// the kernel winds down instead of hanging.
+#include <cuda.h>
+
+#include "lcsa_internal.h"
+
+namespace lcsa {
+namespace {
+
+constexpr int kNB = 128;                    // tokens per query / KV block
+constexpr int kD = 128;                     // head_dim
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr uint32_t kTileBytes = kNB * kD * 2;   // 32 KB
+constexpr uint32_t kHalfBytes = kTileBytes / 2; // 64 columns of a tile
+constexpr int kThreads = 192;
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384, kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kTileBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers, + alignment slack
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t o_done, o_free, mma_drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+struct TcParams {
+  Grid g;
+  const int* row_ptr;
+  const int* col_idx;
+  __nv_bfloat16* out;
+  float scale_log2;
+  unsigned* err;
+  int rows;
+};
+
+// ---- PTX wrappers ---------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `bar` with the given parity. Returns false if
+// the CTA is aborting or the wall-clock limit passed (then records the error).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, unsigned* err,
+                                       unsigned site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        if (atomicCAS(err, kDevErrNone, kDevErrTimeout) == kDevErrNone) {
+          err[1] = site;
+          err[2] = blockIdx.x;
+        }
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            int c4, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], "
+      "[%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: 128-byte swizzle, descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,
+// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M = N = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+#define LCSA_R32(a) \
+  "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), \
+      "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]),   \
+      "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]),  \
+      "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
+#define LCSA_W32(a)                                                                                               \
+  "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]), \
+      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(a[16]), "r"(a[17]), "r"(a[18]), \
+      "r"(a[19]), "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]), "r"(a[24]), "r"(a[25]), "r"(a[26]), "r"(a[27]), \
+      "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
+
+// 32 consecutive TMEM columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : LCSA_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      LCSA_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---- the kernel -----------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  Bars* bars = reinterpret_cast<Bars*>(gbase + kOffBar);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Grid& g = p.g;
+
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bars->q_full), 1);
+    mbar_init(bar(bars->q_empty), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(bars->k_full[s]), 1);
+      mbar_init(bar(bars->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(bars->v_full[s]), 1);
+      mbar_init(bar(bars->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(bars->s_full[s]), 1);
+      mbar_init(bar(bars->s_free[s]), 4);
+      mbar_init(bar(bars->p_full[s]), 4);
+    }
+    mbar_init(bar(bars->o_done), 1);
+    mbar_init(bar(bars->o_free), 4);
+    mbar_init(bar(bars->mma_drain), 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int kv = 0, row_it = 0;
+      bool ok = true;
+      for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+        const int beg = p.row_ptr[rr], n = p.row_ptr[rr + 1] - beg;
+        const int bhh = rr / g.nQB;
+        const int b = bhh / g.Hn, h = bhh % g.Hn;
+        if (row_it > 0) ok = mbar_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1);
+        if (!ok) break;
+        mbar_expect_tx(bar(bars->q_full), kTileBytes);
+        tma_load_2d(base + kOffQ, &tm_q, 0, rr * kNB, bar(bars->q_full));
+        tma_load_2d(base + kOffQ + kHalfBytes, &tm_q, 64, rr * kNB, bar(bars->q_full));
+        for (int j = 0; j < n && ok; ++j, ++kv) {
+          const int kb = p.col_idx[beg + j];
+          const int ks = kv % kKStages, ku = kv / kKStages;
+          if (ku > 0 && !(ok = mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2))) break;
+          const uint32_t kdst = base + kOffK + ks * kTileBytes;
+          mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
+          tma_load_2d(kdst, &tm_k, 0, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
+          tma_load_2d(kdst + kHalfBytes, &tm_k, 64, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
+          const int vs = kv % kVStages, vu = kv / kVStages;
+          if (vu > 0 && !(ok = mbar_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
+          const int tb = kb / g.bpf, rem = kb % g.bpf;
+          const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
+          const uint32_t vdst = base + kOffV + vs * kTileBytes;
+          mbar_expect_tx(bar(bars->v_full[vs]), kTileBytes);
+          tma_load_5d(vdst, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
+          tma_load_5d(vdst + kHalfBytes, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(0), id_pv = idesc_bf16(1);
+      int kv = 0, s_it = 0, pv_it = 0, row_it = 0;
+      bool ok = true, issued = false;
+      for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+        const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+        if (!(ok = mbar_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
+        for (int j = 0; j <= n && ok; ++j) {
+          if (j < n) {
+            const int sb = s_it & 1;
+            if (s_it >= 2 && !(ok = mbar_wait(bar(bars->s_free[sb]), ((s_it >> 1) - 1) & 1, abort, p.err, 11)))
+              break;
+            const int kvj = kv + j, ks = kvj % kKStages;
+            if (!(ok = mbar_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
+            tc_fence_after();
+            const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+              mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
+                     kk > 0 ? 1u : 0u);
+            }
+            issued = true;
+            mma_commit(bar(bars->s_full[sb]));
+            mma_commit(bar(bars->k_empty[ks]));
+            if (j == n - 1) mma_commit(bar(bars->q_empty));
+            ++s_it;
+          }
+          if (j >= 1) {
+            const int i = j - 1, pb = pv_it & 1;
+            if (!(ok = mbar_wait(bar(bars->p_full[pb]), (pv_it >> 1) & 1, abort, p.err, 13))) break;
+            const int kvi = kv + i, vs = kvi % kVStages;
+            if (!(ok = mbar_wait(bar(bars->v_full[vs]), (kvi / kVStages) & 1, abort, p.err, 14))) break;
+            if (i == 0 && row_it > 0 && !(ok = mbar_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
+              break;
+            tc_fence_after();
+            const uint32_t va = base + kOffV + vs * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kNB / 16; ++kk) {
+              mma_ts(tmem + kColO, tmem + kColP + pb * 64 + kk * 8, sdesc(va + kk * 2048, kHalfBytes, 1024), id_pv,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(bars->v_empty[vs]));
+            mma_commit(bar(bars->o_done));
+            ++pv_it;
+          }
+        }
+        kv += n;
+      }
+      if (issued) {
+        mma_commit(bar(bars->mma_drain));
+        mbar_wait(bar(bars->mma_drain), 0, abort, p.err, 16);
+      }
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue ----------------
+    const int sp = warp & 3;                 // TMEM lane quarter of this warp
+    const int row_in_tile = sp * 32 + lane;  // query token index inside the block
+    const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
+    const float c = p.scale_log2;
+    int s_it = 0, pv_wait = 0;
+    bool ok = true;
+    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
+      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n && ok; ++j, ++s_it) {
+        const int sb = s_it & 1;
+        if (!(ok = mbar_wait(bar(bars->s_full[sb]), (s_it >> 1) & 1, abort, p.err, 20))) break;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(lane_addr + kColS + sb * 128 + q4 * 32, sr[q4]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->s_free[sb]));
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[q4][e]));
+        const float m_new = fmaxf(m_used, mx * c);
+        const bool need = m_new > m_used + kRescaleLog2;
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (need) {
+          alpha = exp2f(m_used - m_new);
+          m_used = m_new;
+        }
+        l *= alpha;
+        const float mneg = -m_used;
+        uint32_t pk[2][32];
+        float rs = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = exp2f(fmaf(__uint_as_float(sr[q4][e]), c, mneg));
+            const float p1 = exp2f(fmaf(__uint_as_float(sr[q4][e + 1]), c, mneg));
+            rs += p0 + p1;
+            pk[q4 >> 1][(q4 & 1) * 16 + (e >> 1)] = pack_bf16(p0, p1);
+          }
+        }
+        l += rs;
+        if (j >= 1) {
+          if (!(ok = mbar_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 21))) break;
+          ++pv_wait;
+          tc_fence_after();
+          if (warp_need) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + kColO + q4 * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(lane_addr + kColO + q4 * 32, o);
+            }
+          }
+        }
+        tmem_st32(lane_addr + kColP + sb * 64, pk[0]);
+        tmem_st32(lane_addr + kColP + sb * 64 + 32, pk[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->p_full[sb]));
+      }
+      if (!ok) break;
+      // epilogue: wait for the last P.V, normalise, store the raster output
+      if (!(ok = mbar_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 22))) break;
+      ++pv_wait;
+      tc_fence_after();
+      const int bhh = rr / g.nQB, qb = rr % g.nQB;
+      const int b = bhh / g.Hn, h = bhh % g.Hn;
+      const int tb = qb / g.bpf, rem = qb % g.bpf;
+      const int tt = row_in_tile / (g.bh * g.bw), yy = (row_in_tile / g.bw) % g.bh, xx = row_in_tile % g.bw;
+      const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
+      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD;
+      const float inv = 1.0f / l;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + kColO + q4 * 32, o);
+        tmem_wait_ld();
+        uint4 v[4];
+        uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + q4 * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d4[e] = v[e];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->o_free));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ---- host side ------------------------------------------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool attention_tc_supported(const Grid& g) { return g.nb == kNB; }
+
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows) {
+  EncodeTiled enc = encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(kD * 2)};
+  const cuuint32_t box[2] = {64, cuuint32_t(kNB)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
+  EncodeTiled enc = encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t row = cuuint64_t(g.C) * 2;  // bytes per token
+  const cuuint64_t dims[5] = {cuuint64_t(kD), cuuint64_t(g.Hn), cuuint64_t(g.gw), cuuint64_t(g.gh),
+                              cuuint64_t(g.B) * cuuint64_t(g.Tkv)};
+  const cuuint64_t strides[4] = {cuuint64_t(kD * 2), row, row * cuuint64_t(g.gw), row * cuuint64_t(g.gw) * g.gh};
+  const cuuint32_t box[5] = {64, 1, cuuint32_t(g.bw), cuuint32_t(g.bh), cuuint32_t(g.bt)};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                const CUtensorMap& tm_v, int num_sms, cudaStream_t s) {
+  cudaError_t e =
+      cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  TcParams tp;
+  tp.g = p.g;
+  tp.row_ptr = p.row_ptr;
+  tp.col_idx = p.col_idx;
+  tp.out = p.out;
+  tp.scale_log2 = p.scale_log2;
+  tp.err = p.err;
+  tp.rows = p.g.B * p.g.Hn * p.g.nQB;
+  const int grid = tp.rows < num_sms ? tp.rows : num_sms;
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
+  return cudaGetLastError();
+}
+
+}  // namespace lcsa

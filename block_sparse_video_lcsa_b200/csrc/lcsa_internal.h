@@ -2,6 +2,7 @@
 // launches) and the three kernels. Not installed; the public ABI is lcsa.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -92,5 +93,14 @@ cudaError_t launch_prologue(const K1Params& p, cudaStream_t s);
 size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
 cudaError_t launch_attention_mma(const K3Params& p, cudaStream_t s);
+
+// tcgen05 attention (128-token blocks). Tensor maps: q^ / k^ as [rows][128]
+// bf16 tiles of 128 rows (make_block_map), V through its raster layout
+// (make_raster_map). The kernel is persistent over min(rows, num_sms) CTAs.
+bool attention_tc_supported(const Grid& g);
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows);
+cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g);
+cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                const CUtensorMap& tm_v, int num_sms, cudaStream_t s);
 
 }  // namespace lcsa
