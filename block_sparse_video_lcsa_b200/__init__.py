@@ -85,6 +85,7 @@ SIGNATURES = [
     ("lcsa_check_device_error", _I, [_PLAN, _VP]),
     ("lcsa_plan_set_timing", _I, [_PLAN, _I]),
     ("lcsa_get_kernel_times", _I, [_PLAN, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I)]),
+    ("lcsa_selftest_exp2", _I, [_VP, _VP, _I, _VP]),
     ("lcsa_status_string", ctypes.c_char_p, [_I]),
     ("lcsa_last_error_message", ctypes.c_char_p, []),
     ("lcsa_abi_version", _I, []),
@@ -274,6 +275,12 @@ class Plan:
         n = ctypes.c_int()
         _check(lib().lcsa_get_kernel_times(self._h, ms, ctypes.byref(n)), "lcsa_get_kernel_times")
         return list(ms), n.value
+
+
+def lcsa_selftest_exp2(x, y, stream=None):
+    """y = 2^x through the attention kernel's FMA-pipe exponential (fp32 CUDA tensors)."""
+    _check(lib().lcsa_selftest_exp2(_addr(x), _addr(y), int(x.numel()), _stream(stream)), "lcsa_selftest_exp2")
+    return y
 
 
 def lcsa_status_string(status: int) -> str:

@@ -9,25 +9,22 @@
 // pooling and RoPE as separate glue kernels) and Rebuild sparse attention for
 // Hopper (coalesced RoPE kernel, pooled keys).
 //
-// Work split: a thread-block cluster owns one block of 64 or 128 tokens; each
-// CTA of the cluster owns one token row of that block (block_w tokens), each
-// warp one token at a time. A token's heads*128 bf16 values are read with
-// 16-byte loads, lane l taking 16-byte chunks l, l+32, ... so every load
-// instruction of a warp covers 512 contiguous bytes. The sum of squares is a
-// warp-shuffle reduction; the pooled sums are reduced warp -> CTA in shared
-// memory and CTA -> cluster through distributed shared memory, always in the
-// same order, so the pooled values (and hence the block selection) are
-// deterministic.
-#include <cooperative_groups.h>
-
+// Work split: one CTA of 8 warps owns one block of 64 or 128 tokens; warp w
+// handles tokens w, w+8, ... of the block, loading the next token while it
+// works on the current one. A token's heads*128 bf16 values are read with
+// 16-byte streaming loads, lane l taking 16-byte chunks l, l+32, ... so every
+// load instruction of a warp covers 512 contiguous bytes. The sum of squares
+// is a warp-shuffle reduction; the pooled sums are kept per warp in shared
+// memory (each lane owns its slots) and reduced across the 8 warps in a fixed
+// order, so the pooled values (and hence the block selection) are
+// deterministic. Two CTAs fit on an SM, so a stream chunk's 240 blocks are all
+// resident at once.
 #include "lcsa_internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace lcsa {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 
 __global__ void rope_table_kernel(float2* tab, int Tkv, int gh, int gw, int t0, RopeSplit s) {
@@ -73,16 +70,22 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 
 // CPL = 16-byte chunks per lane per token = ceil(heads * 16 / 32).
 template <int CPL>
-__global__ void __launch_bounds__(kThreads) prologue_kernel(const K1Params p) {
-  extern __shared__ float smem[];
+__device__ __forceinline__ void load_token(const uint4* src, int lane, int nchunks, uint4 (&raw)[CPL]) {
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const int c = i * 32 + lane;
+    raw[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < nchunks) raw[i] = load_stream(src + c);
+  }
+}
+
+template <int CPL>
+__global__ void __launch_bounds__(kThreads, 2) prologue_kernel(const K1Params p) {
+  extern __shared__ float red[];  // [kWarps][C]
   const Grid& g = p.g;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int R = int(cluster.num_blocks());
-  const int rank = int(cluster.block_rank());
-  const int block_global = blockIdx.x / R;
   const int n_qtot = g.B * g.nQB;
-  const bool is_q = block_global < n_qtot;
-  const int bg = is_q ? block_global : block_global - n_qtot;
+  const bool is_q = int(blockIdx.x) < n_qtot;
+  const int bg = is_q ? int(blockIdx.x) : int(blockIdx.x) - n_qtot;
   const int nblk = is_q ? g.nQB : g.nKB;
   const int b = bg / nblk, blk = bg % nblk;
   const __nv_bfloat16* x = is_q ? p.q : p.k;
@@ -93,39 +96,49 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const K1Params p) {
   const int tshift = is_q ? (g.Tkv - g.Tq) : 0;
 
   const int tb = blk / g.bpf, rem = blk % g.bpf;
-  const int hbk = rem / g.nWb, wbk = rem % g.nWb;
-  const int tt = rank / g.bh, yy = rank % g.bh;
-  const int t = tb * g.bt + tt, y = hbk * g.bh + yy;
+  const int t0 = tb * g.bt, y0 = (rem / g.nWb) * g.bh, x0 = (rem % g.nWb) * g.bw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunks = g.C / 8;
+  const int plane = g.bh * g.bw;
   constexpr int PT = 22, PH = 21;  // RoPE pairs on the frame / row axes (head_dim 128)
 
-  float pool[CPL][8];
+  // this lane's pooled partial sums live in its own slots of red[warp][.]
+  float* mine = red + warp * g.C;
 #pragma unroll
-  for (int i = 0; i < CPL; ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) pool[i][e] = 0.f;
+  for (int c4 = 0; c4 < CPL; ++c4) {
+    const int c = c4 * 32 + lane;
+    if (c < nchunks) {
+      reinterpret_cast<float4*>(mine + c * 8)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(mine + c * 8)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+
+  auto token_src = [&](int i, int& t, int& y, int& xc) {
+    t = t0 + i / plane;
+    y = y0 + (i / g.bw) % g.bh;
+    xc = x0 + i % g.bw;
+    const int64_t tok = (int64_t(t) * g.gh + y) * g.gw + xc;
+    return reinterpret_cast<const uint4*>(x + (int64_t(b) * L + tok) * g.C);
+  };
 
   const int jb = 4 * (lane & 15);  // first RoPE pair of this lane (same in every head)
-  for (int xx = warp; xx < g.bw; xx += kWarps) {
-    const int xc = wbk * g.bw + xx;
-    const int64_t tok = (int64_t(t) * g.gh + y) * g.gw + xc;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t(b) * L + tok) * g.C);
+  uint4 nxt[CPL];
+  int nt = 0, ny = 0, nx = 0;
+  if (warp < g.nb) load_token<CPL>(token_src(warp, nt, ny, nx), lane, nchunks, nxt);
+  for (int i = warp; i < g.nb; i += kWarps) {
     uint4 raw[CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int c = i * 32 + lane;
-      raw[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (c < nchunks) raw[i] = load_stream(src + c);
-    }
+    for (int c = 0; c < CPL; ++c) raw[c] = nxt[c];
+    const int t = nt, y = ny, xc = nx;
+    if (i + kWarps < g.nb) load_token<CPL>(token_src(i + kWarps, nt, ny, nx), lane, nchunks, nxt);
     // RMSNorm scale(s)
     float rs[CPL];
     if (p.norm_scope == 0) {
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) {
+      for (int c = 0; c < CPL; ++c) {
         float f[8];
-        unpack8(raw[i], f);
+        unpack8(raw[c], f);
 #pragma unroll
         for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
       }
@@ -133,18 +146,18 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const K1Params p) {
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float r = rsqrtf(ss * (1.0f / float(g.C)) + p.eps);
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) rs[i] = r;
+      for (int c = 0; c < CPL; ++c) rs[c] = r;
     } else {
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) {
+      for (int c = 0; c < CPL; ++c) {
         float f[8];
-        unpack8(raw[i], f);
+        unpack8(raw[c], f);
         float ss = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        rs[i] = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
+        rs[c] = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
       }
     }
     // cos/sin of this lane's four pairs at this token's position
@@ -159,80 +172,55 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const K1Params p) {
       else
         cs[qd] = p.rope[p.rope_w_off + xc * (kHeadDim / 2 - PT - PH) + (j - PT - PH)];
     }
-    const int tokin = (tt * g.bh + yy) * g.bw + xx;
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int c = i * 32 + lane;
+    for (int c4 = 0; c4 < CPL; ++c4) {
+      const int c = c4 * 32 + lane;
       if (c >= nchunks) continue;
       const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma + c * 8));
       const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma + c * 8 + 4));
       const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       float f[8], o[8];
-      unpack8(raw[i], f);
+      unpack8(raw[c4], f);
 #pragma unroll
       for (int qd = 0; qd < 4; ++qd) {
-        const float a = f[2 * qd] * rs[i] * gm[2 * qd];
-        const float bq = f[2 * qd + 1] * rs[i] * gm[2 * qd + 1];
+        const float a = f[2 * qd] * rs[c4] * gm[2 * qd];
+        const float bq = f[2 * qd + 1] * rs[c4] * gm[2 * qd + 1];
         o[2 * qd] = a * cs[qd].x - bq * cs[qd].y;
         o[2 * qd + 1] = a * cs[qd].y + bq * cs[qd].x;
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) pool[i][e] += o[e];
+      float4* acc = reinterpret_cast<float4*>(mine + c * 8);
+      float4 a0 = acc[0], a1 = acc[1];
+      a0.x += o[0]; a0.y += o[1]; a0.z += o[2]; a0.w += o[3];
+      a1.x += o[4]; a1.y += o[5]; a1.z += o[6]; a1.w += o[7];
+      acc[0] = a0;
+      acc[1] = a1;
       const int head = c >> 4, dd = (c & 15) * 8;
       uint4* dst = reinterpret_cast<uint4*>(
-          xhat + (((int64_t(b) * g.Hn + head) * nblk + blk) * g.nb + tokin) * kHeadDim + dd);
+          xhat + (((int64_t(b) * g.Hn + head) * nblk + blk) * g.nb + i) * kHeadDim + dd);
       *dst = pack8(o);
     }
   }
 
-  // warp partials -> shared memory -> CTA partial
-  float* red = smem;                 // [kWarps][C]
-  float* part = smem + kWarps * g.C; // [C]
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    const int c = i * 32 + lane;
-    if (c < nchunks) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[warp * g.C + c * 8 + e] = pool[i][e];
-    }
-  }
+  // warp partials -> block mean, summed over warps in a fixed order
   __syncthreads();
+  const float inv_nb = 1.0f / float(g.nb);
   for (int e = threadIdx.x; e < g.C; e += kThreads) {
     float s = red[e];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) s += red[w * g.C + e];
-    part[e] = s;
-  }
-  cluster.sync();
-  // CTA partials -> block mean, each rank finishing every R-th channel
-  const float inv_nb = 1.0f / float(g.nb);
-  for (int e = rank + R * threadIdx.x; e < g.C; e += R * kThreads) {
-    float s = 0.f;
-    for (int r = 0; r < R; ++r) s += cluster.map_shared_rank(part, r)[e];
     const int head = e / kHeadDim, dd = e % kHeadDim;
     pooled[((int64_t(b) * g.Hn + head) * nblk + blk) * kHeadDim + dd] = s * inv_nb;
   }
-  cluster.sync();  // keep this CTA's shared memory alive until every rank has read it
 }
 
 template <int CPL>
 cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
-  const int R = p.g.bt * p.g.bh;
   const int nblocks = p.g.B * (p.g.nQB + p.g.nKB);
-  const size_t smem = size_t(kWarps + 1) * p.g.C * sizeof(float);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(nblocks * R));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(R);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prologue_kernel<CPL>, p);
+  const size_t smem = size_t(kWarps) * p.g.C * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(prologue_kernel<CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  prologue_kernel<CPL><<<nblocks, kThreads, smem, s>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace

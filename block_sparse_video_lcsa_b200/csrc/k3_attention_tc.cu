@@ -10,20 +10,36 @@
 // operand of the P.V product.
 //
 // Persistent: one CTA per SM walks rows (batch, head, query block) r =
-// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (192 threads):
+// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (320 threads):
 //   warp 0  TMA producer: Q tile of the row, then K^ / V blocks of its CSR list
 //           (K^ from the block-major prologue output, V straight from the
 //           raster input through a 5-D tensor map: d, head, x, y, frame).
-//   warp 1  MMA issuer (one lane): S = Q K^T into one of two TMEM S buffers,
-//           O += P V with P read from TMEM; also owns the TMEM allocation.
-//   warps 2-5 softmax: thread = query row = TMEM lane. Reads its S row,
-//           online softmax in the exp2 domain (scale folded into log2 e),
-//           writes P as bf16 pairs to TMEM, rescales its O row only when the
-//           running max grew by more than 2^8 (exact: O and the row sum use
-//           the same stale max), and finally normalises and stores O.
-// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,512).
-// Shared memory: Q 32 KB, K^ ring 3 x 32 KB, V ring 2 x 32 KB, all in the
-// 128-byte swizzled layout that TMA writes and the MMA descriptors read.
+//   warp 1  MMA issuer (one lane): S = Q K^T into a ring of three TMEM S
+//           buffers, issued two KV blocks ahead of the softmax, and O += P V
+//           with P read from TMEM; also owns the TMEM allocation.
+//   warps 2-9 softmax, two warpgroups: a query row (TMEM lane) is shared by
+//           lane i of warp w and of warp w+4, each owning 64 of its 128 key
+//           columns. The pair trades row maxima (and at the end row sums)
+//           through shared memory, ordered by an mbarrier of 64 arrivals. Online
+//           softmax in the exp2 domain (scale folded into log2 e), P written
+//           to TMEM as bf16 pairs, O rescaled only when the running max grew
+//           by more than 2^8 (exact: O and the row sum use the same stale
+//           max); finally each thread normalises and stores 64 of the row's
+//           output channels. Independent accumulators break the max and sum
+//           chains, and every fourth exponential runs on the FMA pipe
+//           (Cody-Waite reduction 2^x = 2^n 2^f, |f| <= 1/2, and a degree-3
+//           minimax polynomial for 2^f fitted for this kernel, relative
+//           error below 7.5e-5) so the MUFU unit is not the bottleneck (the
+//           pages' "FFMA-form softmax math").
+// TMEM columns: S ring [0,128) [128,256) [256,384), O [384,512). P of block j
+// is written back into S buffer j % 3 (bf16 pairs; keys 0-63 in its columns
+// 0-31, keys 64-127 in columns 64-95, each half inside the columns its own
+// thread has already read). The tensor pipe runs one issuer's MMAs in order,
+// so S of block j+3, issued after P.V of block j, cannot overwrite P_j early.
+// Shared memory: Q 32 KB, K^ ring 2 x 32 KB, V ring 3 x 32 KB, all in the
+// 128-byte swizzled layout that TMA writes and the MMA descriptors read. The
+// producer fetches K^ two blocks ahead of V (K^_{j+2} before V_j), matching
+// the order in which the MMA issuer consumes them.
 //
 // Every wait on an mbarrier is bounded (wall-clock limit); a wait that runs
 // out records LCSA device error "timeout", raises a CTA-wide abort flag and
@@ -37,12 +53,15 @@ namespace {
 
 constexpr int kNB = 128;                    // tokens per query / KV block
 constexpr int kD = 128;                     // head_dim
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;
 constexpr uint32_t kTileBytes = kNB * kD * 2;   // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2; // 64 columns of a tile
-constexpr int kThreads = 192;
-constexpr uint32_t kColS = 0, kColP = 256, kColO = 384, kTmemCols = 512;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kPolyEvery = 4;  // one exponential in kPolyEvery on the FMA pipe
+constexpr int kSBufs = 3;
+constexpr uint32_t kColS = 0, kColO = 384, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -50,18 +69,29 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers, + alignment slack
+constexpr uint32_t kOffXchg = kOffBar + 256;          // row max / sum exchange
+constexpr uint32_t kXchgBytes = (2 * 2 * 128 + 2 * 128) * 4;
+constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
+
+// 2^f on [-1/2, 1/2]: degree-3 minimax coefficients (relative error 7.49e-5),
+// fitted by csrc/fit_exp2_poly.py.
+constexpr float kExp2C0 = 0.9999281167984009f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.24261052906513214f;
+constexpr float kExp2C3 = 0.055171314626932144f;
 
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t s_full[kSBufs], p_full[kSBufs];
   uint64_t o_done, o_free, mma_drain;
+  uint64_t pair[4];  // row max / sum exchange between the two softmax warps of a lane quarter
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(kSoftmaxWarps == 8 && kThreads == 64 + 32 * kSoftmaxWarps, "warp roles");
 
 struct TcParams {
   Grid g;
@@ -207,6 +237,42 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float exp2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x for x <= 8 (Cody-Waite): n = round(x) through the 1.5 * 2^23 shifter,
+// f = x - n, 2^f by the polynomial, 2^n added to the exponent field. Inputs
+// below -125 are clamped (the result, < 2^-124, is negligible next to the
+// row maximum's weight of at least 1).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float shifter = 12582912.0f;
+  const float t = x + shifter;
+  const float n = t - shifter;
+  const float f = x - n;
+  float p = fmaf(kExp2C3, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  const uint32_t ni = __float_as_uint(t) - 0x4B400000u;
+  return __uint_as_float(__float_as_uint(p) + (ni << 23));
+}
+
+// Wait of a whole warp: every lane waits, and the warp fails as one if any
+// lane gave up, so warp-collective instructions never run diverged.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, unsigned* err,
+                                          unsigned site) {
+  const bool ok = mbar_wait(bar, parity, abort, err, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_poly(x[i]);
+}
+
 // ---- the kernel -----------------------------------------------------------
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -234,14 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(bars->v_full[s]), 1);
       mbar_init(bar(bars->v_empty[s]), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(bars->s_full[s]), 1);
-      mbar_init(bar(bars->s_free[s]), 4);
-      mbar_init(bar(bars->p_full[s]), 4);
+      mbar_init(bar(bars->p_full[s]), kSoftmaxWarps);
     }
     mbar_init(bar(bars->o_done), 1);
-    mbar_init(bar(bars->o_free), 4);
+    mbar_init(bar(bars->o_free), kSoftmaxWarps);
     mbar_init(bar(bars->mma_drain), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(bar(bars->pair[s]), 64);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -269,15 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(bar(bars->q_full), kTileBytes);
         tma_load_2d(base + kOffQ, &tm_q, 0, rr * kNB, bar(bars->q_full));
         tma_load_2d(base + kOffQ + kHalfBytes, &tm_q, 64, rr * kNB, bar(bars->q_full));
-        for (int j = 0; j < n && ok; ++j, ++kv) {
+        auto load_k = [&](int j) -> bool {
           const int kb = p.col_idx[beg + j];
-          const int ks = kv % kKStages, ku = kv / kKStages;
-          if (ku > 0 && !(ok = mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2))) break;
+          const int kvj = kv + j, ks = kvj % kKStages, ku = kvj / kKStages;
+          if (ku > 0 && !mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
           const uint32_t kdst = base + kOffK + ks * kTileBytes;
           mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
           tma_load_2d(kdst, &tm_k, 0, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
           tma_load_2d(kdst + kHalfBytes, &tm_k, 64, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
-          const int vs = kv % kVStages, vu = kv / kVStages;
+          return true;
+        };
+        for (int j = 0; j < 2 && j < n && ok; ++j) ok = load_k(j);
+        for (int j = 0; j < n && ok; ++j) {
+          if (j + 2 < n && !(ok = load_k(j + 2))) break;
+          const int kb = p.col_idx[beg + j];
+          const int kvj = kv + j, vs = kvj % kVStages, vu = kvj / kVStages;
           if (vu > 0 && !(ok = mbar_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
           const int tb = kb / g.bpf, rem = kb % g.bpf;
           const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
@@ -286,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_5d(vdst, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
           tma_load_5d(vdst + kHalfBytes, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
         }
+        kv += n;
       }
     }
   } else if (warp == 1) {
@@ -294,48 +367,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_qk = idesc_bf16(0), id_pv = idesc_bf16(1);
       int kv = 0, s_it = 0, pv_it = 0, row_it = 0;
       bool ok = true, issued = false;
+      // S of the row's block j into buffer (s_it % 3)
+      auto issue_s = [&](int j, int n) -> bool {
+        const int sb = s_it % kSBufs;
+        const int kvj = kv + j, ks = kvj % kKStages;
+        if (!mbar_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12)) return false;
+        tc_fence_after();
+        const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
+                 kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        mma_commit(bar(bars->s_full[sb]));
+        mma_commit(bar(bars->k_empty[ks]));
+        if (j == n - 1) mma_commit(bar(bars->q_empty));
+        ++s_it;
+        return true;
+      };
       for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
         const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
         if (!(ok = mbar_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
-        for (int j = 0; j <= n && ok; ++j) {
-          if (j < n) {
-            const int sb = s_it & 1;
-            if (s_it >= 2 && !(ok = mbar_wait(bar(bars->s_free[sb]), ((s_it >> 1) - 1) & 1, abort, p.err, 11)))
-              break;
-            const int kvj = kv + j, ks = kvj % kKStages;
-            if (!(ok = mbar_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
-            tc_fence_after();
-            const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
+        for (int j = 0; j < 2 && j < n && ok; ++j) ok = issue_s(j, n);
+        for (int j = 0; j < n && ok; ++j) {
+          // S two blocks ahead: its buffer last held P of block j-1, whose P.V
+          // was issued in the previous step (in-order pipe)
+          if (j + 2 < n && !(ok = issue_s(j + 2, n))) break;
+          const int pb = pv_it % kSBufs;
+          if (!(ok = mbar_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
+          const int kvi = kv + j, vs = kvi % kVStages;
+          if (!(ok = mbar_wait(bar(bars->v_full[vs]), (kvi / kVStages) & 1, abort, p.err, 14))) break;
+          if (j == 0 && row_it > 0 && !(ok = mbar_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
+            break;
+          tc_fence_after();
+          const uint32_t va = base + kOffV + vs * kTileBytes;
+          const uint32_t pa = tmem + kColS + pb * 128;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-              mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
-                     kk > 0 ? 1u : 0u);
-            }
-            issued = true;
-            mma_commit(bar(bars->s_full[sb]));
-            mma_commit(bar(bars->k_empty[ks]));
-            if (j == n - 1) mma_commit(bar(bars->q_empty));
-            ++s_it;
+          for (int kk = 0; kk < kNB / 16; ++kk) {
+            mma_ts(tmem + kColO, pa + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), sdesc(va + kk * 2048, kHalfBytes, 1024),
+                   id_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
-          if (j >= 1) {
-            const int i = j - 1, pb = pv_it & 1;
-            if (!(ok = mbar_wait(bar(bars->p_full[pb]), (pv_it >> 1) & 1, abort, p.err, 13))) break;
-            const int kvi = kv + i, vs = kvi % kVStages;
-            if (!(ok = mbar_wait(bar(bars->v_full[vs]), (kvi / kVStages) & 1, abort, p.err, 14))) break;
-            if (i == 0 && row_it > 0 && !(ok = mbar_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
-              break;
-            tc_fence_after();
-            const uint32_t va = base + kOffV + vs * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < kNB / 16; ++kk) {
-              mma_ts(tmem + kColO, tmem + kColP + pb * 64 + kk * 8, sdesc(va + kk * 2048, kHalfBytes, 1024), id_pv,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(bar(bars->v_empty[vs]));
-            mma_commit(bar(bars->o_done));
-            ++pv_it;
-          }
+          mma_commit(bar(bars->v_empty[vs]));
+          mma_commit(bar(bars->o_done));
+          ++pv_it;
         }
         kv += n;
       }
@@ -347,105 +423,126 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- softmax / correction / epilogue ----------------
     const int sp = warp & 3;                 // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;        // which 64 key columns / channels
     const int row_in_tile = sp * 32 + lane;  // query token index inside the block
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
+    float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
     const float c = p.scale_log2;
-    int s_it = 0, pv_wait = 0;
+    int s_it = 0, pv_wait = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
       const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j, ++s_it) {
-        const int sb = s_it & 1;
-        if (!(ok = mbar_wait(bar(bars->s_full[sb]), (s_it >> 1) & 1, abort, p.err, 20))) break;
+        const int sb = s_it % kSBufs;
+        if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(lane_addr + kColS + sb * 128 + q4 * 32, sr[q4]);
+        uint32_t sr[2][32];
+        tmem_ld32(lane_addr + kColS + sb * 128 + half * 64, sr[0]);
+        tmem_ld32(lane_addr + kColS + sb * 128 + half * 64 + 32, sr[1]);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bars->s_free[sb]));
-        float mx = -INFINITY;
+        float mk[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
+        for (int a = 0; a < 8; ++a) mk[a] = fmaxf(__uint_as_float(sr[0][a]), __uint_as_float(sr[0][a + 8]));
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[q4][e]));
+        for (int e = 16; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(sr[0][e]));
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(sr[1][e]));
+        const float mpart = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                                  fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
+        float* slot = xmax + (j & 1) * 256;
+        slot[half * 128 + row_in_tile] = mpart;
+        mbar_arrive(bar(bars->pair[sp]));
+        if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 23))) break;
+        ++xk;
+        const float mx = fmaxf(mpart, slot[(half ^ 1) * 128 + row_in_tile]);
         const float m_new = fmaxf(m_used, mx * c);
         const bool need = m_new > m_used + kRescaleLog2;
         const bool warp_need = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
         if (need) {
-          alpha = exp2f(m_used - m_new);
+          alpha = exp2_mufu(m_used - m_new);
           m_used = m_new;
         }
         l *= alpha;
         const float mneg = -m_used;
-        uint32_t pk[2][32];
-        float rs = 0.f;
+        uint32_t pk[32];
+        float rs[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = exp2f(fmaf(__uint_as_float(sr[q4][e]), c, mneg));
-            const float p1 = exp2f(fmaf(__uint_as_float(sr[q4][e + 1]), c, mneg));
-            rs += p0 + p1;
-            pk[q4 >> 1][(q4 & 1) * 16 + (e >> 1)] = pack_bf16(p0, p1);
+            const float x0 = fmaf(__uint_as_float(sr[q2][e]), c, mneg);
+            const float x1 = fmaf(__uint_as_float(sr[q2][e + 1]), c, mneg);
+            const float p0 = exp2_mufu(x0);
+            const float p1 = ((e + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x1) : exp2_mufu(x1);
+            rs[(e >> 1) & 7] += p0 + p1;
+            pk[q2 * 16 + (e >> 1)] = pack_bf16(p0, p1);
           }
         }
-        l += rs;
+        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         if (j >= 1) {
-          if (!(ok = mbar_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 21))) break;
+          if (!(ok = warp_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 21))) break;
           ++pv_wait;
           tc_fence_after();
           if (warp_need) {
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
               uint32_t o[32];
-              tmem_ld32(lane_addr + kColO + q4 * 32, o);
+              const uint32_t oa = lane_addr + kColO + half * 64 + q2 * 32;
+              tmem_ld32(oa, o);
               tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(lane_addr + kColO + q4 * 32, o);
+              tmem_st32(oa, o);
             }
           }
         }
-        tmem_st32(lane_addr + kColP + sb * 64, pk[0]);
-        tmem_st32(lane_addr + kColP + sb * 64 + 32, pk[1]);
+        tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->p_full[sb]));
       }
       if (!ok) break;
-      // epilogue: wait for the last P.V, normalise, store the raster output
-      if (!(ok = mbar_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 22))) break;
+      // epilogue: wait for the last P.V, combine the two halves' row sums,
+      // normalise and store this thread's 64 output channels
+      if (!(ok = warp_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 22))) break;
       ++pv_wait;
       tc_fence_after();
+      xsum[half * 128 + row_in_tile] = l;
+      mbar_arrive(bar(bars->pair[sp]));
+      if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
+      ++xk;
+      const float inv = 1.0f / (l + xsum[(half ^ 1) * 128 + row_in_tile]);
       const int bhh = rr / g.nQB, qb = rr % g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       const int tb = qb / g.bpf, rem = qb % g.bpf;
       const int tt = row_in_tile / (g.bh * g.bw), yy = (row_in_tile / g.bw) % g.bh, xx = row_in_tile % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
-      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD;
-      const float inv = 1.0f / l;
+      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + half * 64;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t o[32];
-        tmem_ld32(lane_addr + kColO + q4 * 32, o);
+        tmem_ld32(lane_addr + kColO + half * 64 + q2 * 32, o);
         tmem_wait_ld();
         uint4 v[4];
         uint32_t* w = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + q4 * 32);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e) d4[e] = v[e];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bars->o_free));
+      // xsum is rewritten only after this row's next exchanges, which need the
+      // partner's arrival, so the partner has read it by then
     }
   }
 
@@ -478,6 +575,11 @@ EncodeTiled encoder() {
 }  // namespace
 
 bool attention_tc_supported(const Grid& g) { return g.nb == kNB; }
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s) {
+  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows) {
   EncodeTiled enc = encoder();

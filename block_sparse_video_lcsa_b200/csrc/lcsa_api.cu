@@ -381,6 +381,7 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k1.rope_w_off = p->rope_w_off;
   k1.norm_scope = p->cfg.norm_scope;
   k1.eps = p->cfg.rms_eps;
+  k1.err = p->err;
 
   lcsa::K2Params k2;
   k2.g = g;
@@ -544,6 +545,13 @@ lcsa_status_t lcsa_get_kernel_times(lcsa_plan_t p, float ms[3], int* count) {
   for (int k = 0; k < 3; ++k) ms[k] = float(acc[k] / double(n));
   if (count) *count = int(n);
   return LCSA_OK;
+}
+
+lcsa_status_t lcsa_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0) return fail(LCSA_ERR_INVALID_ARG, "null pointer or negative count");
+  if (n == 0) return LCSA_OK;
+  cudaError_t e = lcsa::launch_exp2_selftest(x, y, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LCSA_OK : cuda_fail(e, "exp2 self-test launch");
 }
 
 const char* lcsa_status_string(lcsa_status_t s) {

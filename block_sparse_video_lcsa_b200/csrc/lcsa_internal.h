@@ -62,6 +62,7 @@ struct K1Params {
   int rope_h_off, rope_w_off;  // float2 offsets of the row and column tables
   int norm_scope;       // 0 token, 1 head
   float eps;
+  unsigned* err;        // device error word (bounded waits record a timeout here)
 };
 
 struct K2Params {
@@ -100,6 +101,7 @@ cudaError_t launch_attention_mma(const K3Params& p, cudaStream_t s);
 bool attention_tc_supported(const Grid& g);
 cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows);
 cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g);
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s);
 

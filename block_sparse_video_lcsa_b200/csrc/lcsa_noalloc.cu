@@ -215,6 +215,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.rope_w_off = k1.rope_h_off + g.gh * rs.pairs_h;
   k1.norm_scope = cfg->norm_scope;
   k1.eps = cfg->rms_eps;
+  k1.err = err;
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
 
   int sort_n = 32;

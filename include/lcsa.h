@@ -216,6 +216,14 @@ LCSA_API lcsa_status_t lcsa_plan_set_timing(lcsa_plan_t plan, int capacity);
    many were averaged. Synchronises on the newest recorded event. */
 LCSA_API lcsa_status_t lcsa_get_kernel_times(lcsa_plan_t plan, float ms[3], int* count);
 
+/* Self-test of the attention kernel's FMA-pipe exponential: y[i] = 2^x[i]
+   computed exactly as the softmax does for one exponential in four
+   (Cody-Waite reduction and a degree-3 minimax polynomial; relative error
+   below 7.5e-5 for -125 <= x <= 8). x, y: device fp32 [n]. Asynchronous.
+   The pages' FFMA-form softmax math ("FlashVSR: From 17.2 FPS to 57.3 FPS at
+   768x1408", Rebuild sparse attention for Hopper) is the source of the idea. */
+LCSA_API lcsa_status_t lcsa_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 /* Static text of a status code. */
 LCSA_API const char* lcsa_status_string(lcsa_status_t status);
 
