@@ -10,36 +10,45 @@
 // operand of the P.V product.
 //
 // Persistent: one CTA per SM walks rows (batch, head, query block) r =
-// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (320 threads):
+// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (352 threads):
 //   warp 0  TMA producer: Q tile of the row, then K^ / V blocks of its CSR list
 //           (K^ from the block-major prologue output, V straight from the
 //           raster input through a 5-D tensor map: d, head, x, y, frame).
-//   warp 1  MMA issuer (one lane): S = Q K^T into a ring of three TMEM S
-//           buffers, issued two KV blocks ahead of the softmax, and O += P V
-//           with P read from TMEM; also owns the TMEM allocation.
-//   warps 2-9 softmax, two warpgroups: a query row (TMEM lane) is shared by
+//   warp 1  S issuer: S = Q K^T (both operands in shared memory) into a ring
+//           of three TMEM S buffers, running up to three KV blocks ahead of
+//           the softmax; also owns the TMEM allocation.
+//   warp 2  P.V issuer: O += P V with P read from TMEM.
+//           Each issuer is a converged warp (every lane waits, lane 0
+//           issues), so each feeds the tensor pipe one kind of product: a
+//           single thread that alternates the two kinds with barrier waits in
+//           between was measured to issue at half the pipe's rate. The two
+//           streams are ordered only through mbarriers: S of block j+3 waits
+//           until P.V of block j (which reads P_j from the same buffer) has
+//           completed.
+//   warps 3-10 softmax, two warpgroups: a query row (TMEM lane) is shared by
 //           lane i of warp w and of warp w+4, each owning 64 of its 128 key
 //           columns. The pair trades row maxima (and at the end row sums)
 //           through shared memory, ordered by an mbarrier of 64 arrivals. Online
 //           softmax in the exp2 domain (scale folded into log2 e), P written
 //           to TMEM as bf16 pairs, O rescaled only when the running max grew
 //           by more than 2^8 (exact: O and the row sum use the same stale
-//           max); finally each thread normalises and stores 64 of the row's
-//           output channels. Independent accumulators break the max and sum
-//           chains, and every fourth exponential runs on the FMA pipe
-//           (Cody-Waite reduction 2^x = 2^n 2^f, |f| <= 1/2, and a degree-3
-//           minimax polynomial for 2^f fitted for this kernel, relative
-//           error below 7.5e-5) so the MUFU unit is not the bottleneck (the
-//           pages' "FFMA-form softmax math").
+//           max); only a rescale waits for the preceding P.V, so the softmax
+//           of block j overlaps P.V of block j-1. Finally each thread
+//           normalises and stores 64 of the row's output channels.
+//           Independent accumulators break the max and sum chains, and every
+//           fourth exponential runs on the FMA pipe (Cody-Waite reduction
+//           2^x = 2^n 2^f, |f| <= 1/2, and a degree-3 minimax polynomial for
+//           2^f fitted for this kernel, relative error below 7.5e-5) so the
+//           MUFU unit is not the bottleneck (the pages' "FFMA-form softmax
+//           math").
 // TMEM columns: S ring [0,128) [128,256) [256,384), O [384,512). P of block j
 // is written back into S buffer j % 3 (bf16 pairs; keys 0-63 in its columns
 // 0-31, keys 64-127 in columns 64-95, each half inside the columns its own
-// thread has already read). The tensor pipe runs one issuer's MMAs in order,
-// so S of block j+3, issued after P.V of block j, cannot overwrite P_j early.
+// thread has already read).
 // Shared memory: Q 32 KB, K^ ring 2 x 32 KB, V ring 3 x 32 KB, all in the
 // 128-byte swizzled layout that TMA writes and the MMA descriptors read. The
 // producer fetches K^ two blocks ahead of V (K^_{j+2} before V_j), matching
-// the order in which the MMA issuer consumes them.
+// the order in which the issuers consume them.
 //
 // Every wait on an mbarrier is bounded (wall-clock limit); a wait that runs
 // out records LCSA device error "timeout", raises a CTA-wide abort flag and
@@ -57,7 +66,7 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 3;
 constexpr uint32_t kTileBytes = kNB * kD * 2;   // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2; // 64 columns of a tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kPolyEvery = 4;  // one exponential in kPolyEvery on the FMA pipe
 constexpr int kSBufs = 3;
@@ -84,14 +93,15 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[kSBufs], p_full[kSBufs];
-  uint64_t o_done, o_free, mma_drain;
+  uint64_t s_full[kSBufs], p_full[kSBufs], s_free[kSBufs];
+  uint64_t o_done[2];  // o_done[g & 1]: P.V number g (counted per CTA) and all before it have completed
+  uint64_t o_free, mma_drain[2];
   uint64_t pair[4];  // row max / sum exchange between the two softmax warps of a lane quarter
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
-static_assert(kSoftmaxWarps == 8 && kThreads == 64 + 32 * kSoftmaxWarps, "warp roles");
+static_assert(kSoftmaxWarps == 8 && kThreads == 96 + 32 * kSoftmaxWarps, "warp roles");
 
 struct TcParams {
   Grid g;
@@ -153,6 +163,15 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
         return false;
       }
     }
+  }
+}
+
+// Wait for an issuer's own tensor-core work to finish before the TMEM is
+// freed: ignores the abort flag (that work is in flight either way) and gives
+// up only at the wall-clock limit.
+__device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity) && global_ns() - t0 <= kWaitLimitNs) {
   }
 }
 
@@ -303,10 +322,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(bars->s_full[s]), 1);
       mbar_init(bar(bars->p_full[s]), kSoftmaxWarps);
+      mbar_init(bar(bars->s_free[s]), 1);
     }
-    mbar_init(bar(bars->o_done), 1);
+    mbar_init(bar(bars->o_done[0]), 1);
+    mbar_init(bar(bars->o_done[1]), 1);
     mbar_init(bar(bars->o_free), kSoftmaxWarps);
-    mbar_init(bar(bars->mma_drain), 1);
+    mbar_init(bar(bars->mma_drain[0]), 1);
+    mbar_init(bar(bars->mma_drain[1]), 1);
     for (int s = 0; s < 4; ++s) mbar_init(bar(bars->pair[s]), 64);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -362,46 +384,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(0), id_pv = idesc_bf16(1);
-      int kv = 0, s_it = 0, pv_it = 0, row_it = 0;
-      bool ok = true, issued = false;
-      // S of the row's block j into buffer (s_it % 3)
-      auto issue_s = [&](int j, int n) -> bool {
+    // ---------------- S issuer (converged warp, lane 0 issues) ----------------
+    constexpr uint32_t id_qk = idesc_bf16(0);
+    int kv = 0, s_it = 0, row_it = 0;
+    bool ok = true, issued = false;
+    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
+      for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
         const int kvj = kv + j, ks = kvj % kKStages;
-        if (!mbar_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12)) return false;
+        // buffer sb last held P of block s_it - 3: its P.V must have completed
+        if (s_it >= kSBufs &&
+            !(ok = warp_wait(bar(bars->s_free[sb]), ((s_it / kSBufs) - 1) & 1, abort, p.err, 11)))
+          break;
+        if (!(ok = warp_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
         tc_fence_after();
-        const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
+        if (lane == 0) {
+          const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(bars->s_full[sb]));
+          mma_commit(bar(bars->k_empty[ks]));
+          if (j == n - 1) mma_commit(bar(bars->q_empty));
         }
+        __syncwarp();
         issued = true;
-        mma_commit(bar(bars->s_full[sb]));
-        mma_commit(bar(bars->k_empty[ks]));
-        if (j == n - 1) mma_commit(bar(bars->q_empty));
-        ++s_it;
-        return true;
-      };
-      for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-        const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
-        if (!(ok = mbar_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
-        for (int j = 0; j < 2 && j < n && ok; ++j) ok = issue_s(j, n);
-        for (int j = 0; j < n && ok; ++j) {
-          // S two blocks ahead: its buffer last held P of block j-1, whose P.V
-          // was issued in the previous step (in-order pipe)
-          if (j + 2 < n && !(ok = issue_s(j + 2, n))) break;
-          const int pb = pv_it % kSBufs;
-          if (!(ok = mbar_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
-          const int kvi = kv + j, vs = kvi % kVStages;
-          if (!(ok = mbar_wait(bar(bars->v_full[vs]), (kvi / kVStages) & 1, abort, p.err, 14))) break;
-          if (j == 0 && row_it > 0 && !(ok = mbar_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
-            break;
-          tc_fence_after();
+      }
+      kv += n;
+    }
+    if (issued) {
+      if (lane == 0) mma_commit(bar(bars->mma_drain[0]));
+      __syncwarp();
+      mbar_drain(bar(bars->mma_drain[0]), 0);
+    }
+  } else if (warp == 2) {
+    // ---------------- P.V issuer (converged warp, lane 0 issues) ----------------
+    constexpr uint32_t id_pv = idesc_bf16(1);
+    int kv = 0, pv_it = 0, row_it = 0;
+    bool ok = true, issued = false;
+    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      for (int j = 0; j < n; ++j, ++pv_it) {
+        const int pb = pv_it % kSBufs;
+        if (!(ok = warp_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
+        const int kvi = kv + j, vs = kvi % kVStages;
+        if (!(ok = warp_wait(bar(bars->v_full[vs]), (kvi / kVStages) & 1, abort, p.err, 14))) break;
+        if (j == 0 && row_it > 0 && !(ok = warp_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
+          break;
+        tc_fence_after();
+        if (lane == 0) {
           const uint32_t va = base + kOffV + vs * kTileBytes;
           const uint32_t pa = tmem + kColS + pb * 128;
 #pragma unroll
@@ -410,26 +446,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                    id_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(bars->v_empty[vs]));
-          mma_commit(bar(bars->o_done));
-          ++pv_it;
+          mma_commit(bar(bars->s_free[pb]));
+          mma_commit(bar(bars->o_done[pv_it & 1]));
         }
-        kv += n;
+        __syncwarp();
+        issued = true;
       }
-      if (issued) {
-        mma_commit(bar(bars->mma_drain));
-        mbar_wait(bar(bars->mma_drain), 0, abort, p.err, 16);
-      }
+      kv += n;
+    }
+    if (issued) {
+      if (lane == 0) mma_commit(bar(bars->mma_drain[1]));
+      __syncwarp();
+      mbar_drain(bar(bars->mma_drain[1]), 0);
     }
   } else {
     // ---------------- softmax / correction / epilogue ----------------
     const int sp = warp & 3;                 // TMEM lane quarter of this warp
-    const int half = (warp - 2) >> 2;        // which 64 key columns / channels
+    const int half = (warp - 3) >> 2;        // which 64 key columns / channels
     const int row_in_tile = sp * 32 + lane;  // query token index inside the block
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
     float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
     float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
     const float c = p.scale_log2;
-    int s_it = 0, pv_wait = 0, xk = 0;
+    int s_it = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
       const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
@@ -484,21 +523,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-        if (j >= 1) {
-          if (!(ok = warp_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 21))) break;
-          ++pv_wait;
+        // O is touched only to rescale it, once every earlier P.V has
+        // completed; the last of them is P.V number gp = s_it - 1. P.V number
+        // gp + 2 needs a P this warp has not written yet, so the parity wait
+        // on o_done[gp & 1] cannot be overtaken.
+        if (j >= 1 && warp_need) {
+          const int gp = s_it - 1;
+          if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 21))) break;
           tc_fence_after();
-          if (warp_need) {
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              uint32_t o[32];
-              const uint32_t oa = lane_addr + kColO + half * 64 + q2 * 32;
-              tmem_ld32(oa, o);
-              tmem_wait_ld();
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t o[32];
+            const uint32_t oa = lane_addr + kColO + half * 64 + q2 * 32;
+            tmem_ld32(oa, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(oa, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(oa, o);
           }
         }
         tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
@@ -510,8 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: wait for the last P.V, combine the two halves' row sums,
       // normalise and store this thread's 64 output channels
-      if (!(ok = warp_wait(bar(bars->o_done), pv_wait & 1, abort, p.err, 22))) break;
-      ++pv_wait;
+      {
+        const int gp = s_it - 1;  // the row's last P.V (completion implies all earlier ones)
+        if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 22))) break;
+      }
       tc_fence_after();
       xsum[half * 128 + row_in_tile] = l;
       mbar_arrive(bar(bars->pair[sp]));
