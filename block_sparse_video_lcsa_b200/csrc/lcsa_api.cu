@@ -206,7 +206,7 @@ struct lcsa_plan {
   void* st_out = nullptr;
   float* st_gq = nullptr;
   float* st_gk = nullptr;
-  // tcgen05 attention: tensor maps of the plan-owned q^ / k^, SM count
+  // tcgen05 attention: tensor maps of the plan-owned q^ / k^; SM count (persistent grids)
   bool use_tc = false;
   CUtensorMap tm_q, tm_k;
   int num_sms = 0;
@@ -332,10 +332,14 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
     delete p;
     return cuda_fail(e, "plan set-up");
   }
+  if ((e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, cuda_device)) != cudaSuccess) {
+    release(p);
+    delete p;
+    return cuda_fail(e, "device attributes");
+  }
   p->use_tc = lcsa::attention_tc_supported(g);
   if (p->use_tc) {
-    if ((e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, cuda_device)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
+    if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
         (e = lcsa::make_block_map(&p->tm_k, p->khat, int64_t(g.B) * g.Hn * g.nKB * g.nb)) != cudaSuccess) {
       release(p);
       delete p;
@@ -382,6 +386,7 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k1.norm_scope = p->cfg.norm_scope;
   k1.eps = p->cfg.rms_eps;
   k1.err = p->err;
+  k1.num_sms = p->num_sms;
 
   lcsa::K2Params k2;
   k2.g = g;

@@ -63,6 +63,7 @@ struct K1Params {
   int norm_scope;       // 0 token, 1 head
   float eps;
   unsigned* err;        // device error word (bounded waits record a timeout here)
+  int num_sms;          // persistent grid size (one CTA per SM)
 };
 
 struct K2Params {

@@ -216,6 +216,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.norm_scope = cfg->norm_scope;
   k1.eps = cfg->rms_eps;
   k1.err = err;
+  if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return noalloc_fail(LCSA_ERR_CUDA, "device attributes");
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
 
   int sort_n = 32;
@@ -244,9 +246,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.err = err;
   if (lcsa::attention_tc_supported(g)) {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
-    int num_sms = 0;
-    if ((e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
+    const int num_sms = k1.num_sms;
+    if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
         (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb)) != cudaSuccess ||
         (e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess)
       return noalloc_fail(LCSA_ERR_CUDA, "tensor maps");
