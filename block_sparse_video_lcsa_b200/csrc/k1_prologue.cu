@@ -9,28 +9,29 @@
 // pooling and RoPE as separate glue kernels) and Rebuild sparse attention for
 // Hopper (coalesced RoPE kernel, pooled keys).
 //
-// Work split: a persistent grid of one CTA (8 warps) per SM walks the q and
-// k blocks blockIdx.x, blockIdx.x + gridDim.x, ... A block is bt * bh rows of
-// bw tokens, and each row is one contiguous run of bw * heads * 128 bf16 in
-// the raster input, so one thread streams rows into a ring of shared-memory
-// stages with bulk asynchronous copies (cp.async.bulk, completion counted on
-// an mbarrier), several rows ahead and across block boundaries, while the
-// warps work on the oldest stage: warp w takes tokens w, w+8, ... of the row,
-// lane l the 16-byte chunks l, l+32, ... of a token (conflict-free shared
-// loads), so each lane always holds the same channels. The gain and the
-// pooled sums therefore live in registers for the whole block; the sum of
-// squares is a warp-shuffle reduction; at the end of a block the 8 warps'
-// partial sums are added in a fixed order, so the pooled values (and hence
-// the block selection) are deterministic. q^ / k^ are written with 16-byte
-// stores, every store instruction of a warp covering whole 256-byte rows of
-// two heads.
+// Work split: a persistent grid of one CTA (8 warps) per SM; CTA c owns a
+// contiguous range of the combined row list (query blocks, then key blocks;
+// a block is bt * bh rows of bw tokens). Each row is one contiguous run of
+// bw * heads * 128 bf16 in the raster input, so one thread streams the rows
+// into a ring of shared-memory stages with bulk asynchronous copies
+// (cp.async.bulk, completion counted on an mbarrier) several rows ahead,
+// while the warps work on the oldest stage: warp w takes tokens w, w+8, ...
+// of the row, lane l the 16-byte chunks l, l+32, ... of a token
+// (conflict-free shared loads), so each lane always holds the same channels
+// and its pooled sums live in registers (gains: a lane-contiguous table in
+// shared memory). The sum of squares is a warp-shuffle reduction. Pooled
+// sums are added in a fixed order: per lane
+// over its tokens, then over the warps, and for a block cut between two
+// CTAs, first part plus second part; so the pooled values, and hence the
+// block selection, do not depend on timing. q^ / k^ are written with 16-byte
+// stores, each warp store instruction covering whole 256-byte rows of two
+// heads.
 #include "lcsa_internal.h"
 
 namespace lcsa {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kRedRows = 8;  // rows of the pooled-sum reduction buffer
 
 __global__ void rope_table_kernel(float2* tab, int Tkv, int gh, int gw, int t0, RopeSplit s) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -53,26 +54,25 @@ __global__ void rope_table_kernel(float2* tab, int Tkv, int gh, int gw, int t0, 
   tab[i] = make_float2(float(cos(ang)), float(sin(ang)));
 }
 
-// bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 word.
-// Done with integer shifts and masks, which leaves the conversion unit free.
-__device__ __forceinline__ void unpack8(const uint4& r, float (&f)[8]) {
+// bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 word, so
+// unpacking is integer shifts and masks, which leaves the conversion unit free.
+// The bf16 words become float pairs for packed fp32x2 arithmetic: e[qg]
+// holds elements (4qg, 4qg+2), o[qg] elements (4qg+1, 4qg+3), i.e. the first
+// and second members of the rotation pairs 2qg and 2qg+1.
+__device__ __forceinline__ void unpack_eo(const uint4& r, float2 (&e)[2], float2 (&o)[2]) {
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  for (int qg = 0; qg < 2; ++qg) {
+    e[qg] = make_float2(__uint_as_float(w[2 * qg] << 16), __uint_as_float(w[2 * qg + 1] << 16));
+    o[qg] = make_float2(__uint_as_float(w[2 * qg] & 0xFFFF0000u), __uint_as_float(w[2 * qg + 1] & 0xFFFF0000u));
   }
 }
 
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-  uint4 r;
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-  return r;
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// CPL = 16-byte chunks per lane per token = ceil(heads * 16 / 32).
 constexpr int kMaxStages = 4;
 constexpr uint32_t kSmemBudget = 220 * 1024;
 constexpr uint32_t kBarBytes = 128;  // mbarriers of the ring
@@ -136,25 +136,39 @@ __device__ __forceinline__ BlockRef block_ref(const Grid& g, int bid) {
 
 // CPL = 16-byte chunks per lane per token = ceil(heads * 16 / 32); FULL: every
 // lane's CPL chunks exist (even head count); HEAD: per-head norm scope.
+// Warps per CTA. (16, one token of a 16-token row each, measured slower: a
+// lane's pooled sums and token do not fit 128 registers without spills.)
+template <int CPL>
+__host__ __device__ constexpr int k1_warps() { return 8; }
+
 template <int CPL, bool FULL, bool HEAD>
-__global__ void __launch_bounds__(kThreads, 1) prologue_kernel(const K1Params p, int stages, uint32_t row_bytes) {
+__global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const K1Params p, int stages,
+                                                                          uint32_t row_bytes) {
+  constexpr int NW = k1_warps<CPL>(), NT = NW * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   const Grid& g = p.g;
   const uint32_t bars = smem_u32(smem);
   uint8_t* ring = smem + kBarBytes;
-  float* red = reinterpret_cast<float*>(ring + size_t(stages) * row_bytes);  // [kWarps][C]
+  float* red = reinterpret_cast<float*>(ring + size_t(stages) * row_bytes);  // [kRedRows][C]
+  // gains of q and k, [tensor][c4][half][lane] float4: lane-contiguous, so conflict-free
+  float4* gsm = reinterpret_cast<float4*>(red + kRedRows * g.C);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunks = g.C / 8;
   const int R = g.bt * g.bh;  // rows per block
   const int total = g.B * (g.nQB + g.nKB);
-  const int my_blocks = (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x);
-  const int my_rows = my_blocks * R;
+  // this CTA's rows: a contiguous range of the combined row list (blocks in
+  // order, rows of a block in order); every range holds at least R rows, so a
+  // block is cut by at most one range boundary
+  const int64_t nrows = int64_t(total) * R;
+  const int64_t lo = nrows * blockIdx.x / gridDim.x, hi = nrows * (blockIdx.x + 1) / gridDim.x;
+  const int my_rows = int(hi - lo);
   constexpr int PT = 22, PH = 21;  // RoPE pairs on the frame / row axes (head_dim 128)
 
-  // source of the CTA's row number gi (its blocks' rows, in order)
-  auto row_src = [&](int gi) -> const void* {
-    const BlockRef br = block_ref(g, int(blockIdx.x) + (gi / R) * int(gridDim.x));
-    const int r = gi % R;
+  // source of the CTA's row number k (global row lo + k)
+  auto row_src = [&](int k) -> const void* {
+    const int64_t grow = lo + k;
+    const BlockRef br = block_ref(g, int(grow / R));
+    const int r = int(grow % R);
     const int64_t tok = (int64_t(br.t0 + r / g.bh) * g.gh + br.y0 + r % g.bh) * g.gw + br.x0;
     const __nv_bfloat16* x = br.is_q ? p.q : p.k;
     const int64_t L = br.is_q ? g.Lq : g.Lkv;
@@ -173,36 +187,40 @@ __global__ void __launch_bounds__(kThreads, 1) prologue_kernel(const K1Params p,
   __syncthreads();
   if (threadIdx.x == 0)
     for (int gi = 0; gi < stages && gi < my_rows; ++gi) issue(gi);
+  for (int idx = threadIdx.x; idx < 2 * CPL * 64; idx += NT) {
+    const int rem = idx % (CPL * 64);
+    const int c = (rem / 64) * 32 + rem % 32, half = (rem / 32) % 2;
+    const float* gamma = idx < CPL * 64 ? p.gamma_q : p.gamma_k;
+    gsm[idx] = c < nchunks ? __ldg(reinterpret_cast<const float4*>(gamma + c * 8 + half * 4))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
 
   const int jb = 4 * (lane & 15);  // first RoPE pair of this lane (same in every head)
-  float gm[CPL][8], acc[CPL][8];
-  int gi = 0;
+  float2 ae[CPL][2], ao[CPL][2];  // pooled sums, e / o layout of unpack_eo
+  __shared__ int combine;
+  int gi = 0;  // rows of this CTA consumed so far
   bool ok = true;
-  for (int kb = 0; kb < my_blocks && ok; ++kb) {
-    const BlockRef br = block_ref(g, int(blockIdx.x) + kb * int(gridDim.x));
-    const float* gamma = br.is_q ? p.gamma_q : p.gamma_k;
+  while (gi < my_rows && ok) {
+    // one segment: the rows [r_begin, r_end) of block bid that this CTA owns
+    const int bid = int((lo + gi) / R);
+    const int r_begin = int((lo + gi) % R);
+    const int r_end = min(R, r_begin + (my_rows - gi));
+    const BlockRef br = block_ref(g, bid);
+    const float4* gtab = gsm + (br.is_q ? 0 : CPL * 64);
     __nv_bfloat16* xhat = br.is_q ? p.qhat : p.khat;
     float* pooled = br.is_q ? p.pooled_q : p.pooled_k;
     const int tshift = br.is_q ? (g.Tkv - g.Tq) : 0;
 #pragma unroll
-    for (int c4 = 0; c4 < CPL; ++c4) {
-      const int c = c4 * 32 + lane;
-      float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0;
-      if (c < nchunks) {
-        g0 = __ldg(reinterpret_cast<const float4*>(gamma + c * 8));
-        g1 = __ldg(reinterpret_cast<const float4*>(gamma + c * 8 + 4));
-      }
-      gm[c4][0] = g0.x; gm[c4][1] = g0.y; gm[c4][2] = g0.z; gm[c4][3] = g0.w;
-      gm[c4][4] = g1.x; gm[c4][5] = g1.y; gm[c4][6] = g1.z; gm[c4][7] = g1.w;
+    for (int c4 = 0; c4 < CPL; ++c4)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[c4][e] = 0.f;
-    }
-    for (int r = 0; r < R; ++r, ++gi) {
+      for (int qg = 0; qg < 2; ++qg) ae[c4][qg] = ao[c4][qg] = make_float2(0.f, 0.f);
+    for (int r = r_begin; r < r_end; ++r, ++gi) {
       const int s = gi % stages;
       const bool arrived = mbar_wait_bounded(bars + 8 * s, uint32_t(gi / stages) & 1u);
       const int t = br.t0 + r / g.bh, y = br.y0 + r % g.bh;
       const uint4* row = reinterpret_cast<const uint4*>(ring + size_t(s) * row_bytes);
-      for (int i = warp; i < g.bw; i += kWarps) {
+      for (int i = warp; i < g.bw; i += NW) {
         const int xc = br.x0 + i;
         uint4 raw[CPL];
 #pragma unroll
@@ -220,41 +238,52 @@ __global__ void __launch_bounds__(kThreads, 1) prologue_kernel(const K1Params p,
                                         : p.rope_w_off + xc * (kHeadDim / 2 - PT - PH) + (j - PT - PH);
           cs[qd] = __ldg(p.rope + idx);
         }
-        // RMSNorm scale(s), folded into the rotation: x^ = rot(rs * (x * gamma))
-        float ca[HEAD ? CPL : 1][4], cb[HEAD ? CPL : 1][4];
+        // RMSNorm scale(s), folded into the rotation: x^ = rot(rs * (x * gamma)).
+        // ca/cb/nb[qg] = rs * (cos, sin, -sin) of the pairs 2qg and 2qg+1 (per
+        // token; with the head scope, per chunk inside the chunk loop).
+        float2 ca[2], cb[2], nb[2];
+        float rr_h[HEAD ? CPL : 1];
+        auto coefs = [&](float rr) {
+#pragma unroll
+          for (int qg = 0; qg < 2; ++qg) {
+            const float2 cosv = make_float2(cs[2 * qg].x, cs[2 * qg + 1].x);
+            const float2 sinv = make_float2(cs[2 * qg].y, cs[2 * qg + 1].y);
+            ca[qg] = __fmul2_rn(make_float2(rr, rr), cosv);
+            cb[qg] = __fmul2_rn(make_float2(rr, rr), sinv);
+            nb[qg] = __fmul2_rn(make_float2(-rr, -rr), sinv);
+          }
+        };
         if (!HEAD) {
-          float ss = 0.f;
+          float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int c4 = 0; c4 < CPL; ++c4) {
-            float f[8];
-            unpack8(raw[c4], f);
+            float2 e[2], o[2];
+            unpack_eo(raw[c4], e, o);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            for (int qg = 0; qg < 2; ++qg) {
+              ss2 = __ffma2_rn(e[qg], e[qg], ss2);
+              ss2 = __ffma2_rn(o[qg], o[qg], ss2);
+            }
           }
+          float ss = ss2.x + ss2.y;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const float rr = rsqrtf(ss * (1.0f / float(g.C)) + p.eps);
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            ca[0][qd] = rr * cs[qd].x;
-            cb[0][qd] = rr * cs[qd].y;
-          }
+          coefs(rsqrtf(ss * (1.0f / float(g.C)) + p.eps));
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < (HEAD ? CPL : 1); ++c4) {
-            float f[8];
-            unpack8(raw[c4], f);
-            float ss = 0.f;
+            float2 e[2], o[2];
+            unpack_eo(raw[c4], e, o);
+            float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float rr = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              ca[c4][qd] = rr * cs[qd].x;
-              cb[c4][qd] = rr * cs[qd].y;
+            for (int qg = 0; qg < 2; ++qg) {
+              ss2 = __ffma2_rn(e[qg], e[qg], ss2);
+              ss2 = __ffma2_rn(o[qg], o[qg], ss2);
             }
+            float ss = ss2.x + ss2.y;
+#pragma unroll
+            for (int o2 = 8; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
+            rr_h[c4] = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
           }
         }
         const int ti = r * g.bw + i;  // token index inside the block
@@ -262,22 +291,27 @@ __global__ void __launch_bounds__(kThreads, 1) prologue_kernel(const K1Params p,
         for (int c4 = 0; c4 < CPL; ++c4) {
           const int c = c4 * 32 + lane;
           if (!FULL && c >= nchunks) continue;
-          const int cc = HEAD ? c4 : 0;
-          float f[8], o[8];
-          unpack8(raw[c4], f);
+          if (HEAD) coefs(rr_h[HEAD ? c4 : 0]);
+          float2 e[2], o[2];
+          unpack_eo(raw[c4], e, o);
+          const float4 g0 = gtab[(c4 * 2) * 32 + lane], g1 = gtab[(c4 * 2 + 1) * 32 + lane];
+          const float2 ge[2] = {make_float2(g0.x, g0.z), make_float2(g1.x, g1.z)};
+          const float2 go[2] = {make_float2(g0.y, g0.w), make_float2(g1.y, g1.w)};
+          uint32_t w[4];
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const float u0 = f[2 * qd] * gm[c4][2 * qd];
-            const float u1 = f[2 * qd + 1] * gm[c4][2 * qd + 1];
-            o[2 * qd] = fmaf(u0, ca[cc][qd], -u1 * cb[cc][qd]);
-            o[2 * qd + 1] = fmaf(u0, cb[cc][qd], u1 * ca[cc][qd]);
+          for (int qg = 0; qg < 2; ++qg) {
+            const float2 ue = __fmul2_rn(e[qg], ge[qg]), uo = __fmul2_rn(o[qg], go[qg]);
+            const float2 oe = __ffma2_rn(uo, nb[qg], __fmul2_rn(ue, ca[qg]));  // first members
+            const float2 oo = __ffma2_rn(uo, ca[qg], __fmul2_rn(ue, cb[qg]));  // second members
+            ae[c4][qg] = __fadd2_rn(ae[c4][qg], oe);
+            ao[c4][qg] = __fadd2_rn(ao[c4][qg], oo);
+            w[2 * qg] = pack2(oe.x, oo.x);
+            w[2 * qg + 1] = pack2(oe.y, oo.y);
           }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[c4][e] += o[e];
           const int head = c >> 4, dd = (c & 15) * 8;
           uint4* dst = reinterpret_cast<uint4*>(
               xhat + (((int64_t(br.b) * g.Hn + head) * br.nblk + br.blk) * g.nb + ti) * kHeadDim + dd);
-          *dst = pack8(o);
+          *dst = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       // every warp is done with stage s (and agrees on whether the row arrived)
@@ -291,26 +325,64 @@ __global__ void __launch_bounds__(kThreads, 1) prologue_kernel(const K1Params p,
       }
     }
     if (!ok) break;
-    // warp partials -> block mean, summed over warps in a fixed order
-    float* mine = red + warp * g.C;
+    // warp partials -> segment sum: with 16 warps, warp w + 8 first leaves its
+    // sums in row w and warp w adds its own; then the 8 rows are added in order
+    float* mine = red + (warp % kRedRows) * g.C;
 #pragma unroll
-    for (int c4 = 0; c4 < CPL; ++c4) {
-      const int c = c4 * 32 + lane;
-      if (c < nchunks) {
-        reinterpret_cast<float4*>(mine + c * 8)[0] = make_float4(acc[c4][0], acc[c4][1], acc[c4][2], acc[c4][3]);
-        reinterpret_cast<float4*>(mine + c * 8)[1] = make_float4(acc[c4][4], acc[c4][5], acc[c4][6], acc[c4][7]);
+    for (int round = 0; round < NW / kRedRows; ++round) {
+      if (warp / kRedRows == NW / kRedRows - 1 - round) {
+#pragma unroll
+        for (int c4 = 0; c4 < CPL; ++c4) {
+          const int c = c4 * 32 + lane;
+          if (FULL || c < nchunks) {
+#pragma unroll
+            for (int qg = 0; qg < 2; ++qg) {
+              float4* slot = reinterpret_cast<float4*>(mine + c * 8) + qg;
+              float4 v = make_float4(ae[c4][qg].x, ao[c4][qg].x, ae[c4][qg].y, ao[c4][qg].y);
+              if (round > 0) {
+                const float4 prev = *slot;
+                v.x += prev.x; v.y += prev.y; v.z += prev.z; v.w += prev.w;
+              }
+              *slot = v;
+            }
+          }
+        }
       }
+      __syncthreads();
     }
-    __syncthreads();
     const float inv_nb = 1.0f / float(g.nb);
-    for (int e = threadIdx.x; e < g.C; e += kThreads) {
+    float* pooled_row = pooled + (int64_t(br.b) * g.Hn * br.nblk + br.blk) * kHeadDim;  // + head * nblk * d + dd
+    const int64_t head_stride = int64_t(br.nblk) * kHeadDim;
+    auto warp_sum = [&](int e) {
       float sum = red[e];
 #pragma unroll
-      for (int w = 1; w < kWarps; ++w) sum += red[w * g.C + e];
-      const int head = e / kHeadDim, dd = e % kHeadDim;
-      pooled[((int64_t(br.b) * g.Hn + head) * br.nblk + br.blk) * kHeadDim + dd] = sum * inv_nb;
+      for (int w = 1; w < kRedRows; ++w) sum += red[w * g.C + e];
+      return sum;
+    };
+    if (r_begin == 0 && r_end == R) {
+      for (int e = threadIdx.x; e < g.C; e += NT)
+        pooled_row[(e / kHeadDim) * head_stride + e % kHeadDim] = warp_sum(e) * inv_nb;
+    } else {
+      // A block cut between CTA c and c + 1: CTA c holds its first rows (part
+      // 0), CTA c + 1 the rest (part 1). Each writes its part to the cut's
+      // slot; the second to arrive adds part 0 + part 1 (always in that
+      // order) and writes the mean.
+      const int cut = r_begin == 0 ? int(blockIdx.x) : int(blockIdx.x) - 1;
+      float* part = p.split_part + size_t(cut) * 2 * g.C;
+      float* mypart = part + (r_begin == 0 ? 0 : g.C);
+      for (int e = threadIdx.x; e < g.C; e += NT) mypart[e] = warp_sum(e);
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) combine = atomicAdd(p.split_cnt + cut, 1u) == 1u;
+      __syncthreads();
+      if (combine) {
+        __threadfence();
+        for (int e = threadIdx.x; e < g.C; e += NT)
+          pooled_row[(e / kHeadDim) * head_stride + e % kHeadDim] =
+              (__ldcg(part + e) + __ldcg(part + g.C + e)) * inv_nb;
+      }
     }
-    __syncthreads();  // red is rewritten by the next block
+    __syncthreads();  // red and combine are rewritten by the next segment
   }
   if (!ok && threadIdx.x == 0) {
     // a row never arrived: record it, then give the copies still in flight a
@@ -329,15 +401,16 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   const int nblocks = p.g.B * (p.g.nQB + p.g.nKB);
   if (nblocks <= 0) return cudaSuccess;
   const uint32_t row_bytes = uint32_t(p.g.bw) * uint32_t(p.g.C) * 2u;
-  const uint32_t red_bytes = uint32_t(kWarps) * uint32_t(p.g.C) * 4u;
+  const uint32_t red_bytes = uint32_t(kRedRows) * uint32_t(p.g.C) * 4u + 2u * CPL * 64u * 16u;  // + gains
   int stages = int((kSmemBudget - kBarBytes - red_bytes) / row_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2 || p.num_sms <= 0) return cudaErrorInvalidValue;
   const size_t smem = kBarBytes + size_t(stages) * row_bytes + red_bytes;
   cudaError_t e = cudaFuncSetAttribute(prologue_kernel<CPL, FULL, HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  const int grid = nblocks < p.num_sms ? nblocks : p.num_sms;
-  prologue_kernel<CPL, FULL, HEAD><<<grid, kThreads, smem, s>>>(p, stages, row_bytes);
+  int grid = nblocks < p.num_sms ? nblocks : p.num_sms;
+  if (grid > kMaxK1Ctas) grid = kMaxK1Ctas;
+  prologue_kernel<CPL, FULL, HEAD><<<grid, k1_warps<CPL>() * 32, smem, s>>>(p, stages, row_bytes);
   return cudaGetLastError();
 }
 

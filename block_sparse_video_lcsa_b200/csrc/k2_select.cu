@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   const float4 qv = reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * kHeadDim)[lane];
   const float4* pk = reinterpret_cast<const float4*>(p.pooled_k + int64_t(bh) * g.nKB * kHeadDim);
 
+  if (blockIdx.x == 0)
+    for (int c = threadIdx.x; c < p.n_clear; c += kThreads) p.clear_cnt[c] = 0u;
   for (int c = threadIdx.x; c < p.sort_n; c += kThreads) flag[c] = 0;
   for (int c0 = warp * kCandPerIter; c0 < p.sort_n; c0 += kWarps * kCandPerIter) {
     float4 kv[kCandPerIter];

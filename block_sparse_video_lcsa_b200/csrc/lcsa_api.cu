@@ -176,6 +176,7 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   ws += size_t(g.B) * g.Hn * (g.nQB + g.nKB) * size_t(c->head_dim) * 4;         // pooled
   ws += (size_t(rows) + 1) * 4 + size_t(nnz) * 4;                                // CSR
   ws += rope_n * sizeof(float2) + 256;
+  ws += size_t(lcsa::kMaxK1Ctas) * (2 * size_t(g.C) * 4 + 4);                    // K1 split blocks
   if (c->host_io)
     ws += size_t(g.B) * (2 * g.Lq + 2 * g.Lkv) * g.C * 2 + size_t(2) * g.C * 4;
   o.workspace_bytes = ws;
@@ -194,6 +195,8 @@ struct lcsa_plan {
   __nv_bfloat16* khat = nullptr;
   float* pooled_q = nullptr;
   float* pooled_k = nullptr;
+  float* split_part = nullptr;     // K1: partial pooled sums of blocks cut between CTAs
+  unsigned* split_cnt = nullptr;   // K1: arrivals per cut (K2 zeroes them after use)
   int32_t* row_ptr = nullptr;
   int32_t* col_idx = nullptr;
   float2* rope = nullptr;
@@ -217,8 +220,9 @@ struct lcsa_plan {
 namespace {
 
 void release(lcsa_plan* p) {
-  void* ptrs[] = {p->qhat, p->khat, p->pooled_q, p->pooled_k, p->row_ptr, p->col_idx, p->rope, p->err,
-                  p->st_q, p->st_k, p->st_v, p->st_out, p->st_gq, p->st_gk};
+  void* ptrs[] = {p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
+                  p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
+                  p->st_v,  p->st_out,  p->st_gq,    p->st_gk};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (auto& set : p->evsets)
@@ -306,7 +310,9 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
       (st = dev_alloc(&p->row_ptr, (rows + 1) * 4, "row_ptr")) ||
       (st = dev_alloc(&p->col_idx, nnz * 4, "col_idx")) ||
       (st = dev_alloc(&p->rope, rope_n * sizeof(float2), "rope table")) ||
-      (st = dev_alloc(&p->err, 256, "error word"))) {
+      (st = dev_alloc(&p->err, 256, "error word")) ||
+      (st = dev_alloc(&p->split_part, size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4, "K1 split sums")) ||
+      (st = dev_alloc(&p->split_cnt, size_t(lcsa::kMaxK1Ctas) * 4, "K1 split counters"))) {
     release(p);
     delete p;
     return st;
@@ -325,6 +331,7 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
   }
   if ((e = cudaMemcpy(p->row_ptr, p->res.row_ptr.data(), (rows + 1) * 4, cudaMemcpyHostToDevice)) != cudaSuccess ||
       (e = cudaMemset(p->err, 0, 256)) != cudaSuccess ||
+      (e = cudaMemset(p->split_cnt, 0, size_t(lcsa::kMaxK1Ctas) * 4)) != cudaSuccess ||
       (e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, cfg->head_dim, 0)) !=
           cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
@@ -387,6 +394,8 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k1.eps = p->cfg.rms_eps;
   k1.err = p->err;
   k1.num_sms = p->num_sms;
+  k1.split_part = p->split_part;
+  k1.split_cnt = p->split_cnt;
 
   lcsa::K2Params k2;
   k2.g = g;
@@ -397,6 +406,8 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k2.radius = p->res.radius;
   k2.topk = p->res.geo.topk;
   k2.sort_n = p->res.sort_n;
+  k2.clear_cnt = p->split_cnt;
+  k2.n_clear = lcsa::kMaxK1Ctas;
 
   lcsa::K3Params k3;
   k3.g = g;

@@ -12,6 +12,7 @@ namespace lcsa {
 constexpr int kHeadDim = 128;        // the only head size the kernels implement
 constexpr int kMaxHeads = 16;
 constexpr int kMaxCandidates = 4096; // admissible blocks per query block (K2 sort)
+constexpr int kMaxK1Ctas = 256;      // K1 persistent grid cap (sizes its split-block buffers)
 
 // Device error word codes (first word of the plan's error buffer).
 constexpr unsigned kDevErrNone = 0;
@@ -63,7 +64,9 @@ struct K1Params {
   int norm_scope;       // 0 token, 1 head
   float eps;
   unsigned* err;        // device error word (bounded waits record a timeout here)
-  int num_sms;          // persistent grid size (one CTA per SM)
+  int num_sms;          // persistent grid size (one CTA per SM, at most kMaxK1Ctas)
+  float* split_part;    // [kMaxK1Ctas][2][C] partial pooled sums of blocks cut between CTAs
+  unsigned* split_cnt;  // [kMaxK1Ctas] arrivals per cut; zero on entry (K2 clears them)
 };
 
 struct K2Params {
@@ -75,6 +78,8 @@ struct K2Params {
   int radius;           // window radius in blocks, < 0 when unbounded
   int topk;
   int sort_n;           // power of two >= the largest admissible set
+  unsigned* clear_cnt;  // K1's split counters, zeroed here for the next K1 (n_clear entries)
+  int n_clear;
 };
 
 struct K3Params {

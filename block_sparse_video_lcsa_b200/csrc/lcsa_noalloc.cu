@@ -156,7 +156,9 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   const lcsa::RopeSplit rs = lcsa::rope_split(D);
   const size_t rope_n = size_t(g.Tkv) * rs.pairs_t + size_t(g.gh) * rs.pairs_h + size_t(g.gw) * rs.pairs_w;
   const size_t off_err = 0;
-  const size_t off_rope = off_err + 256;
+  const size_t off_cnt = off_err + 256;  // K1 split counters, cleared together with the error word
+  const size_t off_sp = off_cnt + round256(size_t(lcsa::kMaxK1Ctas) * 4);
+  const size_t off_rope = off_sp + round256(size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4);
   const size_t off_rp = off_rope + round256(rope_n * sizeof(float2));
   const size_t off_ci = off_rp + round256((size_t(ng.rows) + 1) * 4);
   const size_t off_pq = off_ci + round256(size_t(ng.nnz) * 4);
@@ -186,6 +188,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned* err = reinterpret_cast<unsigned*>(ws + off_err);
+  unsigned* split_cnt = reinterpret_cast<unsigned*>(ws + off_cnt);
+  float* split_part = reinterpret_cast<float*>(ws + off_sp);
   float2* rope = reinterpret_cast<float2*>(ws + off_rope);
   int* row_ptr = reinterpret_cast<int*>(ws + off_rp);
   int* col_idx = reinterpret_cast<int*>(ws + off_ci);
@@ -194,7 +198,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   __nv_bfloat16* qhat = reinterpret_cast<__nv_bfloat16*>(ws + off_qh);
   __nv_bfloat16* khat = reinterpret_cast<__nv_bfloat16*>(ws + off_kh);
 
-  if ((e = cudaMemsetAsync(err, 0, 256, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "clear error word");
+  if ((e = cudaMemsetAsync(err, 0, off_sp - off_err, s)) != cudaSuccess)
+    return noalloc_fail(LCSA_ERR_CUDA, "clear error word and counters");
   if ((e = lcsa::launch_rope_table(rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, D, s)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "rope table launch");
   noalloc_row_ptr_kernel<<<1, 32, 0, s>>>(row_ptr, g, radius, ng.topk);
@@ -216,6 +221,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.norm_scope = cfg->norm_scope;
   k1.eps = cfg->rms_eps;
   k1.err = err;
+  k1.split_part = split_part;
+  k1.split_cnt = split_cnt;
   if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "device attributes");
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
@@ -231,6 +238,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.radius = radius;
   k2.topk = ng.topk;
   k2.sort_n = sort_n;
+  k2.clear_cnt = split_cnt;
+  k2.n_clear = lcsa::kMaxK1Ctas;
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
 
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));

@@ -32,6 +32,9 @@ SMALL = {
                                topk=2, field=True, unit_gain=False, seed=2),
     "ragged_rows": _T.replace(heads=4, q_frames=1, kv_frames=2, grid_h=56, grid_w=16, block_w=16, local_range=3,
                               topk=4, field=True, unit_gain=False, seed=3),
+    # 192 blocks > one CTA per SM: K1 cuts blocks between CTAs and merges their pooled parts
+    "k1_split_blocks": _T.replace(heads=2, q_frames=1, kv_frames=2, grid_h=64, grid_w=128, block_w=16,
+                                  local_range=3, topk=4, kv_frame_offset=1, field=True, unit_gain=False, seed=5),
     "budget_from_ratio": _T.replace(heads=2, q_frames=2, kv_frames=6, grid_h=48, grid_w=80, block_w=16,
                                     local_range=11, topk=0, sparse_ratio=0.25, field=True, unit_gain=False, seed=4),
 }
