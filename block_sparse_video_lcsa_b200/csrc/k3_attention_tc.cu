@@ -68,7 +68,7 @@ constexpr uint32_t kTileBytes = kNB * kD * 2;   // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2; // 64 columns of a tile
 constexpr int kThreads = 352;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kPolyEvery = 4;  // one exponential in kPolyEvery on the FMA pipe
+constexpr int kPolyEvery = 4;  // one pair of exponentials in kPolyEvery on the FMA pipe
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 384, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
@@ -262,21 +262,29 @@ __device__ __forceinline__ float exp2_mufu(float x) {
   return y;
 }
 
-// 2^x for x <= 8 (Cody-Waite): n = round(x) through the 1.5 * 2^23 shifter,
-// f = x - n, 2^f by the polynomial, 2^n added to the exponent field. Inputs
-// below -125 are clamped (the result, < 2^-124, is negligible next to the
-// row maximum's weight of at least 1).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
+// 2^x for x <= 8 on a pair of values, packed fp32x2 arithmetic (Cody-Waite):
+// n = round(x) through the 1.5 * 2^23 shifter, f = x - n, 2^f by the
+// polynomial, 2^n added to the exponent field. Inputs below -125 are clamped
+// (the result, < 2^-124, is negligible next to the row maximum's weight of at
+// least 1).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float shifter = 12582912.0f;
-  const float t = x + shifter;
-  const float n = t - shifter;
-  const float f = x - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  const uint32_t ni = __float_as_uint(t) - 0x4B400000u;
-  return __uint_as_float(__float_as_uint(p) + (ni << 23));
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(shifter, shifter));
+  const float2 n = __fadd2_rn(t, make_float2(-shifter, -shifter));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + ((__float_as_uint(t.x) - 0x4B400000u) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + ((__float_as_uint(t.y) - 0x4B400000u) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Wait of a whole warp: every lane waits, and the warp fails as one if any
@@ -288,8 +296,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 r = exp2_poly2(make_float2(x[i], i + 1 < n ? x[i + 1] : 0.0f));
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
 }
 
 // ---- the kernel -----------------------------------------------------------
@@ -481,15 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_addr + kColS + sb * 128 + half * 64, sr[0]);
         tmem_ld32(lane_addr + kColS + sb * 128 + half * 64 + 32, sr[1]);
         tmem_wait_ld();
+        // row maximum of this half: 8 independent chains of three-input max
+        auto sv = [&](int e) { return __uint_as_float(sr[e >> 5][e & 31]); };
         float mk[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mk[a] = fmaxf(__uint_as_float(sr[0][a]), __uint_as_float(sr[0][a + 8]));
-#pragma unroll
-        for (int e = 16; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(sr[0][e]));
-#pragma unroll
-        for (int e = 0; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(sr[1][e]));
-        const float mpart = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
-                                  fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
+        for (int a = 0; a < 8; ++a) {
+          mk[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
+          mk[a] = fmax3(mk[a], sv(a + 24), sv(a + 32));
+          mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
+          mk[a] = fmaxf(mk[a], sv(a + 56));
+        }
+        const float mpart = fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
         float* slot = xmax + (j & 1) * 256;
         slot[half * 128 + row_in_tile] = mpart;
         mbar_arrive(bar(bars->pair[sp]));
@@ -507,22 +520,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         const float mneg = -m_used;
         uint32_t pk[32];
-        float rs[8];
+        float2 rs2[4];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+        for (int a = 0; a < 4; ++a) rs2[a] = make_float2(0.f, 0.f);
+        const float2 c2 = make_float2(c, c), m2 = make_float2(mneg, mneg);
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[q2][e]), c, mneg);
-            const float x1 = fmaf(__uint_as_float(sr[q2][e + 1]), c, mneg);
-            const float p0 = exp2_mufu(x0);
-            const float p1 = ((e + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x1) : exp2_mufu(x1);
-            rs[(e >> 1) & 7] += p0 + p1;
-            pk[q2 * 16 + (e >> 1)] = pack_bf16(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[q2][e]), __uint_as_float(sr[q2][e + 1])), c2, m2);
+            const float2 pp = ((e >> 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly2(x)
+                                                                         : make_float2(exp2_mufu(x.x), exp2_mufu(x.y));
+            rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], pp);
+            pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
           }
         }
-        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        l += rsum.x + rsum.y;
         // O is touched only to rescale it, once every earlier P.V has
         // completed; the last of them is P.V number gp = s_it - 1. P.V number
         // gp + 2 needs a P this warp has not written yet, so the parity wait
@@ -620,7 +634,7 @@ EncodeTiled encoder() {
 bool attention_tc_supported(const Grid& g) { return g.nb == kNB; }
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s) {
-  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  exp2_selftest_kernel<<<(n + 511) / 512, 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 
