@@ -13,8 +13,9 @@
 // Determinism: a score is the fp32 sum of four products per lane followed by
 // a butterfly over the warp; every lane ends with the same bits, and the order
 // never depends on timing. The sort key is (order-preserving score bits << 32)
-// | (~block index), so one descending sort of unique keys gives the k best
-// with ties broken toward the lower index. The CSR row offsets depend only on
+// | (~candidate number); candidates run in ascending block order, so one
+// descending sort of unique keys gives the k best with ties broken toward the
+// lower block index. The CSR row offsets depend only on
 // the geometry and are computed once when the plan is made.
 #include "lcsa_internal.h"
 
@@ -49,38 +50,47 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   const int nh = h1 - h0 + 1, nw = w1 - w0 + 1, per = nh * nw;
   const int nc = (g.nKB / g.bpf) * per;  // admissible blocks, ascending index order
 
+  // Candidate c (ascending block order) -> block index, with exact divisions
+  // by the row's constants: floor(c / d) = (c * ceil(2^32 / d)) >> 32 while
+  // c * d < 2^32 (here both are below 2^13).
+  auto magic = [](int d) { return 0xFFFFFFFFull / unsigned(d) + 1ull; };
+  auto fdiv = [](int c, unsigned long long m) { return int((unsigned long long)unsigned(c) * m >> 32); };
+  const unsigned long long m_per = magic(per), m_nw = magic(nw);
+  auto cand_block = [&](int c) {
+    const int tk = fdiv(c, m_per), r2 = c - tk * per;
+    const int hr = fdiv(r2, m_nw), wr = r2 - hr * nw;
+    return tk * g.bpf + (h0 + hr) * g.nWb + (w0 + wr);
+  };
+
   const float4 qv = reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * kHeadDim)[lane];
   const float4* pk = reinterpret_cast<const float4*>(p.pooled_k + int64_t(bh) * g.nKB * kHeadDim);
 
   if (blockIdx.x == 0)
     for (int c = threadIdx.x; c < p.n_clear; c += kThreads) p.clear_cnt[c] = 0u;
-  for (int c = threadIdx.x; c < p.sort_n; c += kThreads) flag[c] = 0;
-  for (int c0 = warp * kCandPerIter; c0 < p.sort_n; c0 += kWarps * kCandPerIter) {
+  for (int c = threadIdx.x; c < p.sort_n; c += kThreads) {
+    flag[c] = 0;
+    if (c >= nc) keys[c] = 0ull;  // padding sorts last
+  }
+  // Sort key: (order-preserving score bits << 32) | ~c, so equal scores go to
+  // the lower candidate, i.e. the lower block index.
+  for (int c0 = warp * kCandPerIter; c0 < nc; c0 += kWarps * kCandPerIter) {
     float4 kv[kCandPerIter];
-    int kb[kCandPerIter];
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
       const int c = c0 + u;
-      kb[u] = -1;
-      kv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c < nc) {
-        const int tk = c / per, r2 = c % per;
-        kb[u] = tk * g.bpf + (h0 + r2 / nw) * g.nWb + (w0 + r2 % nw);
-        kv[u] = pk[int64_t(kb[u]) * (kHeadDim / 4) + lane];
-      }
+      kv[u] = c < nc ? pk[int64_t(cand_block(c)) * (kHeadDim / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
+      const int c = c0 + u;
+      if (c >= nc) break;  // warp-uniform
       float s = qv.x * kv[u].x;
       s = fmaf(qv.y, kv[u].y, s);
       s = fmaf(qv.z, kv[u].z, s);
       s = fmaf(qv.w, kv[u].w, s);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const int c = c0 + u;
-      if (lane == 0 && c < p.sort_n)
-        keys[c] = kb[u] >= 0 ? ((unsigned long long)order_bits(s) << 32) | (0xFFFFFFFFu - unsigned(kb[u]))
-                             : 0ull;
+      if (lane == 0) keys[c] = ((unsigned long long)order_bits(s) << 32) | (0xFFFFFFFFu - unsigned(c));
     }
   }
   __syncthreads();
@@ -106,12 +116,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
 
   // mark the kept candidates, then compact them in ascending block order
   const int keff = min(p.topk, nc);
-  for (int i = threadIdx.x; i < keff; i += kThreads) {
-    const int kbi = int(0xFFFFFFFFu - unsigned(keys[i] & 0xFFFFFFFFull));
-    const int tk = kbi / g.bpf, r2 = kbi % g.bpf;
-    const int c = (tk * nh + (r2 / g.nWb - h0)) * nw + (r2 % g.nWb - w0);
-    flag[c] = 1;
-  }
+  for (int i = threadIdx.x; i < keff; i += kThreads) flag[0xFFFFFFFFu - unsigned(keys[i] & 0xFFFFFFFFull)] = 1;
   __syncthreads();
   const int span = (nc + kThreads - 1) / kThreads;
   const int c_beg = threadIdx.x * span, c_end = min(c_beg + span, nc);
@@ -129,10 +134,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   for (int w = 0; w < warp; ++w) base += warp_sum[w];
   int pos = p.row_ptr[rr] + base + incl - cnt;
   for (int c = c_beg; c < c_end; ++c) {
-    if (flag[c]) {
-      const int tk = c / per, r2 = c % per;
-      p.col_idx[pos++] = tk * g.bpf + (h0 + r2 / nw) * g.nWb + (w0 + r2 % nw);
-    }
+    if (flag[c]) p.col_idx[pos++] = cand_block(c);
   }
 }
 
