@@ -25,6 +25,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCandPerIter = 4;  // candidates in flight per warp
+constexpr int kRankMax = 512;    // admissible sets up to this size: rank selection, else bitonic sort
 
 __device__ __forceinline__ unsigned order_bits(float s) {
   const unsigned u = __float_as_uint(s + 0.0f);  // -0 -> +0
@@ -32,7 +33,7 @@ __device__ __forceinline__ unsigned order_bits(float s) {
 }
 
 __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
-  extern __shared__ unsigned long long keys[];  // [sort_n], then flags [sort_n] bytes
+  extern __shared__ __align__(16) unsigned long long keys[];  // [sort_n], then flags [sort_n] bytes
   unsigned char* flag = reinterpret_cast<unsigned char*>(keys + p.sort_n);
   __shared__ int warp_sum[kWarps];
   const Grid& g = p.g;
@@ -95,28 +96,42 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   }
   __syncthreads();
 
-  // bitonic sort, descending
-  const int n = p.sort_n;
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += kThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], bk = keys[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (a < bk) : (a > bk)) {
-            keys[i] = bk;
-            keys[ixj] = a;
+  const int keff = min(p.topk, nc);
+  if (nc <= kRankMax) {
+    // rank selection: candidate c is kept when fewer than k keys beat it (keys
+    // are unique); every thread reads the same key at each step (broadcast)
+    for (int c = threadIdx.x; c < nc; c += kThreads) {
+      const unsigned long long mine = keys[c];
+      int above = 0;
+      int j = 0;
+      for (; j + 1 < nc; j += 2) {
+        const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(keys + j);
+        above += (kk.x > mine) + (kk.y > mine);
+      }
+      if (j < nc) above += keys[j] > mine;
+      flag[c] = above < keff;
+    }
+  } else {
+    // bitonic sort, descending, then mark the first k
+    const int n = p.sort_n;
+    for (int k = 2; k <= n; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long a = keys[i], bk = keys[ixj];
+            const bool desc = (i & k) == 0;
+            if (desc ? (a < bk) : (a > bk)) {
+              keys[i] = bk;
+              keys[ixj] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
+    for (int i = threadIdx.x; i < keff; i += kThreads) flag[0xFFFFFFFFu - unsigned(keys[i] & 0xFFFFFFFFull)] = 1;
   }
-
-  // mark the kept candidates, then compact them in ascending block order
-  const int keff = min(p.topk, nc);
-  for (int i = threadIdx.x; i < keff; i += kThreads) flag[0xFFFFFFFFu - unsigned(keys[i] & 0xFFFFFFFFull)] = 1;
   __syncthreads();
   const int span = (nc + kThreads - 1) / kThreads;
   const int c_beg = threadIdx.x * span, c_end = min(c_beg + span, nc);
