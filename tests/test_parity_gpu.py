@@ -121,3 +121,51 @@ def test_full_size_workload(name):
     assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
     np.testing.assert_allclose(gpu.pooled_q, pq, rtol=1e-5, atol=2e-5)
     np.testing.assert_allclose(gpu.pooled_k, pk, rtol=1e-5, atol=2e-5)
+
+
+# Exact score ties. k is zero in the first two KV frames, so every block there
+# scores exactly 0 in both the oracle and the kernel; k (the budget) is larger
+# than the number of positive scores, so the cut falls inside that tie group
+# and the lower block index decides. The near-tie exemption of check_selection
+# does not apply: the CSR must equal the oracle's bit for bit.
+TIES = {
+    # 18 admissible blocks per row (a small window)
+    "ties_window": _T.replace(heads=2, q_frames=1, kv_frames=4, grid_h=32, grid_w=64, block_w=16, local_range=3,
+                            topk=10, kv_frame_offset=3, field=True, unit_gain=False, seed=6),
+    # 576 admissible blocks per row (no window)
+    "ties_unbounded": _T.replace(heads=1, q_frames=1, kv_frames=4, grid_h=72, grid_w=256, block_w=16, local_range=0,
+                             topk=300, kv_frame_offset=3, field=True, unit_gain=False, seed=7),
+}
+
+
+@pytest.mark.parametrize("name", list(TIES))
+def test_exact_ties_go_to_the_lower_block(name):
+    import dataclasses
+    wl = TIES[name]
+    inp = synth.make_inputs(wl)
+    og = oracle_geometry(wl)
+    plane = wl.grid_h * wl.grid_w
+    k = inp.k.copy()
+    k[:, : 2 * plane, :] = 0                      # bf16 +0: frames 0 and 1
+    inp = dataclasses.replace(inp, k=k)
+    gpu = run_gpu(wl, inp)
+    pq = oracle.pool(og, inp.q, inp.gamma_q, True)
+    pk = oracle.pool(og, inp.k, inp.gamma_k, False)
+    sel = oracle.select(og, pq, pk, want_scores=True)
+    per_frame = og.nKB // wl.kv_frames
+    zero_blocks = 2 * per_frame
+    # the cut lies inside the zero-score group in at least some rows
+    cut_in_ties = [r for r in range(og.rows) if sel.gap[r] == 0.0]
+    assert cut_in_ties, "the workload no longer puts the cut inside the tie group"
+    for r in cut_in_ties[:3]:
+        row = sel.row(r)
+        zeros = row[row < zero_blocks]
+        tied = np.flatnonzero(sel.scores[r] == 0.0)   # admissible blocks that score exactly 0
+        assert np.array_equal(zeros, tied[: zeros.size]), "oracle: ties must go to the lowest blocks"
+    row_ptr, col = sel.csr()
+    np.testing.assert_array_equal(gpu.row_ptr.astype(np.int64), row_ptr)
+    np.testing.assert_array_equal(gpu.col_idx, col)
+    rows = sample_rows(og, 16)
+    out, wsum = oracle.attention(og, inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, sel, rows)
+    mx, mean = check_output(og, gpu, rows, out)
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
