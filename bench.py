@@ -318,7 +318,7 @@ def run_lcsa(args):
     value = world * flops / (ms_per_step * 1e-3) / 1e12
     k3_tflops = flops / (kms[2] * 1e-3) / 1e12
     k1_gbs = geo.prologue_bytes / (kms[0] * 1e-3) / 1e9
-    k3_src = "k3_attention_tc.cu" if geo.block_tokens == 128 else "k3_attention_mma.cu"
+    k3_src = "k3_attention_tc.cu"
     traffic = _profiled_traffic("k3", [k3_src, "lcsa_internal.h"])
     roofline = {"bound": "tensor", "kernel": "attention (K3, %s)" % k3_src, "achieved": k3_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": k3_tflops / peaks["bf16_tflops"], "traffic": traffic,

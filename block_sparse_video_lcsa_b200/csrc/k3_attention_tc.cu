@@ -1,5 +1,12 @@
 // K3 (tcgen05 form): block-sparse flash attention over the CSR list with the
-// 5th-generation tensor cores, tensor memory and TMA, for 128-token blocks.
+// 5th-generation tensor cores, tensor memory and TMA, for 128- and 64-token
+// blocks. A KV tile is always 128 keys: one 128-token block, or two
+// consecutive selected 64-token blocks (an odd last tile repeats its block and
+// the softmax zeroes the copy). With 64-token blocks the query tile is 64 rows
+// and the products are M = 64 (measured on this part: M64 N128 K16 issues every
+// 64 cycles, half the rate of M128 N128 K16; M64 N64 K16 every 51), whose
+// accumulators hold row m in TMEM lane 32 (m / 16) + m % 16, so only lanes
+// 0-15 of each softmax warp carry rows.
 //
 // Pages: "FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408", Rebuild sparse
 // attention for Hopper: a warp-specialised producer/consumer path with TMA
@@ -60,7 +67,7 @@
 namespace lcsa {
 namespace {
 
-constexpr int kNB = 128;                    // tokens per query / KV block
+constexpr int kNB = 128;                    // keys per KV tile (one 128-token block or two 64-token blocks)
 constexpr int kD = 128;                     // head_dim
 constexpr int kKStages = 2;
 constexpr int kVStages = 3;
@@ -201,9 +208,9 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,
-// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M = N = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), N = 128, M = 128 or 64.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t b_mn, uint32_t m = 128) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((128u >> 3) << 17) | ((m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -305,6 +312,10 @@ __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
 
 // ---- the kernel -----------------------------------------------------------
 
+// QM = tokens per query block (128, or 64: then each KV tile holds two
+// consecutive selected 64-token blocks and the M = 64 accumulators use TMEM
+// lanes 0-15 of each lane quarter).
+template <int QM>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
@@ -316,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = p.g;
+  constexpr int KB = kNB / QM;  // selected blocks per KV tile
 
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
@@ -365,42 +377,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = bhh / g.Hn, h = bhh % g.Hn;
         if (row_it > 0) ok = mbar_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1);
         if (!ok) break;
-        mbar_expect_tx(bar(bars->q_full), kTileBytes);
-        tma_load_2d(base + kOffQ, &tm_q, 0, rr * kNB, bar(bars->q_full));
-        tma_load_2d(base + kOffQ + kHalfBytes, &tm_q, 64, rr * kNB, bar(bars->q_full));
-        auto load_k = [&](int j) -> bool {
-          const int kb = p.col_idx[beg + j];
-          const int kvj = kv + j, ks = kvj % kKStages, ku = kvj / kKStages;
+        mbar_expect_tx(bar(bars->q_full), QM * kD * 2);
+        tma_load_2d(base + kOffQ, &tm_q, 0, rr * QM, bar(bars->q_full));
+        tma_load_2d(base + kOffQ + QM * 128, &tm_q, 64, rr * QM, bar(bars->q_full));
+        const int steps = (n + KB - 1) / KB;
+        // the selected block feeding sub-tile i of step st (an odd last step
+        // repeats its block; the softmax masks the copy)
+        auto step_block = [&](int st, int i) { return p.col_idx[beg + min(st * KB + i, n - 1)]; };
+        auto load_k = [&](int st) -> bool {
+          const int kvj = kv + st, ks = kvj % kKStages, ku = kvj / kKStages;
           if (ku > 0 && !mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
           const uint32_t kdst = base + kOffK + ks * kTileBytes;
           mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
-          tma_load_2d(kdst, &tm_k, 0, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
-          tma_load_2d(kdst + kHalfBytes, &tm_k, 64, (bhh * g.nKB + kb) * kNB, bar(bars->k_full[ks]));
+#pragma unroll
+          for (int i = 0; i < KB; ++i) {
+            const int kb = step_block(st, i);
+            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, (bhh * g.nKB + kb) * QM, bar(bars->k_full[ks]));
+            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, (bhh * g.nKB + kb) * QM, bar(bars->k_full[ks]));
+          }
           return true;
         };
-        for (int j = 0; j < 2 && j < n && ok; ++j) ok = load_k(j);
-        for (int j = 0; j < n && ok; ++j) {
-          if (j + 2 < n && !(ok = load_k(j + 2))) break;
-          const int kb = p.col_idx[beg + j];
-          const int kvj = kv + j, vs = kvj % kVStages, vu = kvj / kVStages;
+        for (int st = 0; st < 2 && st < steps && ok; ++st) ok = load_k(st);
+        for (int st = 0; st < steps && ok; ++st) {
+          if (st + 2 < steps && !(ok = load_k(st + 2))) break;
+          const int kvj = kv + st, vs = kvj % kVStages, vu = kvj / kVStages;
           if (vu > 0 && !(ok = mbar_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
-          const int tb = kb / g.bpf, rem = kb % g.bpf;
-          const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
           const uint32_t vdst = base + kOffV + vs * kTileBytes;
           mbar_expect_tx(bar(bars->v_full[vs]), kTileBytes);
-          tma_load_5d(vdst, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
-          tma_load_5d(vdst + kHalfBytes, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
+#pragma unroll
+          for (int i = 0; i < KB; ++i) {
+            const int kb = step_block(st, i);
+            const int tb = kb / g.bpf, rem = kb % g.bpf;
+            const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
+            tma_load_5d(vdst + i * QM * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
+            tma_load_5d(vdst + kHalfBytes + i * QM * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
+          }
         }
-        kv += n;
+        kv += steps;
       }
     }
   } else if (warp == 1) {
     // ---------------- S issuer (converged warp, lane 0 issues) ----------------
-    constexpr uint32_t id_qk = idesc_bf16(0);
+    constexpr uint32_t id_qk = idesc_bf16(0, QM);
     int kv = 0, s_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n = (p.row_ptr[rr + 1] - p.row_ptr[rr] + KB - 1) / KB;  // KV tiles of the row
       if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
       for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
@@ -415,8 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_ss(tmem + kColS + sb * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk,
+            const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (QM * 128) + (kk & 3) * 32;
+            mma_ss(tmem + kColS + sb * 128, sdesc(qa + qoff, 16, 1024), sdesc(ka + koff, 16, 1024), id_qk,
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(bars->s_full[sb]));
@@ -435,11 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ---------------- P.V issuer (converged warp, lane 0 issues) ----------------
-    constexpr uint32_t id_pv = idesc_bf16(1);
+    constexpr uint32_t id_pv = idesc_bf16(1, QM);
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n = (p.row_ptr[rr + 1] - p.row_ptr[rr] + KB - 1) / KB;  // KV tiles of the row
       for (int j = 0; j < n; ++j, ++pv_it) {
         const int pb = pv_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
@@ -474,7 +497,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- softmax / correction / epilogue ----------------
     const int sp = warp & 3;                 // TMEM lane quarter of this warp
     const int half = (warp - 3) >> 2;        // which 64 key columns / channels
-    const int row_in_tile = sp * 32 + lane;  // query token index inside the block
+    const int row_in_tile = sp * 32 + lane;  // exchange slot of this lane's row
+    // query token of this lane: M = 128 uses every lane, M = 64 lanes 0-15 of each quarter
+    const bool active = QM == 128 || lane < 16;
+    const int m_tok = QM == 128 ? row_in_tile : sp * 16 + (lane & 15);
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
     float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
     float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
@@ -482,9 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_it = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
-      const int n = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n_sel = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n = (n_sel + KB - 1) / KB;  // KV tiles of the row
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j, ++s_it) {
+        // an odd last tile of 64-token blocks repeats its block in keys 64-127
+        const bool masked = KB == 2 && half == 1 && 2 * j + 1 >= n_sel;
         const int sb = s_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
@@ -502,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
           mk[a] = fmaxf(mk[a], sv(a + 56));
         }
-        const float mpart = fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+        const float mpart =
+            masked ? -INFINITY : fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
         float* slot = xmax + (j & 1) * 256;
         slot[half * 128 + row_in_tile] = mpart;
         mbar_arrive(bar(bars->pair[sp]));
@@ -511,9 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mx = fmaxf(mpart, slot[(half ^ 1) * 128 + row_in_tile]);
         const float m_new = fmaxf(m_used, mx * c);
         const bool need = m_new > m_used + kRescaleLog2;
-        const bool warp_need = __any_sync(0xffffffffu, need);
+        const bool warp_need = __any_sync(0xffffffffu, need && active);
         float alpha = 1.f;
-        if (need) {
+        if (need && active) {
           alpha = exp2_mufu(m_used - m_new);
           m_used = m_new;
         }
@@ -535,8 +565,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
           }
         }
-        const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-        l += rsum.x + rsum.y;
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = 0u;
+        } else {
+          const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+          l += rsum.x + rsum.y;
+        }
         // O is touched only to rescale it, once every earlier P.V has
         // completed; the last of them is P.V number gp = s_it - 1. P.V number
         // gp + 2 needs a P this warp has not written yet, so the parity wait
@@ -554,6 +589,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(oa, o);
+          }
+        }
+        // M = 64 tiles: P is stored only once the preceding P.V has completed,
+        // and lanes without a row store zeros. With P stores overlapping an
+        // in-flight M = 64 P.V, outputs varied from run to run on this part
+        // (fewer differences with zeros in the unused lanes, none with the
+        // wait), although isolated M = 64 products read and write lanes 0-15
+        // of each quarter only. The M = 128 path shows no such effect.
+        if (QM == 64) {
+          if (!active) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
+          }
+          if (j >= 1 && !warp_need) {
+            const int gp = s_it - 1;
+            if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 26))) break;
+            tc_fence_after();
           }
         }
         tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
@@ -578,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bhh = rr / g.nQB, qb = rr % g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       const int tb = qb / g.bpf, rem = qb % g.bpf;
-      const int tt = row_in_tile / (g.bh * g.bw), yy = (row_in_tile / g.bw) % g.bh, xx = row_in_tile % g.bw;
+      const int tt = m_tok / (g.bh * g.bw), yy = (m_tok / g.bw) % g.bh, xx = m_tok % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
       __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + half * 64;
 #pragma unroll
@@ -592,8 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
+        if (active) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d4[e] = v[e];
+          for (int e = 0; e < 4; ++e) d4[e] = v[e];
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -631,19 +685,19 @@ EncodeTiled encoder() {
 
 }  // namespace
 
-bool attention_tc_supported(const Grid& g) { return g.nb == kNB; }
+bool attention_tc_supported(const Grid& g) { return g.nb == 128 || g.nb == 64; }
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s) {
   exp2_selftest_kernel<<<(n + 511) / 512, 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 
-cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows) {
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
   EncodeTiled enc = encoder();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(kD * 2)};
-  const cuuint32_t box[2] = {64, cuuint32_t(kNB)};
+  const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -668,8 +722,9 @@ cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
 
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s) {
-  cudaError_t e =
-      cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  if (!attention_tc_supported(p.g)) return cudaErrorInvalidValue;
+  auto kern = p.g.nb == 128 ? attention_tc_kernel<128> : attention_tc_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
   TcParams tp;
   tp.g = p.g;
@@ -680,7 +735,7 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.err = p.err;
   tp.rows = p.g.B * p.g.Hn * p.g.nQB;
   const int grid = tp.rows < num_sms ? tp.rows : num_sms;
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
+  kern<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();
 }
 

@@ -210,7 +210,6 @@ struct lcsa_plan {
   float* st_gq = nullptr;
   float* st_gk = nullptr;
   // tcgen05 attention: tensor maps of the plan-owned q^ / k^; SM count (persistent grids)
-  bool use_tc = false;
   CUtensorMap tm_q, tm_k;
   int num_sms = 0;
   std::vector<std::array<cudaEvent_t, 4>> evsets;  // timing ring
@@ -344,10 +343,9 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
     delete p;
     return cuda_fail(e, "device attributes");
   }
-  p->use_tc = lcsa::attention_tc_supported(g);
-  if (p->use_tc) {
-    if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&p->tm_k, p->khat, int64_t(g.B) * g.Hn * g.nKB * g.nb)) != cudaSuccess) {
+  {
+    if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||
+        (e = lcsa::make_block_map(&p->tm_k, p->khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb)) != cudaSuccess) {
       release(p);
       delete p;
       return cuda_fail(e, "tensor maps");
@@ -427,13 +425,11 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
-  if (p->use_tc) {
+  {
     CUtensorMap tm_v;
     if ((e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
       return cuda_fail(e, "attention launch");
-  } else if ((e = lcsa::launch_attention_mma(k3, s)) != cudaSuccess) {
-    return cuda_fail(e, "attention launch");
   }
   if (ev) {
     if ((e = cudaEventRecord(ev[3], s)) != cudaSuccess) return cuda_fail(e, "event");

@@ -99,13 +99,13 @@ cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, in
 cudaError_t launch_prologue(const K1Params& p, cudaStream_t s);
 size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
-cudaError_t launch_attention_mma(const K3Params& p, cudaStream_t s);
 
-// tcgen05 attention (128-token blocks). Tensor maps: q^ / k^ as [rows][128]
-// bf16 tiles of 128 rows (make_block_map), V through its raster layout
+// tcgen05 attention (128- or 64-token blocks). Tensor maps: q^ / k^ as
+// [rows][128] bf16 with boxes of 64 columns x one block of rows
+// (make_block_map, box_rows = tokens per block), V through its raster layout
 // (make_raster_map). The kernel is persistent over min(rows, num_sms) CTAs.
 bool attention_tc_supported(const Grid& g);
-cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows);
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g);
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,

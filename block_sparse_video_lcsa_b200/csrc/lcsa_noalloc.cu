@@ -253,17 +253,15 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.col_idx = col_idx;
   k3.scale_log2 = scale * 1.4426950408889634f;
   k3.err = err;
-  if (lcsa::attention_tc_supported(g)) {
+  {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
-    if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb)) != cudaSuccess ||
+    if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||
+        (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb)) != cudaSuccess ||
         (e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess)
       return noalloc_fail(LCSA_ERR_CUDA, "tensor maps");
     if ((e = lcsa::launch_attention_tc(k3, tm_q, tm_k, tm_v, num_sms, s)) != cudaSuccess)
       return noalloc_fail(LCSA_ERR_CUDA, "attention launch");
-  } else if ((e = lcsa::launch_attention_mma(k3, s)) != cudaSuccess) {
-    return noalloc_fail(LCSA_ERR_CUDA, "attention launch");
   }
   return LCSA_OK;
 }
