@@ -78,6 +78,9 @@ SIGNATURES = [
     ("lcsa_forward", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_forward_host", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_forward_noalloc", _I, [ctypes.POINTER(lcsa_config_t), _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_plan_create_stream", _I, [ctypes.POINTER(lcsa_config_t), _I, ctypes.POINTER(_PLAN)]),
+    ("lcsa_stream_push", _I, [_PLAN, _VP, _VP, _VP, _I, _VP]),
+    ("lcsa_forward_stream", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_plan_geometry", _I, [_PLAN, ctypes.POINTER(lcsa_geometry_t)]),
     ("lcsa_plan_topk", _I, [_PLAN, ctypes.POINTER(_I)]),
     ("lcsa_get_selection", _I, [_PLAN, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t]),
@@ -160,6 +163,14 @@ def lcsa_plan_create(cfg: lcsa_config_t, device: int = 0) -> "Plan":
     return Plan(h, cfg)
 
 
+def lcsa_plan_create_stream(cfg: lcsa_config_t, device: int = 0) -> "Plan":
+    """A stream plan: the last kv_frames frames of k^, pooled k and v stay in a
+    ring; feed it with Plan.lcsa_stream_push and Plan.lcsa_forward_stream."""
+    h = _PLAN()
+    _check(lib().lcsa_plan_create_stream(ctypes.byref(cfg), int(device), ctypes.byref(h)), "lcsa_plan_create_stream")
+    return Plan(h, cfg)
+
+
 LCSA_NOALLOC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -230,6 +241,29 @@ class Plan:
         return out
 
     forward = lcsa_forward
+
+    def lcsa_stream_push(self, k, v, gamma_k, frames, stream=None):
+        """Append `frames` frames of k and v ([batch, frames * H' * W', heads*d]) to the window."""
+        import torch
+        c, g = self.cfg, self.geometry
+        toks = frames * c.grid_h * c.grid_w
+        self._expect(k, torch.bfloat16, (c.batch, toks, g.channels), "k")
+        self._expect(v, torch.bfloat16, (c.batch, toks, g.channels), "v")
+        self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k")
+        _check(lib().lcsa_stream_push(self._h, _addr(k), _addr(v), _addr(gamma_k), int(frames), _stream(stream)),
+               "lcsa_stream_push")
+
+    def lcsa_forward_stream(self, q, k, v, gamma_q, gamma_k, out, stream=None):
+        """One stream chunk: q, k, v of the q_frames new frames ([batch, q_tokens, heads*d])."""
+        import torch
+        c, g = self.cfg, self.geometry
+        for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+            self._expect(t, torch.bfloat16, (c.batch, g.q_tokens, g.channels), name)
+        self._expect(gamma_q, torch.float32, (g.channels,), "gamma_q")
+        self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k")
+        _check(lib().lcsa_forward_stream(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
+                                         _addr(out), _stream(stream)), "lcsa_forward_stream")
+        return out
 
     def lcsa_forward_host(self, q, k, v, gamma_q, gamma_k, out, stream=None):
         """Host (preferably pinned) tensors in and out; copies are inside the call."""

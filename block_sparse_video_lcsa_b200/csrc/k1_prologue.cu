@@ -113,22 +113,37 @@ __device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
-// Block number bid of the combined list (B * nQB query blocks, then B * nKB
-// key blocks) -> which tensor, batch element, block and its first token.
+// Block number bid of the combined list (the processed query blocks, then the
+// key blocks of the k input) -> tensor, batch element, output block, the
+// input frame and the KV-window frame of its first token.
 struct BlockRef {
   bool is_q;
-  int b, blk, nblk, t0, y0, x0;
+  int b, blk, nblk, t_in0, t_win0, y0, x0;
 };
-__device__ __forceinline__ BlockRef block_ref(const Grid& g, int bid) {
+__device__ __forceinline__ BlockRef block_ref(const K1Params& p, int bid) {
+  const Grid& g = p.g;
   BlockRef r;
-  const int n_qtot = g.B * g.nQB;
-  r.is_q = bid < n_qtot;
-  const int bg = r.is_q ? bid : bid - n_qtot;
-  r.nblk = r.is_q ? g.nQB : g.nKB;
-  r.b = bg / r.nblk;
-  r.blk = bg % r.nblk;
-  const int tb = r.blk / g.bpf, rem = r.blk % g.bpf;
-  r.t0 = tb * g.bt;
+  r.is_q = bid < p.n_qblk;
+  int rem;
+  if (r.is_q) {
+    r.nblk = g.nQB;
+    r.b = bid / g.nQB;
+    r.blk = bid % g.nQB;
+    const int tb = r.blk / g.bpf;
+    rem = r.blk % g.bpf;
+    r.t_in0 = tb * g.bt;
+    r.t_win0 = r.t_in0 + (g.Tkv - g.Tq);  // query frames close the KV window
+  } else {
+    const int bg = bid - p.n_qblk, per_b = p.k_in_fb * g.bpf;
+    r.nblk = g.nKB;
+    r.b = bg / per_b;
+    const int bi = bg % per_b, tb = bi / g.bpf;
+    rem = bi % g.bpf;
+    const int wfb = p.k_first_fb + tb;
+    r.t_in0 = tb * g.bt;
+    r.t_win0 = wfb * g.bt;
+    r.blk = ((p.slot0_fb + wfb) % p.ring_fb) * g.bpf + rem;
+  }
   r.y0 = (rem / g.nWb) * g.bh;
   r.x0 = (rem % g.nWb) * g.bw;
   return r;
@@ -155,7 +170,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunks = g.C / 8;
   const int R = g.bt * g.bh;  // rows per block
-  const int total = g.B * (g.nQB + g.nKB);
+  const int total = p.n_qblk + g.B * p.k_in_fb * g.bpf;
   // this CTA's rows: a contiguous range of the combined row list (blocks in
   // order, rows of a block in order); every range holds at least R rows, so a
   // block is cut by at most one range boundary
@@ -167,11 +182,11 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
   // source of the CTA's row number k (global row lo + k)
   auto row_src = [&](int k) -> const void* {
     const int64_t grow = lo + k;
-    const BlockRef br = block_ref(g, int(grow / R));
+    const BlockRef br = block_ref(p, int(grow / R));
     const int r = int(grow % R);
-    const int64_t tok = (int64_t(br.t0 + r / g.bh) * g.gh + br.y0 + r % g.bh) * g.gw + br.x0;
+    const int64_t tok = (int64_t(br.t_in0 + r / g.bh) * g.gh + br.y0 + r % g.bh) * g.gw + br.x0;
     const __nv_bfloat16* x = br.is_q ? p.q : p.k;
-    const int64_t L = br.is_q ? g.Lq : g.Lkv;
+    const int64_t L = br.is_q ? g.Lq : p.Lk_in;
     return x + (int64_t(br.b) * L + tok) * g.C;
   };
   auto issue = [&](int gi) {
@@ -206,11 +221,10 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
     const int bid = int((lo + gi) / R);
     const int r_begin = int((lo + gi) % R);
     const int r_end = min(R, r_begin + (my_rows - gi));
-    const BlockRef br = block_ref(g, bid);
+    const BlockRef br = block_ref(p, bid);
     const float4* gtab = gsm + (br.is_q ? 0 : CPL * 64);
     __nv_bfloat16* xhat = br.is_q ? p.qhat : p.khat;
     float* pooled = br.is_q ? p.pooled_q : p.pooled_k;
-    const int tshift = br.is_q ? (g.Tkv - g.Tq) : 0;
 #pragma unroll
     for (int c4 = 0; c4 < CPL; ++c4)
 #pragma unroll
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
     for (int r = r_begin; r < r_end; ++r, ++gi) {
       const int s = gi % stages;
       const bool arrived = mbar_wait_bounded(bars + 8 * s, uint32_t(gi / stages) & 1u);
-      const int t = br.t0 + r / g.bh, y = br.y0 + r % g.bh;
+      const int t = br.t_win0 + r / g.bh, y = br.y0 + r % g.bh;  // t: KV-window frame
       const uint4* row = reinterpret_cast<const uint4*>(ring + size_t(s) * row_bytes);
       for (int i = warp; i < g.bw; i += NW) {
         const int xc = br.x0 + i;
@@ -233,7 +247,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) {
           const int j = jb + qd;
-          const int idx = j < PT        ? (tshift + t) * PT + j
+          const int idx = j < PT        ? t * PT + j
                           : j < PT + PH ? p.rope_h_off + y * PH + (j - PT)
                                         : p.rope_w_off + xc * (kHeadDim / 2 - PT - PH) + (j - PT - PH);
           cs[qd] = __ldg(p.rope + idx);
@@ -398,7 +412,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
 
 template <int CPL, bool FULL, bool HEAD>
 cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
-  const int nblocks = p.g.B * (p.g.nQB + p.g.nKB);
+  const int nblocks = p.n_qblk + p.g.B * p.k_in_fb * p.g.bpf;
   if (nblocks <= 0) return cudaSuccess;
   const uint32_t row_bytes = uint32_t(p.g.bw) * uint32_t(p.g.C) * 2u;
   const uint32_t red_bytes = uint32_t(kRedRows) * uint32_t(p.g.C) * 4u + 2u * CPL * 64u * 16u;  // + gains

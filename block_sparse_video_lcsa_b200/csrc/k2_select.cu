@@ -60,10 +60,11 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   auto magic = [](int d) { return 0xFFFFFFFFull / unsigned(d) + 1ull; };
   auto fdiv = [](int c, unsigned long long m) { return int((unsigned long long)unsigned(c) * m >> 32); };
   const unsigned long long m_per = magic(per), m_nw = magic(nw);
-  auto cand_block = [&](int c) {
+  auto cand_block = [&](int c, bool ring) {
     const int tk = fdiv(c, m_per), r2 = c - tk * per;
     const int hr = fdiv(r2, m_nw), wr = r2 - hr * nw;
-    return tk * g.bpf + (h0 + hr) * g.nWb + (w0 + wr);
+    const int slot = ring ? (p.slot0_fb + tk) % p.ring_fb : tk;  // where its pooled k is stored
+    return slot * g.bpf + (h0 + hr) * g.nWb + (w0 + wr);
   };
 
   const float4 qv = reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * kHeadDim)[lane];
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
       const int c = c0 + u;
-      kv[u] = c < nc ? pk[int64_t(cand_block(c)) * (kHeadDim / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+      kv[u] = c < nc ? pk[int64_t(cand_block(c, true)) * (kHeadDim / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   for (int w = 0; w < warp; ++w) base += warp_sum[w];
   int pos = p.row_ptr[rr] + base + incl - cnt;
   for (int c = c_beg; c < c_end; ++c) {
-    if (flag[c]) p.col_idx[pos++] = cand_block(c);
+    if (flag[c]) p.col_idx[pos++] = cand_block(c, false);  // window order
   }
 }
 

@@ -112,6 +112,7 @@ static_assert(kSoftmaxWarps == 8 && kThreads == 96 + 32 * kSoftmaxWarps, "warp r
 
 struct TcParams {
   Grid g;
+  int ring_fb, slot0_fb;
   const int* row_ptr;
   const int* col_idx;
   __nv_bfloat16* out;
@@ -384,6 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the selected block feeding sub-tile i of step st (an odd last step
         // repeats its block; the softmax masks the copy)
         auto step_block = [&](int st, int i) { return p.col_idx[beg + min(st * KB + i, n - 1)]; };
+        // window block -> its k^ block in the ring
+        auto ring_block = [&](int kb) { return ((p.slot0_fb + kb / g.bpf) % p.ring_fb) * g.bpf + kb % g.bpf; };
         auto load_k = [&](int st) -> bool {
           const int kvj = kv + st, ks = kvj % kKStages, ku = kvj / kKStages;
           if (ku > 0 && !mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
@@ -392,8 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < KB; ++i) {
             const int kb = step_block(st, i);
-            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, (bhh * g.nKB + kb) * QM, bar(bars->k_full[ks]));
-            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, (bhh * g.nKB + kb) * QM, bar(bars->k_full[ks]));
+            const int kp = ring_block(kb);
+            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, (bhh * g.nKB + kp) * QM, bar(bars->k_full[ks]));
+            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, (bhh * g.nKB + kp) * QM, bar(bars->k_full[ks]));
           }
           return true;
         };
@@ -407,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < KB; ++i) {
             const int kb = step_block(st, i);
-            const int tb = kb / g.bpf, rem = kb % g.bpf;
+            const int tb = (p.slot0_fb + kb / g.bpf) % p.ring_fb, rem = kb % g.bpf;  // ring slot of its frame-block
             const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
             tma_load_5d(vdst + i * QM * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
             tma_load_5d(vdst + kHalfBytes + i * QM * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
@@ -734,6 +738,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.scale_log2 = p.scale_log2;
   tp.err = p.err;
   tp.rows = p.g.B * p.g.Hn * p.g.nQB;
+  tp.ring_fb = p.ring_fb;
+  tp.slot0_fb = p.slot0_fb;
   const int grid = tp.rows < num_sms ? tp.rows : num_sms;
   kern<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();

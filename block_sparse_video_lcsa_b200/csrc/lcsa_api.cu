@@ -195,6 +195,9 @@ struct lcsa_plan {
   __nv_bfloat16* khat = nullptr;
   float* pooled_q = nullptr;
   float* pooled_k = nullptr;
+  bool streaming = false;          // made by lcsa_plan_create_stream
+  __nv_bfloat16* v_ring = nullptr; // stream plans: raw v of the window, [B][Tkv slots][H'][W'][C]
+  int64_t pushed_fb = 0;           // stream plans: frame-blocks pushed so far
   float* split_part = nullptr;     // K1: partial pooled sums of blocks cut between CTAs
   unsigned* split_cnt = nullptr;   // K1: arrivals per cut (K2 zeroes them after use)
   int32_t* row_ptr = nullptr;
@@ -219,7 +222,7 @@ struct lcsa_plan {
 namespace {
 
 void release(lcsa_plan* p) {
-  void* ptrs[] = {p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
+  void* ptrs[] = {p->v_ring, p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
                   p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
                   p->st_v,  p->st_out,  p->st_gq,    p->st_gk};
   for (void* q : ptrs)
@@ -363,18 +366,24 @@ void lcsa_plan_destroy(lcsa_plan_t p) {
   delete p;
 }
 
-lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
-                           const float* gamma_k, void* out, void* stream) {
-  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
-  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(gamma_q) ||
-      !aligned16(gamma_k))
-    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaSetDevice(p->device);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
-  const lcsa::Grid& g = p->res.grid;
+namespace {
 
+// Which frames one launch sequence covers. The stateless call: the whole
+// window from the caller's tensors. A stream step: `fb` new frame-blocks of
+// k (and v, copied into the plan's ring first), the chunk's queries when q is
+// given, and the ring slot of window frame-block 0.
+struct StepBlocks {
+  bool with_q = true;   // run K1 on q, then K2 and K3
+  int k_in_fb = 0;      // frame-blocks of the k input
+  int k_first_fb = 0;   // window frame-block of the k input's first one
+  int slot0_fb = 0;     // ring slot of window frame-block 0
+  const void* v_attn = nullptr;  // raster v seen by K3 (caller's tensor or the ring)
+};
+
+lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float* gamma_q, const float* gamma_k,
+                       void* out, cudaStream_t s, const StepBlocks& sb) {
+  const lcsa::Grid& g = p->res.grid;
+  cudaError_t e;
   lcsa::K1Params k1;
   k1.g = g;
   k1.q = static_cast<const __nv_bfloat16*>(q);
@@ -394,6 +403,12 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k1.num_sms = p->num_sms;
   k1.split_part = p->split_part;
   k1.split_cnt = p->split_cnt;
+  k1.n_qblk = sb.with_q ? g.B * g.nQB : 0;
+  k1.k_in_fb = sb.k_in_fb;
+  k1.k_first_fb = sb.k_first_fb;
+  k1.ring_fb = g.Tkv / g.bt;
+  k1.slot0_fb = sb.slot0_fb;
+  k1.Lk_in = int64_t(sb.k_in_fb) * g.bt * g.gh * g.gw;
 
   lcsa::K2Params k2;
   k2.g = g;
@@ -406,28 +421,38 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   k2.sort_n = p->res.sort_n;
   k2.clear_cnt = p->split_cnt;
   k2.n_clear = lcsa::kMaxK1Ctas;
+  k2.ring_fb = g.Tkv / g.bt;
+  k2.slot0_fb = sb.slot0_fb;
 
   lcsa::K3Params k3;
   k3.g = g;
   k3.qhat = p->qhat;
   k3.khat = p->khat;
-  k3.v = static_cast<const __nv_bfloat16*>(v);
+  k3.v = static_cast<const __nv_bfloat16*>(sb.v_attn);
   k3.out = static_cast<__nv_bfloat16*>(out);
   k3.row_ptr = p->row_ptr;
   k3.col_idx = p->col_idx;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
   k3.err = p->err;
+  k3.ring_fb = g.Tkv / g.bt;
+  k3.slot0_fb = sb.slot0_fb;
 
   cudaEvent_t* ev = nullptr;
-  if (!p->evsets.empty()) ev = p->evsets[size_t(p->timed % int64_t(p->evsets.size()))].data();
+  if (sb.with_q && !p->evsets.empty()) ev = p->evsets[size_t(p->timed % int64_t(p->evsets.size()))].data();
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
+  if (!sb.with_q) {
+    // no K2 after this K1: clear its merge counters here
+    if ((e = cudaMemsetAsync(p->split_cnt, 0, size_t(lcsa::kMaxK1Ctas) * 4, s)) != cudaSuccess)
+      return cuda_fail(e, "clear merge counters");
+    return LCSA_OK;
+  }
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
   {
     CUtensorMap tm_v;
-    if ((e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
+    if ((e = lcsa::make_raster_map(&tm_v, sb.v_attn, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
       return cuda_fail(e, "attention launch");
   }
@@ -436,6 +461,109 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
     ++p->timed;
   }
   return LCSA_OK;
+}
+
+}  // namespace
+
+lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                           const float* gamma_k, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (p->streaming) return fail(LCSA_ERR_INVALID_ARG, "a stream plan takes lcsa_forward_stream");
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(gamma_q) ||
+      !aligned16(gamma_k))
+    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  const lcsa::Grid& g = p->res.grid;
+  StepBlocks sb;
+  sb.k_in_fb = g.Tkv / g.bt;
+  sb.v_attn = v;
+  return run_step(p, q, k, gamma_q, gamma_k, out, s, sb);
+}
+
+lcsa_status_t lcsa_plan_create_stream(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out) {
+  if (cfg && cfg->host_io) return fail(LCSA_ERR_INVALID_ARG, "stream plans take device tensors (host_io = 0)");
+  lcsa_status_t st = lcsa_plan_create(cfg, cuda_device, out);
+  if (st != LCSA_OK) return st;
+  lcsa_plan* p = *out;
+  const lcsa::Grid& g = p->res.grid;
+  if ((st = dev_alloc(&p->v_ring, size_t(g.B) * g.Lkv * g.C * 2, "v ring")) != LCSA_OK) {
+    lcsa_plan_destroy(p);
+    *out = nullptr;
+    return st;
+  }
+  p->streaming = true;
+  p->pushed_fb = 0;
+  return LCSA_OK;
+}
+
+namespace {
+
+// One stream step: `frames` new frames of k and v (and the chunk's q when
+// given) enter the window; the ring slot of absolute frame-block F is
+// F % (Tkv / bt). Copies v into the ring, rebuilds the frame RoPE table for
+// the window's new absolute position, then runs the kernels.
+lcsa_status_t stream_step(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                          const float* gamma_k, int frames, void* out, cudaStream_t s) {
+  const lcsa::Grid& g = p->res.grid;
+  const int ring = g.Tkv / g.bt;
+  if (frames <= 0 || frames % g.bt || frames > g.Tkv)
+    return fail(LCSA_ERR_SHAPE, "%d frames (a multiple of block_t, at most kv_frames = %d)", frames, g.Tkv);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  const int fb = frames / g.bt;
+  const int64_t after = p->pushed_fb + fb;
+  if (q && after < ring)
+    return fail(LCSA_ERR_INVALID_ARG, "the KV window is not full yet (%lld of %d frame-blocks): push frames first",
+                (long long)after, ring);
+  const size_t frame_bytes = size_t(g.gh) * g.gw * g.C * 2;
+  for (int b = 0; b < g.B; ++b)
+    for (int f = 0; f < frames; ++f) {
+      const int64_t abs_fb = p->pushed_fb + f / g.bt;
+      const int slot = int(abs_fb % ring);
+      char* dst = reinterpret_cast<char*>(p->v_ring) + (size_t(b) * g.Tkv + size_t(slot) * g.bt + f % g.bt) * frame_bytes;
+      const char* src = static_cast<const char*>(v) + (size_t(b) * frames + f) * frame_bytes;
+      if ((e = cudaMemcpyAsync(dst, src, frame_bytes, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+        return cuda_fail(e, "v ring copy");
+    }
+  const int64_t w0_fb = after - ring;  // window frame-block 0, counted from the first push (may be < 0)
+  const int t0 = p->cfg.kv_frame_offset + int(w0_fb) * g.bt;
+  if ((e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, t0, p->cfg.head_dim, s)) != cudaSuccess)
+    return cuda_fail(e, "rope table launch");
+  StepBlocks sb;
+  sb.with_q = q != nullptr;
+  sb.k_in_fb = fb;
+  sb.k_first_fb = ring - fb;
+  sb.slot0_fb = int(((w0_fb % ring) + ring) % ring);
+  sb.v_attn = p->v_ring;
+  lcsa_status_t st = run_step(p, q ? q : k, k, q ? gamma_q : gamma_k, gamma_k, out, s, sb);
+  if (st == LCSA_OK) p->pushed_fb = after;
+  return st;
+}
+
+}  // namespace
+
+lcsa_status_t lcsa_stream_push(lcsa_plan_t p, const void* k, const void* v, const float* gamma_k, int frames,
+                               void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (!p->streaming) return fail(LCSA_ERR_INVALID_ARG, "not a stream plan (lcsa_plan_create_stream)");
+  if (!k || !v || !gamma_k) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(gamma_k))
+    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  return stream_step(p, nullptr, k, v, nullptr, gamma_k, frames, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+lcsa_status_t lcsa_forward_stream(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                                  const float* gamma_k, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (!p->streaming) return fail(LCSA_ERR_INVALID_ARG, "not a stream plan (lcsa_plan_create_stream)");
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(gamma_q) ||
+      !aligned16(gamma_k))
+    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  return stream_step(p, q, k, v, gamma_q, gamma_k, p->res.grid.Tq, out, static_cast<cudaStream_t>(stream));
 }
 
 lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,

@@ -67,6 +67,16 @@ struct K1Params {
   int num_sms;          // persistent grid size (one CTA per SM, at most kMaxK1Ctas)
   float* split_part;    // [kMaxK1Ctas][2][C] partial pooled sums of blocks cut between CTAs
   unsigned* split_cnt;  // [kMaxK1Ctas] arrivals per cut; zero on entry (K2 clears them)
+  // Which blocks this launch processes. A stateless call: all of q and k
+  // (n_qblk = B nQB, k_in_fb = ring_fb, k_first_fb = slot0_fb = 0). A stream
+  // call: the new frames only, k^ / pooled k written to the ring slots
+  // ((slot0_fb + window frame-block) % ring_fb).
+  int n_qblk;           // query blocks processed: B * nQB, or 0 (a KV-only push)
+  int k_in_fb;          // frame-blocks of the k input (its frames / bt)
+  int k_first_fb;       // KV-window frame-block of the k input's first frame-block
+  int ring_fb;          // KV window length in frame-blocks (Tkv / bt)
+  int slot0_fb;         // ring slot of window frame-block 0
+  int64_t Lk_in;        // tokens per batch element of the k input
 };
 
 struct K2Params {
@@ -80,6 +90,7 @@ struct K2Params {
   int sort_n;           // power of two >= the largest admissible set
   unsigned* clear_cnt;  // K1's split counters, zeroed here for the next K1 (n_clear entries)
   int n_clear;
+  int ring_fb, slot0_fb;  // pooled k of window frame-block tk sits in ring slot (slot0_fb + tk) % ring_fb
 };
 
 struct K3Params {
@@ -92,7 +103,16 @@ struct K3Params {
   const int* col_idx;
   float scale_log2;         // softmax scale * log2(e)
   unsigned* err;
+  int ring_fb, slot0_fb;    // k^ / v of window frame-block tk sit in ring slot (slot0_fb + tk) % ring_fb
 };
+
+// The stateless call's block sets: every query and key block, ring = window.
+inline void k1_all_blocks(K1Params& k1) {
+  k1.n_qblk = k1.g.B * k1.g.nQB;
+  k1.ring_fb = k1.k_in_fb = k1.g.Tkv / k1.g.bt;
+  k1.k_first_fb = k1.slot0_fb = 0;
+  k1.Lk_in = k1.g.Lkv;
+}
 
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, int d, cudaStream_t s);

@@ -223,6 +223,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.err = err;
   k1.split_part = split_part;
   k1.split_cnt = split_cnt;
+  lcsa::k1_all_blocks(k1);
   if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "device attributes");
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
@@ -240,6 +241,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.sort_n = sort_n;
   k2.clear_cnt = split_cnt;
   k2.n_clear = lcsa::kMaxK1Ctas;
+  k2.ring_fb = g.Tkv / g.bt;
+  k2.slot0_fb = 0;
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
 
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));
@@ -253,6 +256,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.col_idx = col_idx;
   k3.scale_log2 = scale * 1.4426950408889634f;
   k3.err = err;
+  k3.ring_fb = g.Tkv / g.bt;
+  k3.slot0_fb = 0;
   {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;

@@ -157,6 +157,30 @@ LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void*
 LCSA_API lcsa_status_t lcsa_forward_host(lcsa_plan_t plan, const void* q, const void* k, const void* v,
                                 const float* gamma_q, const float* gamma_k, void* out, void* stream);
 
+/* Streaming, the pages' steady state ("FlashVSR: From 17.2 FPS to 57.3 FPS at
+   768x1408", Rebuild sparse attention for Hopper: incremental pooled-K
+   caching; "FlashVSR Inference", Non-Negotiable Streaming Contract: the KV
+   window is kv_ratio x the query frames). A stream plan keeps the last
+   kv_frames frames of k^, pooled k and raw v in a ring, so each call
+   normalises, rotates and pools only the new frames.
+   lcsa_plan_create_stream: as lcsa_plan_create (host_io must be 0), plus a
+     plan-owned v ring of batch * kv_frames frames. Absolute frame positions
+     (RoPE) start at cfg->kv_frame_offset for the first frame pushed.
+   lcsa_stream_push: appends `frames` frames of k and v ([batch][frames][H'][W']
+     [heads*d] bf16, device) to the window without attention (to fill it before
+     the first chunk); frames is a multiple of block_t, at most kv_frames.
+   lcsa_forward_stream: appends the chunk's q_frames new frames of k and v, and
+     computes attention for its q ([batch][q_frames][H'][W'][heads*d]) over the
+     window of the last kv_frames frames (the new ones last). The window must be
+     full (LCSA_ERR_INVALID_ARG otherwise). The result equals lcsa_forward on
+     that window with kv_frame_offset = the absolute index of its first frame.
+   A stream plan rejects lcsa_forward; calls on one plan must not overlap. */
+LCSA_API lcsa_status_t lcsa_plan_create_stream(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out);
+LCSA_API lcsa_status_t lcsa_stream_push(lcsa_plan_t plan, const void* k, const void* v, const float* gamma_k,
+                                        int frames, void* stream);
+LCSA_API lcsa_status_t lcsa_forward_stream(lcsa_plan_t plan, const void* q, const void* k, const void* v,
+                                           const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
 /* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
    Every GPU that loads the library holds this array until the process exits. */
 #define LCSA_NOALLOC_WORKSPACE_BYTES (32u << 20)
