@@ -50,6 +50,8 @@ def _args():
     ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--stream", action="store_true",
+                    help="time a stream plan: each step brings the chunk's new frames into the KV ring")
     return ap.parse_args()
 
 
@@ -352,10 +354,93 @@ def run_lcsa(args):
     return 0
 
 
+def run_stream(args):
+    """One step = one stream chunk (lcsa_forward_stream): the q_frames new
+    frames of q, k and v enter the plan's KV ring; K1 works on the new frames
+    only. Frames cycle through a 16-frame sequence resident in HBM (377 MB at
+    768x1280, larger than L2), and L2 is flushed before every timed chunk."""
+    import torch
+
+    import block_sparse_video_lcsa_b200 as lcsa
+    from block_sparse_video_lcsa_b200 import synth
+
+    world, rank, local = _dist()
+    if world > 1:
+        print(json.dumps({"impl": "lcsa", "unavailable": "--stream times one GPU"}))
+        return 0
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    nf = 16
+    seq = synth.make_inputs(wl.replace(q_frames=nf, kv_frames=nf))
+    plane = wl.grid_h * wl.grid_w
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+
+    q, k, v = bf(seq.q), bf(seq.k), bf(seq.v)
+    gq, gk = torch.from_numpy(seq.gamma_q).to(dev), torch.from_numpy(seq.gamma_k).to(dev)
+    plan = lcsa.lcsa_plan_create_stream(lcsa.config_from_workload(wl), local)
+    geo = plan.geometry
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty((wl.batch, wl.q_frames * plane, wl.channels), dtype=torch.bfloat16, device=dev)
+    first = wl.kv_frames - wl.q_frames
+    plan.lcsa_stream_push(k[:, :first * plane].contiguous(), v[:, :first * plane].contiguous(), gk, first, stream)
+    starts_f = list(range(0, nf - wl.q_frames + 1, wl.q_frames))
+    chunks = [tuple(t[:, f * plane:(f + wl.q_frames) * plane].contiguous() for t in (q, k, v)) for f in starts_f]
+
+    def chunk(i):
+        cq, ck, cv = chunks[i % len(chunks)]
+        plan.lcsa_forward_stream(cq, ck, cv, gq, gk, out, stream)
+
+    for i in range(args.warmup):
+        chunk(i)
+    plan.lcsa_check_device_error(stream)
+    plan.lcsa_plan_set_timing(args.steps)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    try:
+        gpu_id = "GPU-%s" % torch.cuda.get_device_properties(dev).uuid
+    except Exception:  # noqa: BLE001 - fall back to the index
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            chunk(args.warmup + i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    plan.lcsa_check_device_error(stream)
+    ms = sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)) / args.steps
+    kms, _ = plan.lcsa_get_kernel_times()
+    plan.destroy()
+    flops = geo.selected_flops
+    act = 2.0 * geo.channels
+    k1_bytes = 2.0 * act * wl.batch * 2 * geo.q_tokens   # q and k of the new frames, read and written
+    peaks = _peaks()
+    line = {"metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name + " (stream plan: KV ring, new frames per chunk)",
+                       "q_tokens": geo.q_tokens, "kv_tokens": geo.kv_tokens, "topk": geo.topk,
+                       "l2": "256 MiB buffer written before every timed chunk"},
+            "kernels": {"prologue_ms": kms[0], "select_ms": kms[1], "attention_ms": kms[2],
+                        "prologue_bytes": k1_bytes, "prologue_gbs": k1_bytes / (kms[0] * 1e-3) / 1e9,
+                        "attention_tflops": flops / (kms[2] * 1e-3) / 1e12,
+                        "other_ms": ms - sum(kms), "hbm_peak_gbs": peaks["hbm_gbs"]},
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.stream:
+        return run_stream(args)
     return run_lcsa(args)
 
 
