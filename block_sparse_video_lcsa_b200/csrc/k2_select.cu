@@ -63,7 +63,11 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   auto cand_block = [&](int c, bool ring) {
     const int tk = fdiv(c, m_per), r2 = c - tk * per;
     const int hr = fdiv(r2, m_nw), wr = r2 - hr * nw;
-    const int slot = ring ? (p.slot0_fb + tk) % p.ring_fb : tk;  // where its pooled k is stored
+    int slot = tk;  // where its pooled k is stored: ring slot (slot0 + tk) mod ring, both below ring
+    if (ring) {
+      slot += p.slot0_fb;
+      if (slot >= p.ring_fb) slot -= p.ring_fb;
+    }
     return slot * g.bpf + (h0 + hr) * g.nWb + (w0 + wr);
   };
 

@@ -368,57 +368,88 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      int kv = 0, row_it = 0;
-      bool ok = true;
-      for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-        const int beg = p.row_ptr[rr], n = p.row_ptr[rr + 1] - beg;
-        const int bhh = rr / g.nQB;
-        const int b = bhh / g.Hn, h = bhh % g.Hn;
-        if (row_it > 0) ok = mbar_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1);
-        if (!ok) break;
+    // ---------------- TMA producer (converged warp, lane 0 issues) ----------------
+    // The row's CSR entries are fetched 32 at a time by the whole warp (one
+    // coalesced load), each lane turning its entry into the k^ tile row and
+    // the V box coordinates; lane 0 takes them by shuffle. The issuing lane
+    // thus never waits on a dependent load or an integer division per block.
+    struct Entries {
+      int chunk = -1;
+      int krow = 0, x0 = 0, y0 = 0, f0 = 0;
+    };
+    int kv = 0, row_it = 0;
+    bool ok = true;
+    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+      const int beg = p.row_ptr[rr], n = p.row_ptr[rr + 1] - beg;
+      const int bhh = rr / g.nQB;
+      const int b = bhh / g.Hn, h = bhh % g.Hn;
+      if (row_it > 0 && !(ok = warp_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1))) break;
+      if (lane == 0) {
         mbar_expect_tx(bar(bars->q_full), QM * kD * 2);
         tma_load_2d(base + kOffQ, &tm_q, 0, rr * QM, bar(bars->q_full));
         tma_load_2d(base + kOffQ + QM * 128, &tm_q, 64, rr * QM, bar(bars->q_full));
-        const int steps = (n + KB - 1) / KB;
-        // the selected block feeding sub-tile i of step st (an odd last step
-        // repeats its block; the softmax masks the copy)
-        auto step_block = [&](int st, int i) { return p.col_idx[beg + min(st * KB + i, n - 1)]; };
-        // window block -> its k^ block in the ring
-        auto ring_block = [&](int kb) { return ((p.slot0_fb + kb / g.bpf) % p.ring_fb) * g.bpf + kb % g.bpf; };
-        auto load_k = [&](int st) -> bool {
-          const int kvj = kv + st, ks = kvj % kKStages, ku = kvj / kKStages;
-          if (ku > 0 && !mbar_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
-          const uint32_t kdst = base + kOffK + ks * kTileBytes;
-          mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
+      }
+      __syncwarp();
+      const int steps = (n + KB - 1) / KB;
+      auto fill = [&](Entries& e, int chunk) {
+        e.chunk = chunk;
+        const int j = chunk * 32 + lane;
+        if (j < n) {
+          const int kb = p.col_idx[beg + j];
+          const int fbw = kb / g.bpf, rem = kb - fbw * g.bpf;
+          int slot = p.slot0_fb + fbw;  // ring slot of its frame-block (both terms below ring_fb)
+          if (slot >= p.ring_fb) slot -= p.ring_fb;
+          e.krow = (bhh * g.nKB + slot * g.bpf + rem) * QM;
+          e.x0 = (rem % g.nWb) * g.bw;
+          e.y0 = (rem / g.nWb) * g.bh;
+          e.f0 = b * g.Tkv + slot * g.bt;
+        }
+      };
+      Entries ke, ve;  // cursors of the K loads (two steps ahead) and of the V loads
+      // entry of the selected block feeding sub-tile i of step st (an odd last
+      // step repeats its block; the softmax masks the copy)
+      auto entry = [&](Entries& e, int st, int i) -> int {
+        const int j = min(st * KB + i, n - 1);
+        if (e.chunk != (j >> 5)) fill(e, j >> 5);  // warp-uniform
+        return j & 31;
+      };
+      auto load_k = [&](int st) -> bool {
+        const int kvj = kv + st, ks = kvj % kKStages, ku = kvj / kKStages;
+        if (ku > 0 && !warp_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
+        const uint32_t kdst = base + kOffK + ks * kTileBytes;
+        if (lane == 0) mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
 #pragma unroll
-          for (int i = 0; i < KB; ++i) {
-            const int kb = step_block(st, i);
-            const int kp = ring_block(kb);
-            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, (bhh * g.nKB + kp) * QM, bar(bars->k_full[ks]));
-            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, (bhh * g.nKB + kp) * QM, bar(bars->k_full[ks]));
+        for (int i = 0; i < KB; ++i) {
+          const int src = entry(ke, st, i);
+          const int krow = __shfl_sync(0xffffffffu, ke.krow, src);
+          if (lane == 0) {
+            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, krow, bar(bars->k_full[ks]));
+            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, krow, bar(bars->k_full[ks]));
           }
-          return true;
-        };
-        for (int st = 0; st < 2 && st < steps && ok; ++st) ok = load_k(st);
-        for (int st = 0; st < steps && ok; ++st) {
-          if (st + 2 < steps && !(ok = load_k(st + 2))) break;
-          const int kvj = kv + st, vs = kvj % kVStages, vu = kvj / kVStages;
-          if (vu > 0 && !(ok = mbar_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
-          const uint32_t vdst = base + kOffV + vs * kTileBytes;
-          mbar_expect_tx(bar(bars->v_full[vs]), kTileBytes);
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int st = 0; st < 2 && st < steps && ok; ++st) ok = load_k(st);
+      for (int st = 0; st < steps && ok; ++st) {
+        if (st + 2 < steps && !(ok = load_k(st + 2))) break;
+        const int kvj = kv + st, vs = kvj % kVStages, vu = kvj / kVStages;
+        if (vu > 0 && !(ok = warp_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
+        const uint32_t vdst = base + kOffV + vs * kTileBytes;
+        if (lane == 0) mbar_expect_tx(bar(bars->v_full[vs]), kTileBytes);
 #pragma unroll
-          for (int i = 0; i < KB; ++i) {
-            const int kb = step_block(st, i);
-            const int tb = (p.slot0_fb + kb / g.bpf) % p.ring_fb, rem = kb % g.bpf;  // ring slot of its frame-block
-            const int x0 = (rem % g.nWb) * g.bw, y0 = (rem / g.nWb) * g.bh, f0 = b * g.Tkv + tb * g.bt;
+        for (int i = 0; i < KB; ++i) {
+          const int src = entry(ve, st, i);
+          const int x0 = __shfl_sync(0xffffffffu, ve.x0, src), y0 = __shfl_sync(0xffffffffu, ve.y0, src);
+          const int f0 = __shfl_sync(0xffffffffu, ve.f0, src);
+          if (lane == 0) {
             tma_load_5d(vdst + i * QM * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
             tma_load_5d(vdst + kHalfBytes + i * QM * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
           }
         }
-        kv += steps;
+        __syncwarp();
       }
+      kv += steps;
     }
   } else if (warp == 1) {
     // ---------------- S issuer (converged warp, lane 0 issues) ----------------
