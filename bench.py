@@ -50,6 +50,8 @@ def _args():
     ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time N sequential calls (a DiT chunk's attention layers), eager and as one CUDA graph")
     ap.add_argument("--stream", action="store_true",
                     help="time a stream plan: each step brings the chunk's new frames into the KV ring")
     return ap.parse_args()
@@ -435,12 +437,97 @@ def run_stream(args):
     return 0
 
 
+def run_layers(args):
+    """One step = the attention calls of one DiT chunk: args.layers sequential
+    lcsa_forward calls of one geometry (three distinct input sets, cycled),
+    timed eagerly and as one captured CUDA graph replayed per step."""
+    import torch
+
+    import block_sparse_video_lcsa_b200 as lcsa
+    from block_sparse_video_lcsa_b200 import synth
+
+    world, rank, local = _dist()
+    if world > 1:
+        print(json.dumps({"impl": "lcsa", "unavailable": "--layers times one GPU"}))
+        return 0
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+
+    sets = []
+    for i in range(3):
+        inp = synth.make_inputs(wl.replace(seed=i))
+        sets.append((bf(inp.q), bf(inp.k), bf(inp.v), torch.from_numpy(inp.gamma_q).to(dev),
+                     torch.from_numpy(inp.gamma_k).to(dev)))
+    outs = [torch.empty_like(st[0]) for st in sets]
+    plan = lcsa.lcsa_plan_create(lcsa.config_from_workload(wl), local)
+    geo = plan.geometry
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+
+    def chunk(stream):
+        for layer in range(args.layers):
+            q, k, v, gq, gk = sets[layer % 3]
+            plan.lcsa_forward(q, k, v, gq, gk, outs[layer % 3], stream)
+
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            chunk(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            chunk(side)
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize(dev)
+    plan.lcsa_check_device_error(side)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(side)
+        for _ in range(args.steps):
+            fn()
+        e1.record(side)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    try:
+        gpu_id = "GPU-%s" % torch.cuda.get_device_properties(dev).uuid
+    except Exception:  # noqa: BLE001 - fall back to the index
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        with torch.cuda.stream(side):
+            eager_ms = timed(lambda: chunk(side))
+            graph_ms = timed(graph.replay)
+    plan.lcsa_check_device_error(side)
+    del graph
+    plan.destroy()
+    flops = geo.selected_flops * args.layers
+    line = {"metric": METRIC, "value": flops / (graph_ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": graph_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "%s x %d layers (one CUDA graph per chunk)" % (wl.name, args.layers),
+                       "l2": "three input sets (3 x %.0f MB) cycled over the layers" % (
+                           (sets[0][0].numel() + 2 * sets[0][1].numel()) * 2 / 1e6)},
+            "layers": {"count": args.layers, "eager_ms_per_layer": eager_ms / args.layers,
+                       "graph_ms_per_layer": graph_ms / args.layers,
+                       "eager_tflops": flops / (eager_ms * 1e-3) / 1e12},
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
     if args.stream:
         return run_stream(args)
+    if args.layers > 0:
+        return run_layers(args)
     return run_lcsa(args)
 
 
