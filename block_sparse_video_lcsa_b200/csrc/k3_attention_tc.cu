@@ -256,6 +256,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       LCSA_W32(r)
       : "memory");
 }
+#define LCSA_W16(a)                                                                                               \
+  "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]), \
+      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15])
+
+// 16-lane shapes, for M = 64 accumulators (lanes 0-15 of the warp's lane
+// quarter). .16x256b.x8: for rep r, registers 4r and 4r+1 hold columns
+// 8r + 2(t%4) and 8r + 2(t%4) + 1 of lane t/4, registers 4r+2 and 4r+3 the
+// same columns of lane t/4 + 8 (t = thread of the warp).
+__device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : LCSA_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      LCSA_W32(r)
+      : "memory");
+}
+// .16x128b.x8: for rep r, register 2r holds column 4r + t%4 of lane t/4 and
+// register 2r+1 the same column of lane t/4 + 8.
+__device__ __forceinline__ void tmem_st16x128_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      LCSA_W16(r)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -528,14 +559,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       mbar_drain(bar(bars->mma_drain[1]), 0);
     }
-  } else {
-    // ---------------- softmax / correction / epilogue ----------------
-    const int sp = warp & 3;                 // TMEM lane quarter of this warp
-    const int half = (warp - 3) >> 2;        // which 64 key columns / channels
-    const int row_in_tile = sp * 32 + lane;  // exchange slot of this lane's row
-    // query token of this lane: M = 128 uses every lane, M = 64 lanes 0-15 of each quarter
-    const bool active = QM == 128 || lane < 16;
-    const int m_tok = QM == 128 ? row_in_tile : sp * 16 + (lane & 15);
+  } else if constexpr (QM == 64) {
+    // ---------------- softmax / correction / epilogue, 64-token tiles ----------------
+    // Query row m of an M = 64 accumulator sits in TMEM lane 32 * (m / 16) +
+    // m % 16, so a lane quarter holds 16 rows. The 16-lane load shapes spread
+    // them over the whole warp: thread t carries rows mA = 16 sp + t / 4 and
+    // mB = mA + 8, 16 of the half's 64 key columns each; the four threads of
+    // a row combine their maxima and sums by shuffles.
+    const int sp = warp & 3;
+    const int half = (warp - 3) >> 2;
+    const int cq = lane & 3;
+    const int mA = sp * 16 + (lane >> 2), mB = mA + 8;
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
     float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
     float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
@@ -544,11 +578,180 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
       const int n_sel = p.row_ptr[rr + 1] - p.row_ptr[rr];
-      const int n = (n_sel + KB - 1) / KB;  // KV tiles of the row
+      const int n = (n_sel + 1) / 2;  // KV tiles of the row, two blocks each
+      float mu[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      for (int j = 0; j < n && ok; ++j, ++s_it) {
+        // an odd last tile repeats its block in keys 64-127
+        const bool masked = half == 1 && 2 * j + 1 >= n_sel;
+        const int sb = s_it % kSBufs;
+        if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld16x256_x8(lane_addr + kColS + sb * 128 + half * 64, sr);
+        tmem_wait_ld();
+        auto sv = [&](int e) { return __uint_as_float(sr[e]); };
+        float mx[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float t[16];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            t[2 * r] = sv(4 * r + 2 * h2);
+            t[2 * r + 1] = sv(4 * r + 2 * h2 + 1);
+          }
+          const float a0 = fmax3(t[0], t[1], t[2]), a1 = fmax3(t[3], t[4], t[5]), a2 = fmax3(t[6], t[7], t[8]);
+          const float a3 = fmax3(t[9], t[10], t[11]), a4 = fmax3(t[12], t[13], t[14]);
+          float m = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, t[15]));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+          mx[h2] = masked ? -INFINITY : m;
+        }
+        float* slot = xmax + (j & 1) * 256;
+        if (cq == 0) {
+          slot[half * 128 + mA] = mx[0];
+          slot[half * 128 + mB] = mx[1];
+        }
+        mbar_arrive(bar(bars->pair[sp]));
+        if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 23))) break;
+        ++xk;
+        mx[0] = fmaxf(mx[0], slot[(half ^ 1) * 128 + mA]);
+        mx[1] = fmaxf(mx[1], slot[(half ^ 1) * 128 + mB]);
+        float alpha[2];
+        bool need_any = false;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float m_new = fmaxf(mu[h2], mx[h2] * c);
+          const bool need = m_new > mu[h2] + kRescaleLog2;
+          alpha[h2] = 1.f;
+          if (need) {
+            alpha[h2] = exp2_mufu(mu[h2] - m_new);
+            mu[h2] = m_new;
+          }
+          l[h2] *= alpha[h2];
+          need_any |= need;
+        }
+        const bool warp_need = __any_sync(0xffffffffu, need_any);
+        uint32_t pk[16];
+        float2 rs[2][2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) rs[h2][0] = rs[h2][1] = make_float2(0.f, 0.f);
+        const float2 c2 = make_float2(c, c);
+        const float2 mneg[2] = {make_float2(-mu[0], -mu[0]), make_float2(-mu[1], -mu[1])};
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 4 * r + 2 * h2;
+            const float2 x = __ffma2_rn(make_float2(sv(e), sv(e + 1)), c2, mneg[h2]);
+            const float2 pp = ((2 * r + h2) % kPolyEvery == kPolyEvery - 1) ? exp2_poly2(x)
+                                                                           : make_float2(exp2_mufu(x.x), exp2_mufu(x.y));
+            rs[h2][r & 1] = __fadd2_rn(rs[h2][r & 1], pp);
+            pk[2 * r + h2] = pack_bf16(pp.x, pp.y);
+          }
+        }
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+        } else {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const float2 s2 = __fadd2_rn(rs[h2][0], rs[h2][1]);
+            l[h2] += s2.x + s2.y;
+          }
+        }
+        // O is rescaled once every earlier P.V has completed (the last of them
+        // is P.V number gp = s_it - 1; P.V gp + 2 needs a P this warp has not
+        // written yet, so the parity wait on o_done[gp & 1] cannot be
+        // overtaken). P is stored only after that P.V has completed too: with
+        // M = 64 P stores overlapping an in-flight P.V, outputs varied from run
+        // to run on this part, although isolated M = 64 products read and
+        // write lanes 0-15 of each quarter only.
+        if (j >= 1) {
+          const int gp = s_it - 1;
+          if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 21))) break;
+          tc_fence_after();
+          if (warp_need) {
+            uint32_t o[32];
+            const uint32_t oa = lane_addr + kColO + half * 64;
+            tmem_ld16x256_x8(oa, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              o[4 * r] = __float_as_uint(__uint_as_float(o[4 * r]) * alpha[0]);
+              o[4 * r + 1] = __float_as_uint(__uint_as_float(o[4 * r + 1]) * alpha[0]);
+              o[4 * r + 2] = __float_as_uint(__uint_as_float(o[4 * r + 2]) * alpha[1]);
+              o[4 * r + 3] = __float_as_uint(__uint_as_float(o[4 * r + 3]) * alpha[1]);
+            }
+            tmem_st16x256_x8(oa, o);
+          }
+        }
+        // P columns: key pair (2i, 2i+1) of this half in column half * 64 + i
+        tmem_st16x128_x8(lane_addr + kColS + sb * 128 + half * 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->p_full[sb]));
+      }
+      if (!ok) break;
+      {
+        const int gp = s_it - 1;  // the row's last P.V (completion implies all earlier ones)
+        if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 22))) break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 1);
+        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 2);
+      }
+      if (cq == 0) {
+        xsum[half * 128 + mA] = l[0];
+        xsum[half * 128 + mB] = l[1];
+      }
+      mbar_arrive(bar(bars->pair[sp]));
+      if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
+      ++xk;
+      const float invA = 1.0f / (l[0] + xsum[(half ^ 1) * 128 + mA]);
+      const float invB = 1.0f / (l[1] + xsum[(half ^ 1) * 128 + mB]);
+      const int bhh = rr / g.nQB, qb = rr % g.nQB;
+      const int b = bhh / g.Hn, h = bhh % g.Hn;
+      const int tb = qb / g.bpf, rem = qb % g.bpf;
+      auto token = [&](int m) {
+        const int tt = m / (g.bh * g.bw), yy = (m / g.bw) % g.bh, xx = m % g.bw;
+        return (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
+      };
+      const int ch = h * kD + half * 64 + 2 * cq;
+      __nv_bfloat16* dA = p.out + (int64_t(b) * g.Lq + token(mA)) * g.C + ch;
+      __nv_bfloat16* dB = p.out + (int64_t(b) * g.Lq + token(mB)) * g.C + ch;
+      uint32_t o[32];
+      tmem_ld16x256_x8(lane_addr + kColO + half * 64, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        *reinterpret_cast<uint32_t*>(dA + 8 * r) =
+            pack_bf16(__uint_as_float(o[4 * r]) * invA, __uint_as_float(o[4 * r + 1]) * invA);
+        *reinterpret_cast<uint32_t*>(dB + 8 * r) =
+            pack_bf16(__uint_as_float(o[4 * r + 2]) * invB, __uint_as_float(o[4 * r + 3]) * invB);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->o_free));
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue, 128-token tiles ----------------
+    const int sp = warp & 3;                 // TMEM lane quarter of this warp
+    const int half = (warp - 3) >> 2;        // which 64 key columns / channels
+    const int row_in_tile = sp * 32 + lane;  // query token of this lane's row
+    const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
+    float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
+    const float c = p.scale_log2;
+    int s_it = 0, xk = 0;
+    bool ok = true;
+    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
+      const int n_sel = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n = n_sel;  // KV tiles of the row
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j, ++s_it) {
-        // an odd last tile of 64-token blocks repeats its block in keys 64-127
-        const bool masked = KB == 2 && half == 1 && 2 * j + 1 >= n_sel;
         const int sb = s_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
@@ -566,8 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
           mk[a] = fmaxf(mk[a], sv(a + 56));
         }
-        const float mpart =
-            masked ? -INFINITY : fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+        const float mpart = fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
         float* slot = xmax + (j & 1) * 256;
         slot[half * 128 + row_in_tile] = mpart;
         mbar_arrive(bar(bars->pair[sp]));
@@ -576,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mx = fmaxf(mpart, slot[(half ^ 1) * 128 + row_in_tile]);
         const float m_new = fmaxf(m_used, mx * c);
         const bool need = m_new > m_used + kRescaleLog2;
-        const bool warp_need = __any_sync(0xffffffffu, need && active);
+        const bool warp_need = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
-        if (need && active) {
+        if (need) {
           alpha = exp2_mufu(m_used - m_new);
           m_used = m_new;
         }
@@ -600,10 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
           }
         }
-        if (masked) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = 0u;
-        } else {
+        {
           const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
           l += rsum.x + rsum.y;
         }
@@ -624,23 +823,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(oa, o);
-          }
-        }
-        // M = 64 tiles: P is stored only once the preceding P.V has completed,
-        // and lanes without a row store zeros. With P stores overlapping an
-        // in-flight M = 64 P.V, outputs varied from run to run on this part
-        // (fewer differences with zeros in the unused lanes, none with the
-        // wait), although isolated M = 64 products read and write lanes 0-15
-        // of each quarter only. The M = 128 path shows no such effect.
-        if (QM == 64) {
-          if (!active) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pk[e] = 0u;
-          }
-          if (j >= 1 && !warp_need) {
-            const int gp = s_it - 1;
-            if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 26))) break;
-            tc_fence_after();
           }
         }
         tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
@@ -665,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bhh = rr / g.nQB, qb = rr % g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       const int tb = qb / g.bpf, rem = qb % g.bpf;
-      const int tt = m_tok / (g.bh * g.bw), yy = (m_tok / g.bw) % g.bh, xx = m_tok % g.bw;
+      const int tt = row_in_tile / (g.bh * g.bw), yy = (row_in_tile / g.bw) % g.bh, xx = row_in_tile % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
       __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + half * 64;
 #pragma unroll
@@ -679,10 +861,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
-        if (active) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = v[e];
-        }
+        for (int e = 0; e < 4; ++e) d4[e] = v[e];
       }
       tc_fence_before();
       __syncwarp();
