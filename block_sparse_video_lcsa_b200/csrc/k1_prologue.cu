@@ -9,29 +9,33 @@
 // pooling and RoPE as separate glue kernels) and Rebuild sparse attention for
 // Hopper (coalesced RoPE kernel, pooled keys).
 //
-// Work split: a persistent grid of one CTA (8 warps) per SM; CTA c owns a
-// contiguous range of the combined row list (query blocks, then key blocks;
-// a block is bt * bh rows of bw tokens). Each row is one contiguous run of
-// bw * heads * 128 bf16 in the raster input, so one thread streams the rows
-// into a ring of shared-memory stages with bulk asynchronous copies
-// (cp.async.bulk, completion counted on an mbarrier) several rows ahead,
-// while the warps work on the oldest stage: warp w takes tokens w, w+8, ...
-// of the row, lane l the 16-byte chunks l, l+32, ... of a token
-// (conflict-free shared loads), so each lane always holds the same channels
-// and its pooled sums live in registers (gains: a lane-contiguous table in
-// shared memory). The sum of squares is a warp-shuffle reduction. Pooled
-// sums are added in a fixed order: per lane
-// over its tokens, then over the warps, and for a block cut between two
-// CTAs, first part plus second part; so the pooled values, and hence the
-// block selection, do not depend on timing. q^ / k^ are written with 16-byte
-// stores, each warp store instruction covering whole 256-byte rows of two
-// heads.
+// Work split: a persistent grid of one CTA per SM (8 compute warps and one
+// copy warp); CTA c owns a contiguous range of the combined row list (query
+// blocks, then key blocks; a block is bt * bh rows of bw tokens). Each row is
+// one contiguous run of bw * heads * 128 bf16 in the raster input, so the
+// copy warp streams the rows into a ring of shared-memory stages with bulk
+// asynchronous copies (cp.async.bulk, completion counted on a "full"
+// mbarrier per stage) several rows ahead. Warp w takes tokens w, w+8, ... of
+// a row, lane l the 16-byte chunks l, l+32, ... of a token (conflict-free
+// shared loads), so each lane always holds the same channels and its pooled
+// sums live in registers (gains: a lane-contiguous table in shared memory).
+// The sum of squares is a warp-shuffle reduction. Each lane writes its
+// results back over the chunks it read, so a finished stage holds the row's
+// q^ / k^ in raster order; each compute warp then arrives on the stage's
+// "done" mbarrier and goes on to the next row without waiting for the
+// others. Once all have arrived, the copy warp writes the stage out with one
+// bulk tensor store (a box of all heads x bw tokens over the head-major
+// layout) and refills it when the store has read it. Pooled sums are added in
+// a fixed order: per lane over its tokens, then over the warps (at the end of
+// each block's rows, the only point where the compute warps synchronise),
+// and for a block cut between two CTAs, first part plus second part; so the
+// pooled values, and hence the block selection, do not depend on timing.
 #include "lcsa_internal.h"
 
 namespace lcsa {
 namespace {
 
-constexpr int kRedRows = 8;  // rows of the pooled-sum reduction buffer
+constexpr int kRedRows = 2;  // rows of the pooled-sum reduction buffer
 
 __global__ void rope_table_kernel(float2* tab, int Tkv, int gh, int gw, int t0, RopeSplit s) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -156,14 +160,52 @@ __device__ __forceinline__ BlockRef block_ref(const K1Params& p, int bid) {
 template <int CPL>
 __host__ __device__ constexpr int k1_warps() { return 8; }
 
+// A processed row (bw tokens x heads x 128, token-major as it arrived) goes
+// from its ring stage to q^ / k^ in one bulk tensor store: the map's box is
+// (128 channels, all heads, bw tokens of one block) over the head-major
+// layout, so the shared-memory side is exactly the raster row.
+__device__ __forceinline__ void store_row(const CUtensorMap* map, uint32_t src, int r_tok, int blk, int b) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];" ::"l"(map), "r"(0),
+      "r"(0), "r"(r_tok), "r"(blk), "r"(b), "r"(src)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Barrier of the compute warps only (named barrier 1; the copy warp never
+// joins it), plain and with an AND over the threads' votes.
+__device__ __forceinline__ void compute_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+__device__ __forceinline__ bool compute_sync_and(int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void record_timeout(unsigned* err, unsigned site) {
+  if (atomicCAS(err, kDevErrNone, kDevErrTimeout) == kDevErrNone) {
+    err[1] = site;
+    err[2] = blockIdx.x;
+  }
+}
+
+// Warps 0..NW-1 compute; warp NW is the copy warp (one lane issues every bulk
+// copy, so the compute warps never block on the copy engine).
 template <int CPL, bool FULL, bool HEAD>
-__global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const K1Params p, int stages,
-                                                                          uint32_t row_bytes) {
+__global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
+    prologue_kernel(const __grid_constant__ CUtensorMap tm_qhat, const __grid_constant__ CUtensorMap tm_khat,
+                    const K1Params p, int stages, uint32_t row_bytes) {
   constexpr int NW = k1_warps<CPL>(), NT = NW * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   const Grid& g = p.g;
   const uint32_t bars = smem_u32(smem);
-  uint8_t* ring = smem + kBarBytes;
+  // ring stages start on a 128-byte boundary (bulk tensor copies need it)
+  uint8_t* ring = smem + kBarBytes + (128u - (bars + kBarBytes) % 128u) % 128u;
   float* red = reinterpret_cast<float*>(ring + size_t(stages) * row_bytes);  // [kRedRows][C]
   // gains of q and k, [tensor][c4][half][lane] float4: lane-contiguous, so conflict-free
   float4* gsm = reinterpret_cast<float4*>(red + kRedRows * g.C);
@@ -179,9 +221,25 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
   const int my_rows = int(hi - lo);
   constexpr int PT = 22, PH = 21;  // RoPE pairs on the frame / row axes (head_dim 128)
 
-  // source of the CTA's row number k (global row lo + k)
+  // full[s]: the stage's row has landed; done[s]: every compute warp has
+  // finished the stage's row in place
+  auto full_bar = [&](int st) { return bars + 8u * uint32_t(st); };
+  auto done_bar = [&](int st) { return bars + 8u * uint32_t(kMaxStages + st); };
+
+  // Order of the range's rows: the cut segments first (the head [lo, a),
+  // the tail [bb, hi)), then the complete blocks [a, bb). The partial sums of
+  // the cut blocks are then merged early, while the ring streams later rows,
+  // and the range ends with a complete block, which needs no merge. (a <= bb:
+  // the range holds at least R rows, so it reaches a block boundary.)
+  const int64_t a = (lo + R - 1) / R * R, bb = hi / R * R;
+  const int nh = int(a - lo), nt = int(hi - bb);
+  auto grow_of = [&](int k) -> int64_t {
+    return k < nh ? lo + k : (k < nh + nt ? bb + (k - nh) : a + (k - nh - nt));
+  };
+
+  // source of the CTA's row number k
   auto row_src = [&](int k) -> const void* {
-    const int64_t grow = lo + k;
+    const int64_t grow = grow_of(k);
     const BlockRef br = block_ref(p, int(grow / R));
     const int r = int(grow % R);
     const int64_t tok = (int64_t(br.t_in0 + r / g.bh) * g.gh + br.y0 + r % g.bh) * g.gw + br.x0;
@@ -191,17 +249,53 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
   };
   auto issue = [&](int gi) {
     const int s = gi % stages;
-    bulk_row(smem_u32(ring + size_t(s) * row_bytes), row_src(gi), row_bytes, bars + 8 * s);
+    bulk_row(smem_u32(ring + size_t(s) * row_bytes), row_src(gi), row_bytes, full_bar(s));
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bars + 8 * s));
+    for (int s = 0; s < stages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar(s)));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(done_bar(s)), "r"(NW));
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (threadIdx.x == 0)
-    for (int gi = 0; gi < stages && gi < my_rows; ++gi) issue(gi);
+
+  if (warp == NW) {
+    // copy warp: rows in as far ahead as the ring allows; each finished row
+    // out with one bulk tensor store, its stage refilled once the store has
+    // read it
+    if (lane == 0) {
+      int issued = min(stages, my_rows);
+      for (int k = 0; k < issued; ++k) issue(k);
+      bool cok = true;
+      for (int k = 0; k < my_rows; ++k) {
+        const int s = k % stages;
+        if (!(cok = mbar_wait_bounded(done_bar(s), uint32_t(k / stages) & 1u))) break;
+        const int64_t grow = grow_of(k);
+        const BlockRef br = block_ref(p, int(grow / R));
+        store_row(br.is_q ? &tm_qhat : &tm_khat, smem_u32(ring + size_t(s) * row_bytes), int(grow % R) * g.bw,
+                  br.blk, br.b);
+        if (k + stages < my_rows) {
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          issue(k + stages);
+          issued = k + stages + 1;
+        }
+      }
+      // stores finish before the CTA exits
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      if (!cok) {
+        // the compute warps stopped: record it, then give the loads still in
+        // flight a bounded chance to land before shared memory goes away
+        record_timeout(p.err, 2);
+        for (int k = max(0, issued - stages); k < issued; ++k)
+          (void)mbar_wait_bounded(full_bar(k % stages), uint32_t(k / stages) & 1u);
+      }
+    }
+    return;
+  }
+
+  // the gains table (compute warps; the first rows are already on their way)
   for (int idx = threadIdx.x; idx < 2 * CPL * 64; idx += NT) {
     const int rem = idx % (CPL * 64);
     const int c = (rem / 64) * 32 + rem % 32, half = (rem / 32) % 2;
@@ -209,7 +303,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
     gsm[idx] = c < nchunks ? __ldg(reinterpret_cast<const float4*>(gamma + c * 8 + half * 4))
                            : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
+  compute_sync(NT);
 
   const int jb = 4 * (lane & 15);  // first RoPE pair of this lane (same in every head)
   float2 ae[CPL][2], ao[CPL][2];  // pooled sums, e / o layout of unpack_eo
@@ -218,12 +312,12 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
   bool ok = true;
   while (gi < my_rows && ok) {
     // one segment: the rows [r_begin, r_end) of block bid that this CTA owns
-    const int bid = int((lo + gi) / R);
-    const int r_begin = int((lo + gi) % R);
-    const int r_end = min(R, r_begin + (my_rows - gi));
+    const int64_t g0 = grow_of(gi);
+    const int bid = int(g0 / R);
+    const int r_begin = int(g0 % R);
+    const int r_end = gi < nh ? R : (gi < nh + nt ? nt : R);
     const BlockRef br = block_ref(p, bid);
     const float4* gtab = gsm + (br.is_q ? 0 : CPL * 64);
-    __nv_bfloat16* xhat = br.is_q ? p.qhat : p.khat;
     float* pooled = br.is_q ? p.pooled_q : p.pooled_k;
 #pragma unroll
     for (int c4 = 0; c4 < CPL; ++c4)
@@ -231,9 +325,12 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
       for (int qg = 0; qg < 2; ++qg) ae[c4][qg] = ao[c4][qg] = make_float2(0.f, 0.f);
     for (int r = r_begin; r < r_end; ++r, ++gi) {
       const int s = gi % stages;
-      const bool arrived = mbar_wait_bounded(bars + 8 * s, uint32_t(gi / stages) & 1u);
+      // after a failed wait the warp skips to the segment's end, where the
+      // compute warps agree on it
+      if (!ok || !(ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), uint32_t(gi / stages) & 1u))))
+        continue;
       const int t = br.t_win0 + r / g.bh, y = br.y0 + r % g.bh;  // t: KV-window frame
-      const uint4* row = reinterpret_cast<const uint4*>(ring + size_t(s) * row_bytes);
+      uint4* row = reinterpret_cast<uint4*>(ring + size_t(s) * row_bytes);
       for (int i = warp; i < g.bw; i += NW) {
         const int xc = br.x0 + i;
         uint4 raw[CPL];
@@ -300,7 +397,6 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
             rr_h[c4] = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
           }
         }
-        const int ti = r * g.bw + i;  // token index inside the block
 #pragma unroll
         for (int c4 = 0; c4 < CPL; ++c4) {
           const int c = c4 * 32 + lane;
@@ -322,23 +418,19 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
             w[2 * qg] = pack2(oe.x, oo.x);
             w[2 * qg + 1] = pack2(oe.y, oo.y);
           }
-          const int head = c >> 4, dd = (c & 15) * 8;
-          uint4* dst = reinterpret_cast<uint4*>(
-              xhat + (((int64_t(br.b) * g.Hn + head) * br.nblk + br.blk) * g.nb + ti) * kHeadDim + dd);
-          *dst = make_uint4(w[0], w[1], w[2], w[3]);
+          row[i * nchunks + c] = make_uint4(w[0], w[1], w[2], w[3]);  // in place: this lane read it
         }
       }
-      // every warp is done with stage s (and agrees on whether the row arrived)
-      if (__syncthreads_or(!arrived)) {
-        ok = false;
-        break;
-      }
-      if (threadIdx.x == 0 && gi + stages < my_rows) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(gi + stages);
-      }
+      // the row's results, written in place, become visible to the bulk copy
+      // engine; this warp is done with stage s
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(done_bar(s)) : "memory");
     }
-    if (!ok) break;
+    if (!compute_sync_and(NT, ok)) {
+      ok = false;
+      break;
+    }
     // warp partials -> segment sum: with 16 warps, warp w + 8 first leaves its
     // sums in row w and warp w adds its own; then the 8 rows are added in order
     float* mine = red + (warp % kRedRows) * g.C;
@@ -362,7 +454,7 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
           }
         }
       }
-      __syncthreads();
+      compute_sync(NT);
     }
     const float inv_nb = 1.0f / float(g.nb);
     float* pooled_row = pooled + (int64_t(br.b) * g.Hn * br.nblk + br.blk) * kHeadDim;  // + head * nblk * d + dd
@@ -385,29 +477,27 @@ __global__ void __launch_bounds__(k1_warps<CPL>() * 32, 1) prologue_kernel(const
       float* part = p.split_part + size_t(cut) * 2 * g.C;
       float* mypart = part + (r_begin == 0 ? 0 : g.C);
       for (int e = threadIdx.x; e < g.C; e += NT) mypart[e] = warp_sum(e);
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) combine = atomicAdd(p.split_cnt + cut, 1u) == 1u;
-      __syncthreads();
+      // The barrier orders the CTA's part before thread 0's count, whose
+      // release publishes it at GPU scope and whose acquire (for the second
+      // arrival) makes the other part visible; the barrier after it extends
+      // that to every thread.
+      compute_sync(NT);
+      if (threadIdx.x == 0) {
+        unsigned old;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.split_cnt + cut) : "memory");
+        combine = old == 1u;
+      }
+      compute_sync(NT);
       if (combine) {
-        __threadfence();
         for (int e = threadIdx.x; e < g.C; e += NT)
           pooled_row[(e / kHeadDim) * head_stride + e % kHeadDim] =
               (__ldcg(part + e) + __ldcg(part + g.C + e)) * inv_nb;
       }
     }
-    __syncthreads();  // red and combine are rewritten by the next segment
+    compute_sync(NT);  // red and combine are rewritten by the next segment
   }
-  if (!ok && threadIdx.x == 0) {
-    // a row never arrived: record it, then give the copies still in flight a
-    // bounded chance to land before the CTA (and its shared memory) goes away
-    if (atomicCAS(p.err, kDevErrNone, kDevErrTimeout) == kDevErrNone) {
-      p.err[1] = 1;
-      p.err[2] = blockIdx.x;
-    }
-    for (int k = gi; k < gi + stages && k < my_rows; ++k)
-      (void)mbar_wait_bounded(bars + 8 * (k % stages), uint32_t(k / stages) & 1u);
-  }
+  // a row never arrived (the copy warp then waits out the loads in flight)
+  if (!ok && threadIdx.x == 0) record_timeout(p.err, 1);
 }
 
 template <int CPL, bool FULL, bool HEAD>
@@ -416,15 +506,20 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   if (nblocks <= 0) return cudaSuccess;
   const uint32_t row_bytes = uint32_t(p.g.bw) * uint32_t(p.g.C) * 2u;
   const uint32_t red_bytes = uint32_t(kRedRows) * uint32_t(p.g.C) * 4u + 2u * CPL * 64u * 16u;  // + gains
-  int stages = int((kSmemBudget - kBarBytes - red_bytes) / row_bytes);
+  int stages = int((kSmemBudget - kBarBytes - 128 - red_bytes) / row_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2 || p.num_sms <= 0) return cudaErrorInvalidValue;
-  const size_t smem = kBarBytes + size_t(stages) * row_bytes + red_bytes;
+  const size_t smem = kBarBytes + 128 + size_t(stages) * row_bytes + red_bytes;  // + alignment of the ring
   cudaError_t e = cudaFuncSetAttribute(prologue_kernel<CPL, FULL, HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   int grid = nblocks < p.num_sms ? nblocks : p.num_sms;
   if (grid > kMaxK1Ctas) grid = kMaxK1Ctas;
-  prologue_kernel<CPL, FULL, HEAD><<<grid, k1_warps<CPL>() * 32, smem, s>>>(p, stages, row_bytes);
+  CUtensorMap tm_qhat, tm_khat;
+  if ((e = make_xhat_row_map(&tm_qhat, p.qhat, p.g, p.g.nQB)) != cudaSuccess ||
+      (e = make_xhat_row_map(&tm_khat, p.khat, p.g, p.g.nKB)) != cudaSuccess)
+    return e;
+  prologue_kernel<CPL, FULL, HEAD><<<grid, (k1_warps<CPL>() + 1) * 32, smem, s>>>(tm_qhat, tm_khat, p, stages,
+                                                                                 row_bytes);
   return cudaGetLastError();
 }
 

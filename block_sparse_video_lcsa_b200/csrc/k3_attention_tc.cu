@@ -920,6 +920,20 @@ cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_xhat_row_map(CUtensorMap* map, void* base, const Grid& g, int nblk) {
+  EncodeTiled enc = encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t tok = cuuint64_t(kD) * 2, blk = tok * cuuint64_t(g.nb), head = blk * cuuint64_t(nblk);
+  const cuuint64_t dims[5] = {cuuint64_t(kD), cuuint64_t(g.Hn), cuuint64_t(g.nb), cuuint64_t(nblk), cuuint64_t(g.B)};
+  const cuuint64_t strides[4] = {head, tok, blk, head * cuuint64_t(g.Hn)};
+  const cuuint32_t box[5] = {cuuint32_t(kD), cuuint32_t(g.Hn), cuuint32_t(g.bw), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
   EncodeTiled enc = encoder();
   if (!enc) return cudaErrorNotSupported;

@@ -127,6 +127,10 @@ cudaError_t launch_select(const K2Params& p, cudaStream_t s);
 bool attention_tc_supported(const Grid& g);
 cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g);
+// q^ / k^ ([B][Hn][nblk][nb][128]) seen as (channel, head, token of the block,
+// block, batch) with boxes of (128, Hn, bw, 1, 1): one box is one raster row of
+// bw tokens with all heads, token-major in shared memory (K1's bulk stores).
+cudaError_t make_xhat_row_map(CUtensorMap* map, void* base, const Grid& g, int nblk);
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s);
