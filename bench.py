@@ -152,6 +152,18 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def _max_over_ranks(value, device):
+    """The largest `value` over the ranks of the default process group (the
+    timing of a multi-GPU run is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -285,11 +297,7 @@ def run_lcsa(args):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kms, kcount = plan.lcsa_get_kernel_times()
     plan.lcsa_plan_set_timing(0)
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = _max_over_ranks(sum(step_ms), dev)
 
     # end to end: pinned host buffers through lcsa_forward_host (copies inside)
     hq = torch.from_numpy(inp.q).view(torch.bfloat16).pin_memory()
@@ -310,11 +318,8 @@ def run_lcsa(args):
         plan.lcsa_forward_host(hq, hk, hv, hgq, hgk, hout, stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
     plan.destroy()
 

@@ -15,6 +15,7 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcsa.so")
 
+ABI_VERSION = 2  # the LCSA_ABI_VERSION of include/lcsa.h this binding's structures follow
 LCSA_OK = 0
 LCSA_ERR_INVALID_ARG = 1
 LCSA_ERR_SHAPE = 2
@@ -48,6 +49,7 @@ class lcsa_config_t(ctypes.Structure):
         ("local_range", ctypes.c_int), ("topk", ctypes.c_int), ("sparse_ratio", ctypes.c_float),
         ("kv_frame_offset", ctypes.c_int), ("norm_scope", ctypes.c_int),
         ("rms_eps", ctypes.c_float), ("softmax_scale", ctypes.c_float), ("host_io", ctypes.c_int),
+        ("heads_total", ctypes.c_int),
     ]
 
 
@@ -81,6 +83,8 @@ SIGNATURES = [
     ("lcsa_plan_create_stream", _I, [ctypes.POINTER(lcsa_config_t), _I, ctypes.POINTER(_PLAN)]),
     ("lcsa_stream_push", _I, [_PLAN, _VP, _VP, _VP, _I, _VP]),
     ("lcsa_forward_stream", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_sumsq", _I, [_PLAN, _VP, _VP, _VP, _VP]),
+    ("lcsa_forward_sharded", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_plan_geometry", _I, [_PLAN, ctypes.POINTER(lcsa_geometry_t)]),
     ("lcsa_plan_topk", _I, [_PLAN, ctypes.POINTER(_I)]),
     ("lcsa_get_selection", _I, [_PLAN, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t]),
@@ -110,6 +114,9 @@ def lib():
             f = getattr(L, name)
             f.restype = res
             f.argtypes = args
+        if L.lcsa_abi_version() != ABI_VERSION:
+            raise LcsaLibraryMissing("liblcsa.so has ABI version %d, this binding needs %d: rebuild it"
+                                     % (L.lcsa_abi_version(), ABI_VERSION))
         _lib = L
     return _lib
 
@@ -263,6 +270,33 @@ class Plan:
         self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k")
         _check(lib().lcsa_forward_stream(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
                                          _addr(out), _stream(stream)), "lcsa_forward_stream")
+        return out
+
+    def lcsa_sumsq(self, q, k, ssq, stream=None):
+        """Per-token sums of squares of this plan's q then k channels into ssq
+        (fp32 [batch*(q_tokens + kv_tokens)]), for a head-sharded layer."""
+        import torch
+        c, g = self.cfg, self.geometry
+        self._expect(q, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "q")
+        self._expect(k, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "k")
+        self._expect(ssq, torch.float32, (c.batch * (g.q_tokens + g.kv_tokens),), "ssq")
+        _check(lib().lcsa_sumsq(self._h, _addr(q), _addr(k), _addr(ssq), _stream(stream)), "lcsa_sumsq")
+        return ssq
+
+    def lcsa_forward_sharded(self, q, k, v, gamma_q, gamma_k, ssq, out, stream=None):
+        """lcsa_forward of a head-sharded plan, the RMS norm taken from ssq
+        (the sums of lcsa_sumsq over all ranks)."""
+        import torch
+        c, g = self.cfg, self.geometry
+        self._expect(q, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "q")
+        self._expect(k, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "k")
+        self._expect(v, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "v")
+        self._expect(out, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "out")
+        self._expect(gamma_q, torch.float32, (g.channels,), "gamma_q")
+        self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k")
+        self._expect(ssq, torch.float32, (c.batch * (g.q_tokens + g.kv_tokens),), "ssq")
+        _check(lib().lcsa_forward_sharded(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
+                                          _addr(ssq), _addr(out), _stream(stream)), "lcsa_forward_sharded")
         return out
 
     def lcsa_forward_host(self, q, k, v, gamma_q, gamma_k, out, stream=None):

@@ -331,6 +331,11 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
         continue;
       const int t = br.t_win0 + r / g.bh, y = br.y0 + r % g.bh;  // t: KV-window frame
       uint4* row = reinterpret_cast<uint4*>(ring + size_t(s) * row_bytes);
+      // head-sharded layer: the row's per-token sums of squares over all heads
+      const float* ss_row =
+          (!HEAD && p.ss_ext) ? p.ss_ext + (br.is_q ? int64_t(br.b) * g.Lq : int64_t(g.B) * g.Lq + int64_t(br.b) * p.Lk_in) +
+                         (int64_t(br.t_in0 + r / g.bh) * g.gh + y) * g.gw + br.x0
+                   : nullptr;
       for (int i = warp; i < g.bw; i += NW) {
         const int xc = br.x0 + i;
         uint4 raw[CPL];
@@ -379,7 +384,8 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
           float ss = ss2.x + ss2.y;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          coefs(rsqrtf(ss * (1.0f / float(g.C)) + p.eps));
+          if (ss_row) ss = __ldg(ss_row + i);  // head-sharded layer: the sum over all its heads
+          coefs(rsqrtf(ss * p.norm_inv_c + p.eps));
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < (HEAD ? CPL : 1); ++c4) {
@@ -523,12 +529,41 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// One warp per token: 16-byte chunks strided over the lanes, fp32 squares,
+// then a butterfly.
+__global__ void __launch_bounds__(256) sumsq_kernel(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss) {
+  const int64_t t = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= tokens) return;
+  const uint4* row = reinterpret_cast<const uint4*>(x + t * channels);
+  float2 acc = make_float2(0.f, 0.f);
+  for (int c = lane; c < channels / 8; c += 32) {
+    float2 e[2], o[2];
+    unpack_eo(__ldg(row + c), e, o);
+#pragma unroll
+    for (int qg = 0; qg < 2; ++qg) {
+      acc = __ffma2_rn(e[qg], e[qg], acc);
+      acc = __ffma2_rn(o[qg], o[qg], acc);
+    }
+  }
+  float v = acc.x + acc.y;
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+  if (lane == 0) ss[t] = v;
+}
+
 }  // namespace
 
 cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, int d, cudaStream_t s) {
   const RopeSplit rs = rope_split(d);
   const int n = Tkv * rs.pairs_t + gh * rs.pairs_h + gw * rs.pairs_w;
   rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(table, Tkv, gh, gw, t0, rs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sumsq(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss, cudaStream_t s) {
+  if (tokens <= 0) return cudaSuccess;
+  sumsq_kernel<<<unsigned((tokens + 7) / 8), 256, 0, s>>>(x, tokens, channels, ss);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ struct Resolved {
   int sort_n;
   std::vector<int32_t> row_ptr;
   float scale;
+  int heads_total;     // heads of the whole (possibly head-sharded) layer
 };
 
 // Budget in blocks: topk_ratio = sparse_ratio * 768 * 1280 / (H * W) with the
@@ -77,6 +78,9 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   if (nb != 64 && nb != 128) return fail(LCSA_ERR_UNSUPPORTED, "block of %d tokens (64 or 128)", nb);
   if (c->block_t * c->block_h > 8)
     return fail(LCSA_ERR_UNSUPPORTED, "block_t*block_h = %d > 8 token rows", c->block_t * c->block_h);
+  if (c->heads_total != 0 && c->heads_total < c->heads)
+    return fail(LCSA_ERR_INVALID_ARG, "heads_total %d < heads %d", c->heads_total, c->heads);
+  r->heads_total = c->heads_total == 0 ? c->heads : c->heads_total;
 
   lcsa::Grid& g = r->grid;
   g.B = c->batch;
@@ -378,6 +382,7 @@ struct StepBlocks {
   int k_first_fb = 0;   // window frame-block of the k input's first one
   int slot0_fb = 0;     // ring slot of window frame-block 0
   const void* v_attn = nullptr;  // raster v seen by K3 (caller's tensor or the ring)
+  const float* ss_ext = nullptr; // head-sharded token-scope norm: reduced per-token sums of squares
 };
 
 lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float* gamma_q, const float* gamma_k,
@@ -409,6 +414,8 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k1.ring_fb = g.Tkv / g.bt;
   k1.slot0_fb = sb.slot0_fb;
   k1.Lk_in = int64_t(sb.k_in_fb) * g.bt * g.gh * g.gw;
+  k1.ss_ext = sb.ss_ext;
+  k1.norm_inv_c = 1.0f / float(int64_t(p->res.heads_total) * lcsa::kHeadDim);
 
   lcsa::K2Params k2;
   k2.g = g;
@@ -465,10 +472,14 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
 
 }  // namespace
 
-lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
-                           const float* gamma_k, void* out, void* stream) {
-  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
-  if (p->streaming) return fail(LCSA_ERR_INVALID_ARG, "a stream plan takes lcsa_forward_stream");
+namespace {
+
+bool sharded_token_norm(lcsa_plan_t p) {
+  return p->res.heads_total > p->res.grid.Hn && p->cfg.norm_scope == LCSA_NORM_TOKEN;
+}
+
+lcsa_status_t forward_common(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                             const float* gamma_k, const float* ssq, void* out, void* stream) {
   if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(gamma_q) ||
       !aligned16(gamma_k))
@@ -480,11 +491,53 @@ lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const vo
   StepBlocks sb;
   sb.k_in_fb = g.Tkv / g.bt;
   sb.v_attn = v;
+  sb.ss_ext = ssq;
   return run_step(p, q, k, gamma_q, gamma_k, out, s, sb);
+}
+
+}  // namespace
+
+lcsa_status_t lcsa_forward(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                           const float* gamma_k, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (p->streaming) return fail(LCSA_ERR_INVALID_ARG, "a stream plan takes lcsa_forward_stream");
+  if (sharded_token_norm(p))
+    return fail(LCSA_ERR_INVALID_ARG, "a head-sharded plan with token-scope norm takes lcsa_forward_sharded");
+  return forward_common(p, q, k, v, gamma_q, gamma_k, nullptr, out, stream);
+}
+
+lcsa_status_t lcsa_sumsq(lcsa_plan_t p, const void* q, const void* k, float* ssq, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (p->streaming) return fail(LCSA_ERR_INVALID_ARG, "stream plans are not head-sharded");
+  if (!q || !k || !ssq) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(ssq))
+    return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  const lcsa::Grid& g = p->res.grid;
+  const int64_t nq = int64_t(g.B) * g.Lq, nk = int64_t(g.B) * g.Lkv;
+  if ((e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(q), nq, g.C, ssq, s)) != cudaSuccess ||
+      (e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(k), nk, g.C, ssq + nq, s)) != cudaSuccess)
+    return cuda_fail(e, "sum of squares launch");
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_forward_sharded(lcsa_plan_t p, const void* q, const void* k, const void* v, const float* gamma_q,
+                                   const float* gamma_k, const float* ssq, void* out, void* stream) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (p->streaming) return fail(LCSA_ERR_INVALID_ARG, "stream plans are not head-sharded");
+  if (!ssq) return fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(ssq)) return fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
+  if (p->cfg.norm_scope != LCSA_NORM_TOKEN)
+    return fail(LCSA_ERR_INVALID_ARG, "head-scope norm needs no exchange: use lcsa_forward");
+  return forward_common(p, q, k, v, gamma_q, gamma_k, ssq, out, stream);
 }
 
 lcsa_status_t lcsa_plan_create_stream(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out) {
   if (cfg && cfg->host_io) return fail(LCSA_ERR_INVALID_ARG, "stream plans take device tensors (host_io = 0)");
+  if (cfg && cfg->heads_total != 0 && cfg->heads_total != cfg->heads)
+    return fail(LCSA_ERR_UNSUPPORTED, "stream plans are not head-sharded");
   lcsa_status_t st = lcsa_plan_create(cfg, cuda_device, out);
   if (st != LCSA_OK) return st;
   lcsa_plan* p = *out;

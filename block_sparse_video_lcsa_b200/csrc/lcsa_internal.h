@@ -77,6 +77,12 @@ struct K1Params {
   int ring_fb;          // KV window length in frame-blocks (Tkv / bt)
   int slot0_fb;         // ring slot of window frame-block 0
   int64_t Lk_in;        // tokens per batch element of the k input
+  // Head-sharded layer, token-scope norm: per-token sums of squares over all
+  // the layer's heads ([B*Lq] for q, then [B*Lk_in] for k), or null (the
+  // kernel sums the token's own channels); norm_inv_c = 1 / channels the
+  // mean runs over.
+  const float* ss_ext;
+  float norm_inv_c;
 };
 
 struct K2Params {
@@ -117,6 +123,9 @@ inline void k1_all_blocks(K1Params& k1) {
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, int d, cudaStream_t s);
 cudaError_t launch_prologue(const K1Params& p, cudaStream_t s);
+// Per-token sum of squares of x ([tokens][channels] bf16, channels a multiple
+// of 8, 16-byte aligned rows) into ss[tokens] (fp32).
+cudaError_t launch_sumsq(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss, cudaStream_t s);
 size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
 

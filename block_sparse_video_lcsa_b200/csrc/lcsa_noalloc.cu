@@ -140,6 +140,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
                                               const float* gamma_q, const float* gamma_k, void* out, void* stream) {
   if (!cfg) return noalloc_fail(LCSA_ERR_INVALID_ARG, "config is null");
   if (cfg->host_io) return noalloc_fail(LCSA_ERR_INVALID_ARG, "host_io needs staging buffers; use a plan");
+  if (cfg->heads_total != 0 && cfg->heads_total != cfg->heads)
+    return noalloc_fail(LCSA_ERR_UNSUPPORTED, "head-sharded layers need a plan (lcsa_forward_sharded)");
   NoallocGeom ng;
   lcsa_status_t st = noalloc_resolve(cfg, &ng);
   if (st != LCSA_OK) return st;
@@ -223,6 +225,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.err = err;
   k1.split_part = split_part;
   k1.split_cnt = split_cnt;
+  k1.ss_ext = nullptr;
+  k1.norm_inv_c = 1.0f / float(g.C);
   lcsa::k1_all_blocks(k1);
   if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "device attributes");

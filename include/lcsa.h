@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define LCSA_ABI_VERSION 1
+#define LCSA_ABI_VERSION 2  /* 2: lcsa_config_t.heads_total, head-sharded entry points */
 
 #if defined(__GNUC__)
 #define LCSA_API __attribute__((visibility("default")))
@@ -106,6 +106,8 @@ typedef struct lcsa_config {
   float rms_eps;        /* > 0 */
   float softmax_scale;  /* 0: 1/sqrt(head_dim) */
   int host_io;          /* 1: also allocate device staging for lcsa_forward_host */
+  int heads_total;      /* 0, or the heads of the whole layer when this plan holds
+                           `heads` of them (head-sharded; see lcsa_forward_sharded) */
 } lcsa_config_t;
 
 /* Sizes derived from a configuration (host-side, no device needed). */
@@ -180,6 +182,30 @@ LCSA_API lcsa_status_t lcsa_stream_push(lcsa_plan_t plan, const void* k, const v
                                         int frames, void* stream);
 LCSA_API lcsa_status_t lcsa_forward_stream(lcsa_plan_t plan, const void* q, const void* k, const void* v,
                                            const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
+/* Head-sharded layers: the tensor-parallel form of the pages ("Add FlashVSR
+   contrib model with video super-resolution on Neuron", Model Information
+   and Additional Information: the QK RMSNorm all-reduces across the ranks
+   that hold a layer's heads, so it spans all heads of a token). A plan with
+   heads_total > heads holds `heads` consecutive heads of a layer of
+   heads_total heads: q, k, v, out and the gains are the plan's slice
+   ([batch][tokens][heads*d], gains [heads*d]). With token-scope norm the
+   RMS mean runs over heads_total*head_dim channels, so each rank:
+     1. lcsa_sumsq writes ssq (device fp32, 16-byte aligned,
+        batch*(q_tokens + kv_tokens) entries): per token the sum of squares of
+        its own q channels (batch-major, first batch*q_tokens entries), then of
+        its own k channels;
+     2. sums ssq over the ranks (an all-reduce, by the caller: NCCL);
+     3. lcsa_forward_sharded runs lcsa_forward with the norm taken from the
+        reduced ssq (it must hold the sums over all heads_total heads).
+   lcsa_forward rejects such a plan (LCSA_ERR_INVALID_ARG). With head-scope
+   norm no exchange is needed and lcsa_forward serves sharded plans directly
+   (lcsa_forward_sharded then returns LCSA_ERR_INVALID_ARG). Stream plans and
+   lcsa_forward_noalloc are not head-sharded (LCSA_ERR_UNSUPPORTED). */
+LCSA_API lcsa_status_t lcsa_sumsq(lcsa_plan_t plan, const void* q, const void* k, float* ssq, void* stream);
+LCSA_API lcsa_status_t lcsa_forward_sharded(lcsa_plan_t plan, const void* q, const void* k, const void* v,
+                                            const float* gamma_q, const float* gamma_k, const float* ssq, void* out,
+                                            void* stream);
 
 /* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
    Every GPU that loads the library holds this array until the process exits. */

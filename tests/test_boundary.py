@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported_and_bound():
 
 
 def test_abi_version_and_status_strings():
-    assert L.lcsa_abi_version() == 1
+    assert L.lcsa_abi_version() == L.ABI_VERSION == 2
     for code in range(9):
         assert L.lcsa_status_string(code).startswith("LCSA_")
 
