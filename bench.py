@@ -54,6 +54,10 @@ def _args():
                     help="time N sequential calls (a DiT chunk's attention layers), eager and as one CUDA graph")
     ap.add_argument("--stream", action="store_true",
                     help="time a stream plan: each step brings the chunk's new frames into the KV ring")
+    ap.add_argument("--reuse", action="store_true",
+                    help="threshold reuse: calls after the first keep blocks by the recorded thresholds (no top-k)")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="one layer's heads split over the ranks: per-token sums of squares all-reduced (NCCL)")
     return ap.parse_args()
 
 
@@ -262,6 +266,8 @@ def run_lcsa(args):
     geo = plan.geometry
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if args.reuse:
+        plan.lcsa_plan_set_threshold_reuse(True)
 
     for _ in range(args.warmup):
         plan.lcsa_forward(q, k, v, gq, gk, out, stream)
@@ -297,6 +303,7 @@ def run_lcsa(args):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kms, kcount = plan.lcsa_get_kernel_times()
     plan.lcsa_plan_set_timing(0)
+    kept = plan.lcsa_selection_nnz()  # the blocks the timed calls kept (threshold reuse may differ from k)
     total_ms = _max_over_ranks(sum(step_ms), dev)
 
     # end to end: pinned host buffers through lcsa_forward_host (copies inside)
@@ -329,7 +336,7 @@ def run_lcsa(args):
         return 0
 
     peaks = _peaks()
-    flops = geo.selected_flops
+    flops = geo.selected_flops * kept / geo.nnz
     ms_per_step = total_ms / args.steps
     value = world * flops / (ms_per_step * 1e-3) / 1e12
     k3_tflops = flops / (kms[2] * 1e-3) / 1e12
@@ -348,7 +355,8 @@ def run_lcsa(args):
             "config": {"workload": wl.name, "q_tokens": geo.q_tokens, "kv_tokens": geo.kv_tokens,
                        "heads": wl.heads, "head_dim": wl.head_dim,
                        "block": "%dx%dx%d" % (wl.block_t, wl.block_h, wl.block_w), "local_range": wl.local_range,
-                       "sparse_ratio": wl.sparse_ratio, "topk": geo.topk, "kept_blocks": geo.nnz,
+                       "sparse_ratio": wl.sparse_ratio, "topk": geo.topk, "kept_blocks": kept,
+                       "selection": "threshold reuse (recorded on the warm-up)" if args.reuse else "top-k",
                        "l2": "256 MiB buffer written before every timed call", "parallelism": "replicas%d" % world,
                        "kernel_times": "second pass of the same calls, CUDA events around each kernel"},
             "roofline": roofline,
@@ -539,6 +547,99 @@ def run_layers(args):
     return 0
 
 
+def run_sharded(args):
+    """One step = one layer's LCSA call with its heads split over the ranks
+    (strong scaling: the layer is fixed, each rank computes its heads): the
+    rank's per-token sums of squares, their all-reduce and the sharded call."""
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_video_lcsa_b200 as lcsa
+    from block_sparse_video_lcsa_b200 import synth
+    from block_sparse_video_lcsa_b200.sharded import forward_heads_sharded, head_slices, sumsq_buffer
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl)  # the same layer on every rank
+    h0, h1 = head_slices(wl.heads, world)[rank]
+    D = wl.head_dim
+    sl = slice(h0 * D, h1 * D)
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16)[..., sl].contiguous().to(dev)
+
+    q, k, v = bf(inp.q), bf(inp.k), bf(inp.v)
+    gq, gk = torch.from_numpy(inp.gamma_q[sl].copy()).to(dev), torch.from_numpy(inp.gamma_k[sl].copy()).to(dev)
+    out = torch.empty_like(q)
+    plan = lcsa.lcsa_plan_create(lcsa.config_from_workload(wl, heads=h1 - h0, heads_total=wl.heads), local)
+    full_geo = lcsa.lcsa_config_resolve(lcsa.config_from_workload(wl))
+    ssq = sumsq_buffer(plan, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        forward_heads_sharded(plan, q, k, v, gq, gk, out, ssq=ssq)
+    plan.lcsa_check_device_error(stream)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    s_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    s_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    try:
+        gpu_id = "GPU-%s" % torch.cuda.get_device_properties(dev).uuid
+    except Exception:  # noqa: BLE001 - fall back to the index
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            forward_heads_sharded(plan, q, k, v, gq, gk, out, ssq=ssq)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        # the sums-of-squares kernel alone
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            s_starts[i].record(stream)
+            plan.lcsa_sumsq(q, k, ssq, stream)
+            s_ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    plan.lcsa_check_device_error(stream)
+    ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps, dev)
+    ss_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(s_starts, s_ends)) / args.steps, dev)
+    ss_bytes = (q.numel() + k.numel()) * 2 + ssq.numel() * 4
+    plan.destroy()
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+    peaks = _peaks()
+    flops = full_geo.selected_flops
+    line = {"metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name + " (heads split over the ranks, sums of squares all-reduced)",
+                       "heads_per_rank": [b - a for a, b in head_slices(wl.heads, world)],
+                       "l2": "256 MiB buffer written before every timed call", "parallelism": "heads%d" % world},
+            "sumsq": {"ms": ss_ms, "bytes": ss_bytes, "gbs": ss_bytes / (ss_ms * 1e-3) / 1e9,
+                      "hbm_frac": ss_bytes / (ss_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
@@ -547,6 +648,8 @@ def main():
         return run_stream(args)
     if args.layers > 0:
         return run_layers(args)
+    if args.shard_heads:
+        return run_sharded(args)
     return run_lcsa(args)
 
 

@@ -84,6 +84,8 @@ SIGNATURES = [
     ("lcsa_stream_push", _I, [_PLAN, _VP, _VP, _VP, _I, _VP]),
     ("lcsa_forward_stream", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_sumsq", _I, [_PLAN, _VP, _VP, _VP, _VP]),
+    ("lcsa_plan_set_threshold_reuse", _I, [_PLAN, _I]),
+    ("lcsa_selection_nnz", _I, [_PLAN, ctypes.POINTER(ctypes.c_int64)]),
     ("lcsa_forward_sharded", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_plan_geometry", _I, [_PLAN, ctypes.POINTER(lcsa_geometry_t)]),
     ("lcsa_plan_topk", _I, [_PLAN, ctypes.POINTER(_I)]),
@@ -310,14 +312,24 @@ class Plan:
         _check(lib().lcsa_plan_topk(self._h, ctypes.byref(k)), "lcsa_plan_topk")
         return k.value
 
+    def lcsa_plan_set_threshold_reuse(self, on: bool):
+        """Later calls keep blocks by the recorded per-row thresholds instead of selecting the top k."""
+        _check(lib().lcsa_plan_set_threshold_reuse(self._h, 1 if on else 0), "lcsa_plan_set_threshold_reuse")
+
+    def lcsa_selection_nnz(self) -> int:
+        n = ctypes.c_int64()
+        _check(lib().lcsa_selection_nnz(self._h, ctypes.byref(n)), "lcsa_selection_nnz")
+        return n.value
+
     def lcsa_get_selection(self):
         import numpy as np
         g = self.geometry
+        nnz = self.lcsa_selection_nnz()
         rp = np.empty(g.rows + 1, dtype=np.int32)
-        ci = np.empty(max(1, g.nnz), dtype=np.int32)
+        ci = np.empty(max(1, nnz), dtype=np.int32)
         _check(lib().lcsa_get_selection(self._h, rp.ctypes.data, rp.size, ci.ctypes.data, ci.size),
                "lcsa_get_selection")
-        return rp, ci[: g.nnz]
+        return rp, ci[:nnz]
 
     def lcsa_get_intermediates(self):
         """(q^, k^ as uint16 bf16 bits, pooled q, pooled k) in the plan's layouts."""

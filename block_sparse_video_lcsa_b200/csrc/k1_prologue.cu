@@ -529,27 +529,37 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// One warp per token: 16-byte chunks strided over the lanes, fp32 squares,
-// then a butterfly.
-__global__ void __launch_bounds__(256) sumsq_kernel(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss) {
+// One warp per token (q tokens, then k tokens): every 16-byte chunk of the
+// token is requested before any is summed (at most 8 per lane: heads <= 16),
+// fp32 squares, then a butterfly.
+__global__ void __launch_bounds__(256) sumsq_kernel(const __nv_bfloat16* xq, int64_t nq, const __nv_bfloat16* xk,
+                                                    int64_t nk, int channels, float* ss) {
   const int64_t t = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= tokens) return;
-  const uint4* row = reinterpret_cast<const uint4*>(x + t * channels);
-  float2 acc = make_float2(0.f, 0.f);
-  for (int c = lane; c < channels / 8; c += 32) {
+  if (t >= nq + nk) return;
+  const uint4* row = reinterpret_cast<const uint4*>(t < nq ? xq + t * channels : xk + (t - nq) * channels);
+  const int nch = channels / 8;
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = lane + 32 * i;
+    v[i] = c < nch ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
     float2 e[2], o[2];
-    unpack_eo(__ldg(row + c), e, o);
+    unpack_eo(v[i], e, o);
 #pragma unroll
     for (int qg = 0; qg < 2; ++qg) {
-      acc = __ffma2_rn(e[qg], e[qg], acc);
-      acc = __ffma2_rn(o[qg], o[qg], acc);
+      acc[qg] = __ffma2_rn(e[qg], e[qg], acc[qg]);
+      acc[qg] = __ffma2_rn(o[qg], o[qg], acc[qg]);
     }
   }
-  float v = acc.x + acc.y;
+  float sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
 #pragma unroll
-  for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-  if (lane == 0) ss[t] = v;
+  for (int o2 = 16; o2 > 0; o2 >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o2);
+  if (lane == 0) ss[t] = sum;
 }
 
 }  // namespace
@@ -561,9 +571,11 @@ cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_sumsq(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss, cudaStream_t s) {
-  if (tokens <= 0) return cudaSuccess;
-  sumsq_kernel<<<unsigned((tokens + 7) / 8), 256, 0, s>>>(x, tokens, channels, ss);
+cudaError_t launch_sumsq(const __nv_bfloat16* q, int64_t nq, const __nv_bfloat16* k, int64_t nk, int channels,
+                         float* ss, cudaStream_t s) {
+  if (channels % 8 || channels > 2048) return cudaErrorInvalidValue;
+  if (nq + nk <= 0) return cudaSuccess;
+  sumsq_kernel<<<unsigned((nq + nk + 7) / 8), 256, 0, s>>>(q, nq, k, nk, channels, ss);
   return cudaGetLastError();
 }
 

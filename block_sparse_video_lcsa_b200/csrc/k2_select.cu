@@ -21,6 +21,13 @@
 // both a bitonic sort and counting each candidate's rank, at 180 and at up
 // to 726 candidates per row). The CSR row offsets
 // depend only on the geometry and are computed once when the plan is made.
+//
+// Threshold reuse (the same pages, Remove the remaining control-plane tax and
+// Measured Results: the mask-generation threshold of the previous steady
+// chunk reused per DiT block): a selecting call records each row's k-th best
+// score (its order bits); a reuse call keeps every admissible block scoring at
+// least that, in ascending order, into the row's slot of a padded CSR with a
+// count per row; a row where no block reaches it keeps its best block.
 #include "lcsa_internal.h"
 
 namespace lcsa {
@@ -102,7 +109,35 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   __syncthreads();
 
   const int keff = min(p.topk, nc);
-  {
+  if (p.reuse) {
+    // threshold reuse: every admissible block scoring at least the recorded
+    // k-th best score of this row
+    const unsigned th = p.thresh[rr];
+    int any = 0;
+    for (int c = threadIdx.x; c < nc; c += kThreads) {
+      const unsigned char f = unsigned(keys[c] >> 32) >= th;
+      flag[c] = f;
+      any |= f;
+    }
+    if (!__syncthreads_or(any)) {
+      // no block reaches it: keep the row's best block (largest key: highest
+      // score, then the lower block)
+      __shared__ unsigned long long wmax[kWarps];
+      unsigned long long mk = 0ull;
+      for (int c = threadIdx.x; c < nc; c += kThreads) mk = keys[c] > mk ? keys[c] : mk;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long t = __shfl_xor_sync(0xffffffffu, mk, o);
+        mk = t > mk ? t : mk;
+      }
+      if (lane == 0) wmax[warp] = mk;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        for (int w = 1; w < kWarps; ++w) mk = wmax[w] > mk ? wmax[w] : mk;
+        flag[0xFFFFFFFFu - unsigned(mk & 0xFFFFFFFFull)] = 1;
+      }
+    }
+  } else {
     // the k-th largest score (order-preserving bits, four 8-bit digits from
     // the top, one shared histogram per digit), then all candidates above it
     // and the lowest-numbered `remain` of those equal to it (equal scores go
@@ -172,6 +207,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
       if (sb == prefix) keep = unsigned(tr++) < remain;
       flag[c] = keep;
     }
+    // the threshold a later reuse call applies (all blocks kept: any score)
+    if (p.thresh && threadIdx.x == 0) p.thresh[rr] = keff < nc ? prefix : 0u;
   }
   __syncthreads();
   const int span = (nc + kThreads - 1) / kThreads;
@@ -188,10 +225,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   __syncthreads();
   int base = 0;
   for (int w = 0; w < warp; ++w) base += warp_sum[w];
-  int pos = p.row_ptr[rr] + base + incl - cnt;
+  int* dst = p.reuse ? p.col_pad + int64_t(rr) * p.pad_cap : p.col_idx + p.row_ptr[rr];
+  int pos = base + incl - cnt;
   for (int c = c_beg; c < c_end; ++c) {
-    if (flag[c]) p.col_idx[pos++] = cand_block(c, false);  // window order
+    if (flag[c]) dst[pos++] = cand_block(c, false);  // window order
   }
+  if (p.reuse && threadIdx.x == kThreads - 1) p.row_len[rr] = pos;  // the last thread's end is the row's count
 }
 
 }  // namespace

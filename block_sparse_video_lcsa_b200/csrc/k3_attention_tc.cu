@@ -115,11 +115,21 @@ struct TcParams {
   int ring_fb, slot0_fb;
   const int* row_ptr;
   const int* col_idx;
+  const int* row_len;  // null, or the counts of a padded CSR (threshold reuse)
+  int pad_cap;
   __nv_bfloat16* out;
   float scale_log2;
   unsigned* err;
   int rows;
 };
+
+// Selected blocks of row rr: col_idx[row_begin .. row_begin + row_count).
+__device__ __forceinline__ int64_t row_begin(const TcParams& p, int rr) {
+  return p.row_len ? int64_t(rr) * p.pad_cap : int64_t(p.row_ptr[rr]);
+}
+__device__ __forceinline__ int row_count(const TcParams& p, int rr) {
+  return p.row_len ? p.row_len[rr] : p.row_ptr[rr + 1] - p.row_ptr[rr];
+}
 
 // ---- PTX wrappers ---------------------------------------------------------
 
@@ -411,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, row_it = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int beg = p.row_ptr[rr], n = p.row_ptr[rr + 1] - beg;
+      const int64_t beg = row_begin(p, rr);
+      const int n = row_count(p, rr);
       const int bhh = rr / g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       if (row_it > 0 && !(ok = warp_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1))) break;
@@ -488,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, s_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = (p.row_ptr[rr + 1] - p.row_ptr[rr] + KB - 1) / KB;  // KV tiles of the row
+      const int n = (row_count(p, rr) + KB - 1) / KB;  // KV tiles of the row
       if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
       for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
@@ -528,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = (p.row_ptr[rr + 1] - p.row_ptr[rr] + KB - 1) / KB;  // KV tiles of the row
+      const int n = (row_count(p, rr) + KB - 1) / KB;  // KV tiles of the row
       for (int j = 0; j < n; ++j, ++pv_it) {
         const int pb = pv_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
@@ -577,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_it = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
-      const int n_sel = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n_sel = row_count(p, rr);
       const int n = (n_sel + 1) / 2;  // KV tiles of the row, two blocks each
       float mu[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
       for (int j = 0; j < n && ok; ++j, ++s_it) {
@@ -748,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_it = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
-      const int n_sel = p.row_ptr[rr + 1] - p.row_ptr[rr];
+      const int n_sel = row_count(p, rr);
       const int n = n_sel;  // KV tiles of the row
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j, ++s_it) {
@@ -958,6 +969,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   TcParams tp;
   tp.g = p.g;
   tp.row_ptr = p.row_ptr;
+  tp.row_len = p.row_len;
+  tp.pad_cap = p.pad_cap;
   tp.col_idx = p.col_idx;
   tp.out = p.out;
   tp.scale_log2 = p.scale_log2;

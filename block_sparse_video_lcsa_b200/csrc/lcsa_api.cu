@@ -179,6 +179,7 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   ws += size_t(g.B) * g.Lq * g.C * 2 + size_t(g.B) * g.Lkv * g.C * 2;            // q^, k^
   ws += size_t(g.B) * g.Hn * (g.nQB + g.nKB) * size_t(c->head_dim) * 4;         // pooled
   ws += (size_t(rows) + 1) * 4 + size_t(nnz) * 4;                                // CSR
+  ws += size_t(rows) * (8 + size_t(wmax) * 4);                                    // threshold reuse
   ws += rope_n * sizeof(float2) + 256;
   ws += size_t(lcsa::kMaxK1Ctas) * (2 * size_t(g.C) * 4 + 4);                    // K1 split blocks
   if (c->host_io)
@@ -206,6 +207,14 @@ struct lcsa_plan {
   unsigned* split_cnt = nullptr;   // K1: arrivals per cut (K2 zeroes them after use)
   int32_t* row_ptr = nullptr;
   int32_t* col_idx = nullptr;
+  // threshold reuse: recorded k-th best scores (order bits) and the padded
+  // CSR of reuse calls (max_window entries per row, a count per row)
+  unsigned* thresh = nullptr;
+  int32_t* row_len = nullptr;
+  int32_t* col_pad = nullptr;
+  bool reuse_mode = false;   // lcsa_plan_set_threshold_reuse
+  bool have_thresh = false;  // a selecting call has recorded thresholds
+  bool last_reuse = false;   // the last call kept blocks by threshold
   float2* rope = nullptr;
   int rope_h_off = 0, rope_w_off = 0;
   unsigned* err = nullptr;
@@ -228,7 +237,7 @@ namespace {
 void release(lcsa_plan* p) {
   void* ptrs[] = {p->v_ring, p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
                   p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
-                  p->st_v,  p->st_out,  p->st_gq,    p->st_gk};
+                  p->st_v,  p->st_out,  p->st_gq,    p->st_gk,    p->thresh,     p->row_len, p->col_pad};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (auto& set : p->evsets)
@@ -315,6 +324,9 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
       (st = dev_alloc(&p->pooled_k, size_t(g.B) * g.Hn * g.nKB * D * 4, "pooled k")) ||
       (st = dev_alloc(&p->row_ptr, (rows + 1) * 4, "row_ptr")) ||
       (st = dev_alloc(&p->col_idx, nnz * 4, "col_idx")) ||
+      (st = dev_alloc(&p->thresh, rows * 4, "thresholds")) ||
+      (st = dev_alloc(&p->row_len, rows * 4, "row counts")) ||
+      (st = dev_alloc(&p->col_pad, rows * size_t(p->res.geo.max_window) * 4, "padded col_idx")) ||
       (st = dev_alloc(&p->rope, rope_n * sizeof(float2), "rope table")) ||
       (st = dev_alloc(&p->err, 256, "error word")) ||
       (st = dev_alloc(&p->split_part, size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4, "K1 split sums")) ||
@@ -430,6 +442,12 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k2.n_clear = lcsa::kMaxK1Ctas;
   k2.ring_fb = g.Tkv / g.bt;
   k2.slot0_fb = sb.slot0_fb;
+  const bool reuse = p->reuse_mode && p->have_thresh;
+  k2.thresh = p->thresh;
+  k2.reuse = reuse ? 1 : 0;
+  k2.col_pad = p->col_pad;
+  k2.row_len = p->row_len;
+  k2.pad_cap = p->res.geo.max_window;
 
   lcsa::K3Params k3;
   k3.g = g;
@@ -438,7 +456,9 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k3.v = static_cast<const __nv_bfloat16*>(sb.v_attn);
   k3.out = static_cast<__nv_bfloat16*>(out);
   k3.row_ptr = p->row_ptr;
-  k3.col_idx = p->col_idx;
+  k3.col_idx = reuse ? p->col_pad : p->col_idx;
+  k3.row_len = reuse ? p->row_len : nullptr;
+  k3.pad_cap = p->res.geo.max_window;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
   k3.err = p->err;
   k3.ring_fb = g.Tkv / g.bt;
@@ -456,6 +476,8 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   }
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  p->have_thresh = true;
+  p->last_reuse = reuse;
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
   {
     CUtensorMap tm_v;
@@ -517,8 +539,8 @@ lcsa_status_t lcsa_sumsq(lcsa_plan_t p, const void* q, const void* k, float* ssq
   if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
   const lcsa::Grid& g = p->res.grid;
   const int64_t nq = int64_t(g.B) * g.Lq, nk = int64_t(g.B) * g.Lkv;
-  if ((e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(q), nq, g.C, ssq, s)) != cudaSuccess ||
-      (e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(k), nk, g.C, ssq + nq, s)) != cudaSuccess)
+  if ((e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(q), nq, static_cast<const __nv_bfloat16*>(k), nk,
+                              g.C, ssq, s)) != cudaSuccess)
     return cuda_fail(e, "sum of squares launch");
   return LCSA_OK;
 }
@@ -655,9 +677,55 @@ lcsa_status_t lcsa_plan_topk(lcsa_plan_t p, int* k_out) {
   return LCSA_OK;
 }
 
+lcsa_status_t lcsa_plan_set_threshold_reuse(lcsa_plan_t p, int on) {
+  if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
+  if (on != 0 && on != 1) return fail(LCSA_ERR_INVALID_ARG, "on = %d (0 or 1)", on);
+  p->reuse_mode = on != 0;
+  return LCSA_OK;
+}
+
+lcsa_status_t lcsa_selection_nnz(lcsa_plan_t p, int64_t* nnz) {
+  if (!p || !nnz) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  if (!p->last_reuse) {
+    *nnz = p->res.geo.nnz;
+    return LCSA_OK;
+  }
+  const size_t rows = size_t(p->res.geo.rows);
+  std::vector<int32_t> len(rows);
+  cudaError_t e = cudaSetDevice(p->device);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(len.data(), p->row_len, rows * 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "copy row counts");
+  int64_t n = 0;
+  for (int32_t v : len) n += v;
+  *nnz = n;
+  return LCSA_OK;
+}
+
 lcsa_status_t lcsa_get_selection(lcsa_plan_t p, int32_t* row_ptr, size_t row_ptr_cap, int32_t* col_idx,
                                  size_t col_idx_cap) {
   if (!p || !row_ptr || !col_idx) return fail(LCSA_ERR_INVALID_ARG, "null argument");
+  if (p->last_reuse) {
+    // the padded CSR of a reuse call, compacted on the host
+    const size_t rows = size_t(p->res.geo.rows), cap = size_t(p->res.geo.max_window);
+    std::vector<int32_t> len(rows), pad(rows * cap);
+    cudaError_t e = cudaSetDevice(p->device);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(len.data(), p->row_len, rows * 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(pad.data(), p->col_pad, rows * cap * 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "copy selection");
+    size_t n = 0;
+    for (size_t r = 0; r < rows; ++r) n += size_t(len[r]);
+    if (row_ptr_cap < rows + 1 || col_idx_cap < n)
+      return fail(LCSA_ERR_INVALID_ARG, "capacity %zu/%zu < %zu/%zu", row_ptr_cap, col_idx_cap, rows + 1, n);
+    row_ptr[0] = 0;
+    for (size_t r = 0; r < rows; ++r) {
+      if (len[r] < 0 || size_t(len[r]) > cap) return fail(LCSA_ERR_DEVICE_BOUNDS, "row %zu count %d", r, len[r]);
+      std::memcpy(col_idx + row_ptr[r], pad.data() + r * cap, size_t(len[r]) * 4);
+      row_ptr[r + 1] = row_ptr[r] + len[r];
+    }
+    return LCSA_OK;
+  }
   const size_t rows = size_t(p->res.geo.rows), nnz = size_t(p->res.geo.nnz);
   if (row_ptr_cap < rows + 1 || col_idx_cap < nnz)
     return fail(LCSA_ERR_INVALID_ARG, "capacity %zu/%zu < %zu/%zu", row_ptr_cap, col_idx_cap, rows + 1, nnz);

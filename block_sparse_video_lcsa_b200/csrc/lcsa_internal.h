@@ -97,6 +97,16 @@ struct K2Params {
   unsigned* clear_cnt;  // K1's split counters, zeroed here for the next K1 (n_clear entries)
   int n_clear;
   int ring_fb, slot0_fb;  // pooled k of window frame-block tk sits in ring slot (slot0_fb + tk) % ring_fb
+  // Threshold reuse. thresh[row]: order bits of the row's k-th best score.
+  // reuse == 0: select the top k (row_ptr / col_idx) and, if thresh is set,
+  // record the thresholds. reuse == 1: keep every admissible block whose
+  // score is >= the recorded threshold, in ascending order, into row r's
+  // padded slot col_pad[r * pad_cap ...], its count into row_len[r].
+  unsigned* thresh;
+  int reuse;
+  int* col_pad;
+  int* row_len;
+  int pad_cap;
 };
 
 struct K3Params {
@@ -110,6 +120,10 @@ struct K3Params {
   float scale_log2;         // softmax scale * log2(e)
   unsigned* err;
   int ring_fb, slot0_fb;    // k^ / v of window frame-block tk sit in ring slot (slot0_fb + tk) % ring_fb
+  // null: row r's blocks are col_idx[row_ptr[r] .. row_ptr[r+1]); else they
+  // are col_idx[r * pad_cap ...], row_len[r] of them (threshold reuse)
+  const int* row_len;
+  int pad_cap;
 };
 
 // The stateless call's block sets: every query and key block, ring = window.
@@ -123,9 +137,10 @@ inline void k1_all_blocks(K1Params& k1) {
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_rope_table(float2* table, int Tkv, int gh, int gw, int t0, int d, cudaStream_t s);
 cudaError_t launch_prologue(const K1Params& p, cudaStream_t s);
-// Per-token sum of squares of x ([tokens][channels] bf16, channels a multiple
-// of 8, 16-byte aligned rows) into ss[tokens] (fp32).
-cudaError_t launch_sumsq(const __nv_bfloat16* x, int64_t tokens, int channels, float* ss, cudaStream_t s);
+// Per-token sums of squares of q ([nq][channels] bf16) then k ([nk][channels])
+// into ss[nq + nk] (fp32); channels a multiple of 8, at most 2048.
+cudaError_t launch_sumsq(const __nv_bfloat16* q, int64_t nq, const __nv_bfloat16* k, int64_t nk, int channels,
+                         float* ss, cudaStream_t s);
 size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
 

@@ -247,6 +247,11 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.n_clear = lcsa::kMaxK1Ctas;
   k2.ring_fb = g.Tkv / g.bt;
   k2.slot0_fb = 0;
+  k2.thresh = nullptr;  // no threshold reuse without a plan
+  k2.reuse = 0;
+  k2.col_pad = nullptr;
+  k2.row_len = nullptr;
+  k2.pad_cap = 0;
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
 
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));
@@ -262,6 +267,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.err = err;
   k3.ring_fb = g.Tkv / g.bt;
   k3.slot0_fb = 0;
+  k3.row_len = nullptr;
+  k3.pad_cap = 0;
   {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;

@@ -207,6 +207,21 @@ LCSA_API lcsa_status_t lcsa_forward_sharded(lcsa_plan_t plan, const void* q, con
                                             const float* gamma_q, const float* gamma_k, const float* ssq, void* out,
                                             void* stream);
 
+/* Threshold reuse: the mask-generation threshold of the previous steady
+   chunk reused per DiT block ("FlashVSR: From 17.2 FPS to 57.3 FPS at
+   768x1408", Remove the remaining control-plane tax and Measured Results; a
+   plan is one DiT block's attention). Every call that selects records, per
+   query block, the score of its k-th best block. With reuse on, later calls
+   (lcsa_forward, lcsa_forward_stream, lcsa_forward_sharded) skip the top-k
+   selection and keep every admissible block whose score is at least the
+   recorded one (ascending order; a query block where none reaches it keeps
+   its best block), so a query block may keep more or fewer than k blocks: an
+   approximation the caller gates on quality. A call with reuse on and no
+   recorded thresholds selects (and records). on: 1 reuse, 0 select every call.
+   lcsa_selection_nnz: total kept blocks of the last call (synchronises). */
+LCSA_API lcsa_status_t lcsa_plan_set_threshold_reuse(lcsa_plan_t plan, int on);
+LCSA_API lcsa_status_t lcsa_selection_nnz(lcsa_plan_t plan, int64_t* nnz);
+
 /* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
    Every GPU that loads the library holds this array until the process exits. */
 #define LCSA_NOALLOC_WORKSPACE_BYTES (32u << 20)
@@ -236,7 +251,8 @@ LCSA_API lcsa_status_t lcsa_plan_geometry(lcsa_plan_t plan, lcsa_geometry_t* out
 /* Resolved budget k in blocks. */
 LCSA_API lcsa_status_t lcsa_plan_topk(lcsa_plan_t plan, int* k_out);
 
-/* Copy the last call's CSR to host: row_ptr [rows+1], col_idx [nnz]. The
+/* Copy the last call's CSR to host: row_ptr [rows+1], col_idx [nnz] (nnz:
+   the geometry's, or lcsa_selection_nnz after a threshold-reuse call). The
    capacities are element counts; too small -> LCSA_ERR_INVALID_ARG.
    Synchronises the device. */
 LCSA_API lcsa_status_t lcsa_get_selection(lcsa_plan_t plan, int32_t* row_ptr, size_t row_ptr_cap,

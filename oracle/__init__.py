@@ -190,6 +190,41 @@ def select(g: Geometry, pq: np.ndarray, pk: np.ndarray, want_scores: bool = Fals
     return Selection(row_len, cols, gap, scores)
 
 
+def kth_thresholds(g: Geometry, scores: np.ndarray) -> np.ndarray:
+    """Per row, the score of its k-th best admissible block (-inf when the
+    budget covers the whole window): the threshold a selecting call records
+    for later reuse ("FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408",
+    Remove the remaining control-plane tax: the mask-generation threshold of
+    the previous steady chunk, reused per DiT block). scores: [rows, nKB]
+    fp64 from select(want_scores=True), non-finite where not admissible."""
+    th = np.full(scores.shape[0], -np.inf)
+    for r in range(scores.shape[0]):
+        adm = np.sort(scores[r][np.isfinite(scores[r])])[::-1]
+        if g.topk < adm.size:
+            th[r] = adm[g.topk - 1]
+    return th
+
+
+def threshold_select(g: Geometry, scores: np.ndarray, thresholds: np.ndarray) -> Selection:
+    """Selection by a reused threshold (same pages and passage): per row every
+    admissible block whose score is >= the row's threshold, ascending; a row
+    where none reaches it keeps its best block (the lower index among equal
+    scores). Rows may keep more or fewer than k blocks."""
+    rows, nkb = scores.shape
+    cols = np.full((rows, nkb), -1, dtype=np.int32)
+    row_len = np.zeros(rows, dtype=np.int32)
+    for r in range(rows):
+        sc = scores[r]
+        adm = np.isfinite(sc)
+        keep = np.flatnonzero(adm & (sc >= thresholds[r]))
+        if keep.size == 0:
+            best = np.max(sc[adm])
+            keep = np.flatnonzero(adm & (sc == best))[:1]
+        row_len[r] = keep.size
+        cols[r, : keep.size] = keep
+    return Selection(row_len, cols, np.full(rows, np.inf), scores)
+
+
 def attention(g: Geometry, q, k, v, gamma_q, gamma_k, sel: Selection, rows=None):
     """fp64 outputs [nrows, nb, d] and weight sums [nrows, nb] of the given rows."""
     if rows is None:

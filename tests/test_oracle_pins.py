@@ -294,3 +294,58 @@ def test_pooled_score_is_mean_of_token_dot_products():
                 tk = block_raster_tokens(g, kb)
                 dots = qt[tq, h * D:(h + 1) * D] @ kt[tk, h * D:(h + 1) * D].T
                 assert pq[0, h, qb] @ pk[0, h, kb] == pytest.approx(dots.mean(), rel=1e-12, abs=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Threshold reuse: on the scores it was recorded from, the recorded k-th best
+# score keeps exactly the top-k selection (where the k-th and (k+1)-th scores
+# differ); no threshold keeps the whole window; a threshold above every score
+# keeps the single best block.
+
+def test_threshold_of_a_selection_reproduces_it():
+    wl, g = tiny(grid_h=48, grid_w=48, q_frames=1, kv_frames=2, local_range=5, topk=7, field=True,
+                 unit_gain=False, seed=9)
+    inp = synth.make_inputs(wl)
+    pq = oracle.pool(g, inp.q, inp.gamma_q, True)
+    pk = oracle.pool(g, inp.k, inp.gamma_k, False)
+    sel = oracle.select(g, pq, pk, want_scores=True)
+    th = oracle.kth_thresholds(g, sel.scores)
+    again = oracle.threshold_select(g, sel.scores, th)
+    sizes = oracle.window_sizes(g)
+    checked = 0
+    for r in range(g.rows):
+        if sel.gap[r] <= 0:
+            continue
+        np.testing.assert_array_equal(again.row(r), sel.row(r))
+        # the threshold is the k-th best score of the admissible set
+        adm = np.sort(sel.scores[r][np.isfinite(sel.scores[r])])[::-1]
+        assert adm.size == sizes[r % g.nQB]
+        if g.topk < adm.size:
+            assert th[r] == adm[g.topk - 1] and adm[g.topk] < th[r]
+        else:
+            assert th[r] == -np.inf
+        checked += 1
+    assert checked > g.rows // 2
+
+
+def test_threshold_extremes_keep_all_or_the_best_block():
+    wl, g = tiny(grid_h=32, grid_w=32, q_frames=1, kv_frames=2, local_range=3, topk=3, field=True,
+                 unit_gain=False, seed=10)
+    inp = synth.make_inputs(wl)
+    pq = oracle.pool(g, inp.q, inp.gamma_q, True)
+    pk = oracle.pool(g, inp.k, inp.gamma_k, False)
+    sc = oracle.select(g, pq, pk, want_scores=True).scores
+    sizes = oracle.window_sizes(g)
+    every = oracle.threshold_select(g, sc, np.full(g.rows, -np.inf))
+    none = oracle.threshold_select(g, sc, np.full(g.rows, np.inf))
+    for r in range(g.rows):
+        adm = np.flatnonzero(np.isfinite(sc[r]))
+        assert every.row_len[r] == sizes[r % g.nQB]
+        np.testing.assert_array_equal(every.row(r), adm)
+        assert none.row_len[r] == 1
+        assert none.row(r)[0] == adm[np.argmax(sc[r][adm])]
+    # equal best scores: the lower block
+    flat = np.where(np.isfinite(sc), 0.0, sc)
+    tie = oracle.threshold_select(g, flat, np.full(g.rows, 1.0))
+    for r in range(g.rows):
+        assert tie.row(r).tolist() == [np.flatnonzero(np.isfinite(sc[r]))[0]]

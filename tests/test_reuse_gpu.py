@@ -1,0 +1,144 @@
+"""Threshold reuse through the C ABI against the fp64 oracle.
+
+A plan with reuse on selects on its first call (recording each query block's
+k-th best score) and on later calls keeps every admissible block scoring at
+least that threshold. The kept sets must equal the oracle's
+(oracle.threshold_select with oracle.kth_thresholds of the first call's
+inputs) except for blocks whose score is within 1e-4 of the threshold, and the
+outputs must match the oracle run on the GPU's own kept sets.
+"""
+import numpy as np
+import pytest
+
+import block_sparse_video_lcsa_b200 as L
+import oracle
+from block_sparse_video_lcsa_b200 import synth
+
+from lcsa_harness import (OUT_MAX_ABS, OUT_MEAN_ABS, TIE_GAP, GpuResult, check_output, oracle_geometry, sample_rows,
+                          torch_inputs)
+
+pytestmark = pytest.mark.gpu
+
+_T = synth.WORKLOADS["tiny"]
+CASES = {
+    "stream_small": _T.replace(heads=3, q_frames=1, kv_frames=3, grid_h=24, grid_w=48, block_w=16, local_range=3,
+                               topk=5, kv_frame_offset=2, field=True, unit_gain=False),
+    "blocks64_odd_heads": _T.replace(heads=5, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                                     field=True, unit_gain=False, seed=1),
+    "stream_768x1280": synth.WORKLOADS["stream_768x1280"],
+}
+
+
+def _calls(wl, inputs):
+    """One plan with reuse on; one lcsa_forward per input set. Returns, per
+    call, (output bits, row_ptr, col_idx)."""
+    import torch
+    plan = L.lcsa_plan_create(L.config_from_workload(wl), 0)
+    res = []
+    try:
+        plan.lcsa_plan_set_threshold_reuse(True)
+        for inp in inputs:
+            q, k, v, gq, gk = torch_inputs(inp)
+            out = torch.empty_like(q)
+            plan.lcsa_forward(q, k, v, gq, gk, out)
+            plan.lcsa_check_device_error()
+            rp, ci = plan.lcsa_get_selection()
+            res.append((out.view(torch.int16).cpu().numpy().view(np.uint16), rp.copy(), ci.copy()))
+    finally:
+        plan.destroy()
+    return res
+
+
+def _scores(og, inp):
+    pq = oracle.pool(og, inp.q, inp.gamma_q, True)
+    pk = oracle.pool(og, inp.k, inp.gamma_k, False)
+    return oracle.select(og, pq, pk, want_scores=True)
+
+
+def _as_selection(rp, ci, nkb):
+    rows = rp.size - 1
+    lens = np.diff(rp).astype(np.int32)
+    cols = np.full((rows, max(1, int(lens.max()))), -1, dtype=np.int32)
+    for r in range(rows):
+        cols[r, : lens[r]] = ci[rp[r]:rp[r + 1]]
+    return oracle.Selection(lens, cols, np.full(rows, np.inf), None)
+
+
+def _check_kept(og, rp, ci, want, scores, th):
+    """GPU kept sets vs the oracle's, blocks within TIE_GAP of the threshold excused."""
+    bad = []
+    for r in range(og.rows):
+        got = ci[rp[r]:rp[r + 1]]
+        assert np.all(np.diff(got) > 0)
+        assert np.all(np.isfinite(scores[r][got])), "non-admissible block kept"
+        exp = want.row(r)
+        if np.array_equal(got, exp):
+            continue
+        diff = np.setxor1d(got, exp)
+        if want.row_len[r] == 1 and not np.any(scores[r][np.isfinite(scores[r])] >= th[r]):
+            # fallback row: the best block, up to near-ties of the best score
+            best = np.max(scores[r][np.isfinite(scores[r])])
+            if got.size == 1 and scores[r][got[0]] >= best - TIE_GAP:
+                continue
+        elif np.all(np.abs(scores[r][diff] - th[r]) < TIE_GAP):
+            continue
+        bad.append(r)
+    assert not bad, "kept sets differ beyond near-threshold blocks on rows %s" % bad[:5]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_reuse_keeps_the_blocks_over_the_recorded_threshold(name):
+    wl = CASES[name]
+    og = oracle_geometry(wl)
+    a = synth.make_inputs(wl)
+    b = synth.make_inputs(wl.replace(seed=wl.seed + 100))
+    (out_a, rp_a, ci_a), (out_b, rp_b, ci_b), (out_a2, rp_a2, ci_a2) = _calls(wl, [a, b, a])
+    sel_a, sel_b = _scores(og, a), _scores(og, b)
+    th = oracle.kth_thresholds(og, sel_a.scores)
+    want = oracle.threshold_select(og, sel_b.scores, th)
+    _check_kept(og, rp_b, ci_b, want, sel_b.scores, th)
+    # outputs of the reuse call against the oracle on the GPU's kept sets
+    rows = np.arange(og.rows) if og.rows <= 256 else sample_rows(og, 48)
+    ref, wsum = oracle.attention(og, b.q, b.k, b.v, b.gamma_q, b.gamma_k, _as_selection(rp_b, ci_b, og.nKB), rows)
+    np.testing.assert_allclose(wsum, 1.0, atol=1e-12)
+    gpu = GpuResult(out_b, rp_b, ci_b, None, None, None, None, None)
+    mx, mean = check_output(og, gpu, rows, ref)
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
+    # back on the recording inputs: the recorded selection again (rows with a
+    # clear k-th / (k+1)-th gap), and then the same output bits
+    clear = sel_a.gap > TIE_GAP
+    for r in np.flatnonzero(clear):
+        np.testing.assert_array_equal(ci_a2[rp_a2[r]:rp_a2[r + 1]], ci_a[rp_a[r]:rp_a[r + 1]])
+    if np.all(clear) and np.array_equal(rp_a2, rp_a):
+        np.testing.assert_array_equal(out_a2, out_a)
+
+
+def test_reuse_keeps_the_best_block_when_none_reaches_the_threshold():
+    """k = 0 on the reuse call: every score is exactly 0. Query blocks whose
+    recorded threshold is positive keep their first admissible block (the
+    lower index among equal best scores); those with a negative one keep the
+    whole window."""
+    wl = _T.replace(heads=2, q_frames=1, kv_frames=2, grid_h=32, grid_w=48, block_w=16, local_range=3, topk=2,
+                    field=True, unit_gain=False, seed=12)
+    og = oracle_geometry(wl)
+    a = synth.make_inputs(wl)
+    z = synth.make_inputs(wl)
+    z.k[...] = 0
+    (_, _, _), (out_z, rp, ci) = _calls(wl, [a, z])
+    th = oracle.kth_thresholds(og, _scores(og, a).scores)
+    sc = _scores(og, z).scores
+    above = below = 0
+    for r in range(og.rows):
+        adm = np.flatnonzero(np.isfinite(sc[r]))
+        got = ci[rp[r]:rp[r + 1]]
+        if th[r] >= TIE_GAP:
+            assert got.tolist() == [adm[0]], (r, got, adm[:3])
+            above += 1
+        elif th[r] <= -TIE_GAP:
+            np.testing.assert_array_equal(got, adm)
+            below += 1
+    assert above > 0
+    ref, _ = oracle.attention(og, z.q, z.k, z.v, z.gamma_q, z.gamma_k, _as_selection(rp, ci, og.nKB))
+    gpu = GpuResult(out_z, rp, ci, None, None, None, None, None)
+    mx, mean = check_output(og, gpu, np.arange(og.rows), ref)
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
