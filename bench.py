@@ -511,15 +511,21 @@ def run_layers(args):
     torch.cuda.synchronize(dev)
     plan.lcsa_check_device_error(side)
 
-    def timed(fn):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def timed_pair():
+        """Eager and graph steps alternate (so both see the same clocks under
+        the power cap); returns the mean ms of each."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
         torch.cuda.synchronize(dev)
-        e0.record(side)
-        for _ in range(args.steps):
-            fn()
-        e1.record(side)
+        for e in ev:
+            e[0].record(side)
+            chunk(side)
+            e[1].record(side)
+            e[2].record(side)
+            graph.replay()
+            e[3].record(side)
         torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / args.steps
+        return (sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps,
+                sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps)
 
     try:
         gpu_id = "GPU-%s" % torch.cuda.get_device_properties(dev).uuid
@@ -527,8 +533,7 @@ def run_layers(args):
         gpu_id = str(local)
     with ClockSampler(gpu_id) as clocks:
         with torch.cuda.stream(side):
-            eager_ms = timed(lambda: chunk(side))
-            graph_ms = timed(graph.replay)
+            eager_ms, graph_ms = timed_pair()
     plan.lcsa_check_device_error(side)
     del graph
     plan.destroy()
