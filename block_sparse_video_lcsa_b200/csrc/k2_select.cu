@@ -233,7 +233,55 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   if (p.reuse && threadIdx.x == kThreads - 1) p.row_len[rr] = pos;  // the last thread's end is the row's count
 }
 
+// Union of the selections of two query blocks, ascending: a byte per KV
+// block marks which of the two kept it (bit 0 the first, bit 1 the second),
+// then a block scan emits the marked blocks with their marks.
+__global__ void __launch_bounds__(kThreads) pair_union_kernel(const PairParams p) {
+  extern __shared__ unsigned char mark[];  // [nkb]
+  __shared__ int warp_sum[kWarps];
+  const int pr = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int c = threadIdx.x; c < p.nkb; c += kThreads) mark[c] = 0;
+  __syncthreads();
+  int rows2[2];
+  pair_rows(p.g, pr, rows2[0], rows2[1]);
+#pragma unroll 1
+  for (int side = 0; side < 2; ++side) {
+    const int row = rows2[side];
+    if (row >= 0) {
+      const int64_t beg = p.row_len ? int64_t(row) * p.pad_cap : int64_t(p.row_ptr[row]);
+      const int n = p.row_len ? p.row_len[row] : p.row_ptr[row + 1] - p.row_ptr[row];
+      for (int i = threadIdx.x; i < n; i += kThreads) mark[p.col_idx[beg + i]] |= (unsigned char)(1u << side);
+    }
+    __syncthreads();  // one side's blocks are distinct; the sides run one after the other
+  }
+  const int span = (p.nkb + kThreads - 1) / kThreads;
+  const int c_beg = min(int(threadIdx.x) * span, p.nkb), c_end = min(c_beg + span, p.nkb);
+  int cnt = 0;
+  for (int c = c_beg; c < c_end; ++c) cnt += mark[c] != 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int pos = incl - cnt;
+  for (int w = 0; w < warp; ++w) pos += warp_sum[w];
+  int* dst = p.pair_col + int64_t(pr) * p.pair_cap;
+  for (int c = c_beg; c < c_end; ++c)
+    if (mark[c]) dst[pos++] = c | (int(mark[c]) << kPairShift);
+  if (threadIdx.x == kThreads - 1) p.pair_len[pr] = pos;
+}
+
 }  // namespace
+
+cudaError_t launch_pair_union(const PairParams& p, cudaStream_t s) {
+  if (p.npairs <= 0) return cudaSuccess;
+  if (p.nkb > 48 * 1024) return cudaErrorInvalidValue;
+  pair_union_kernel<<<p.npairs, kThreads, size_t(p.nkb), s>>>(p);
+  return cudaGetLastError();
+}
 
 size_t select_smem_bytes(int sort_n) { return size_t(sort_n) * (sizeof(unsigned long long) + 1); }
 

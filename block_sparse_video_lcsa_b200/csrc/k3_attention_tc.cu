@@ -117,6 +117,9 @@ struct TcParams {
   const int* col_idx;
   const int* row_len;  // null, or the counts of a padded CSR (threshold reuse)
   int pad_cap;
+  const int* pair_col;  // paired 64-token query blocks: union lists (entries kb | marks << kPairShift)
+  const int* pair_len;
+  int pair_cap;
   __nv_bfloat16* out;
   float scale_log2;
   unsigned* err;
@@ -130,6 +133,17 @@ __device__ __forceinline__ int64_t row_begin(const TcParams& p, int rr) {
 __device__ __forceinline__ int row_count(const TcParams& p, int rr) {
   return p.row_len ? p.row_len[rr] : p.row_ptr[rr + 1] - p.row_ptr[rr];
 }
+
+// The KV list of work item rr: a row, or (PAIR) a pair of query blocks.
+template <bool PAIR>
+__device__ __forceinline__ int64_t list_begin(const TcParams& p, int rr) {
+  return PAIR ? int64_t(rr) * p.pair_cap : row_begin(p, rr);
+}
+template <bool PAIR>
+__device__ __forceinline__ int list_count(const TcParams& p, int rr) {
+  return PAIR ? p.pair_len[rr] : row_count(p, rr);
+}
+constexpr int kEntryMask = (1 << kPairShift) - 1;
 
 // ---- PTX wrappers ---------------------------------------------------------
 
@@ -357,7 +371,7 @@ __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
 // QM = tokens per query block (128, or 64: then each KV tile holds two
 // consecutive selected 64-token blocks and the M = 64 accumulators use TMEM
 // lanes 0-15 of each lane quarter).
-template <int QM>
+template <int QM, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
@@ -369,7 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = p.g;
-  constexpr int KB = kNB / QM;  // selected blocks per KV tile
+  // tokens per query / KV block, and KV blocks per tile: 128-token blocks;
+  // 64-token blocks as M = 64 tiles; or (PAIR) 64-token blocks with two query
+  // blocks in one M = 128 tile
+  constexpr int NBLK = PAIR ? 64 : QM;
+  constexpr int KB = kNB / NBLK;
 
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
@@ -421,15 +439,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, row_it = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int64_t beg = row_begin(p, rr);
-      const int n = row_count(p, rr);
-      const int bhh = rr / g.nQB;
+      const int64_t beg = list_begin<PAIR>(p, rr);
+      const int n = list_count<PAIR>(p, rr);
+      int ra = rr, rb = rr;  // the query block(s) of this work item
+      if constexpr (PAIR) {
+        pair_rows(g, rr, ra, rb);
+        if (rb < 0) rb = ra;  // a single block fills both halves; the second is not written out
+      }
+      const int bhh = ra / g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       if (row_it > 0 && !(ok = warp_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1))) break;
       if (lane == 0) {
         mbar_expect_tx(bar(bars->q_full), QM * kD * 2);
-        tma_load_2d(base + kOffQ, &tm_q, 0, rr * QM, bar(bars->q_full));
-        tma_load_2d(base + kOffQ + QM * 128, &tm_q, 64, rr * QM, bar(bars->q_full));
+        if constexpr (PAIR) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            tma_load_2d(base + kOffQ + hh * QM * 128, &tm_q, hh * 64, ra * NBLK, bar(bars->q_full));
+            tma_load_2d(base + kOffQ + hh * QM * 128 + NBLK * 128, &tm_q, hh * 64, rb * NBLK, bar(bars->q_full));
+          }
+        } else {
+          tma_load_2d(base + kOffQ, &tm_q, 0, rr * QM, bar(bars->q_full));
+          tma_load_2d(base + kOffQ + QM * 128, &tm_q, 64, rr * QM, bar(bars->q_full));
+        }
       }
       __syncwarp();
       const int steps = (n + KB - 1) / KB;
@@ -437,11 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.chunk = chunk;
         const int j = chunk * 32 + lane;
         if (j < n) {
-          const int kb = p.col_idx[beg + j];
+          const int kb = (PAIR ? p.pair_col : p.col_idx)[beg + j] & kEntryMask;
           const int fbw = kb / g.bpf, rem = kb - fbw * g.bpf;
           int slot = p.slot0_fb + fbw;  // ring slot of its frame-block (both terms below ring_fb)
           if (slot >= p.ring_fb) slot -= p.ring_fb;
-          e.krow = (bhh * g.nKB + slot * g.bpf + rem) * QM;
+          e.krow = (bhh * g.nKB + slot * g.bpf + rem) * NBLK;
           e.x0 = (rem % g.nWb) * g.bw;
           e.y0 = (rem / g.nWb) * g.bh;
           e.f0 = b * g.Tkv + slot * g.bt;
@@ -465,8 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int src = entry(ke, st, i);
           const int krow = __shfl_sync(0xffffffffu, ke.krow, src);
           if (lane == 0) {
-            tma_load_2d(kdst + i * QM * 128, &tm_k, 0, krow, bar(bars->k_full[ks]));
-            tma_load_2d(kdst + kHalfBytes + i * QM * 128, &tm_k, 64, krow, bar(bars->k_full[ks]));
+            tma_load_2d(kdst + i * NBLK * 128, &tm_k, 0, krow, bar(bars->k_full[ks]));
+            tma_load_2d(kdst + kHalfBytes + i * NBLK * 128, &tm_k, 64, krow, bar(bars->k_full[ks]));
           }
         }
         __syncwarp();
@@ -485,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int x0 = __shfl_sync(0xffffffffu, ve.x0, src), y0 = __shfl_sync(0xffffffffu, ve.y0, src);
           const int f0 = __shfl_sync(0xffffffffu, ve.f0, src);
           if (lane == 0) {
-            tma_load_5d(vdst + i * QM * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
-            tma_load_5d(vdst + kHalfBytes + i * QM * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
+            tma_load_5d(vdst + i * NBLK * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
+            tma_load_5d(vdst + kHalfBytes + i * NBLK * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
           }
         }
         __syncwarp();
@@ -499,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, s_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = (row_count(p, rr) + KB - 1) / KB;  // KV tiles of the row
+      const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
       if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
       for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
@@ -539,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
-      const int n = (row_count(p, rr) + KB - 1) / KB;  // KV tiles of the row
+      const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
       for (int j = 0; j < n; ++j, ++pv_it) {
         const int pb = pv_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
@@ -759,10 +790,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_it = 0, xk = 0;
     bool ok = true;
     for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
-      const int n_sel = row_count(p, rr);
-      const int n = n_sel;  // KV tiles of the row
+      const int n_sel = list_count<PAIR>(p, rr);
+      const int n = (n_sel + KB - 1) / KB;  // KV tiles of the work item
+      const int* lst = PAIR ? p.pair_col + list_begin<PAIR>(p, rr) : nullptr;
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j, ++s_it) {
+        // paired 64-token blocks: this warp's 64 keys are one KV block and its
+        // rows one query block; the block counts for these rows only if their
+        // query block selected it (and exists: an odd last tile repeats it)
+        bool masked = false;
+        if constexpr (PAIR) {
+          const int e = KB * j + half;
+          masked = e >= n_sel || !((__ldg(lst + e) >> kPairShift) & (sp < 2 ? 1 : 2));
+        }
         const int sb = s_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
@@ -780,7 +820,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
           mk[a] = fmaxf(mk[a], sv(a + 56));
         }
-        const float mpart = fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+        const float mpart =
+            masked ? -INFINITY : fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
         float* slot = xmax + (j & 1) * 256;
         slot[half * 128 + row_in_tile] = mpart;
         mbar_arrive(bar(bars->pair[sp]));
@@ -813,7 +854,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
           }
         }
-        {
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = 0u;
+        } else {
           const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
           l += rsum.x + rsum.y;
         }
@@ -836,6 +880,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(oa, o);
           }
         }
+        if constexpr (PAIR) {
+          // 64-token KV blocks: P is stored only once the P.V two blocks back
+          // has completed. Without this wait one lane quarter (32 rows, every
+          // channel) of an occasional tile differed from run to run on this
+          // part; with it, 10 of 10 full-size runs were identical (the same
+          // effect, and the same cure one block closer, as on the M = 64 path
+          // below; the 128-token path shows neither).
+          if (j >= 2) {
+            const int gp = s_it - 2;
+            if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 26))) break;
+            tc_fence_after();
+          }
+        }
         tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -855,10 +912,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
       ++xk;
       const float inv = 1.0f / (l + xsum[(half ^ 1) * 128 + row_in_tile]);
-      const int bhh = rr / g.nQB, qb = rr % g.nQB;
+      int qrow = rr, m_tok = row_in_tile;  // query block (row) and token of this lane's row
+      bool store = true;
+      if constexpr (PAIR) {
+        int ra, rb;
+        pair_rows(g, rr, ra, rb);
+        qrow = sp < 2 ? ra : rb;
+        m_tok = row_in_tile & (NBLK - 1);
+        store = qrow >= 0;  // a single block's second half is a copy
+        qrow = store ? qrow : ra;
+      }
+      const int bhh = qrow / g.nQB, qb = qrow % g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       const int tb = qb / g.bpf, rem = qb % g.bpf;
-      const int tt = row_in_tile / (g.bh * g.bw), yy = (row_in_tile / g.bw) % g.bh, xx = row_in_tile % g.bw;
+      const int tt = m_tok / (g.bh * g.bw), yy = (m_tok / g.bw) % g.bh, xx = m_tok % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
       __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + half * 64;
 #pragma unroll
@@ -872,8 +939,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
+        if (store) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d4[e] = v[e];
+          for (int e = 0; e < 4; ++e) d4[e] = v[e];
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -963,10 +1032,12 @@ cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s) {
   if (!attention_tc_supported(p.g)) return cudaErrorInvalidValue;
-  auto kern = p.g.nb == 128 ? attention_tc_kernel<128> : attention_tc_kernel<64>;
+  const bool paired = p.g.nb == 64 && p.pair_col != nullptr;
+  auto kern = p.g.nb == 128 ? attention_tc_kernel<128, false>
+                            : (paired ? attention_tc_kernel<128, true> : attention_tc_kernel<64, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
-  TcParams tp;
+  TcParams tp{};  // every field zero unless set below
   tp.g = p.g;
   tp.row_ptr = p.row_ptr;
   tp.row_len = p.row_len;
@@ -975,7 +1046,10 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.out = p.out;
   tp.scale_log2 = p.scale_log2;
   tp.err = p.err;
-  tp.rows = p.g.B * p.g.Hn * p.g.nQB;
+  tp.rows = paired ? p.npairs : p.g.B * p.g.Hn * p.g.nQB;
+  tp.pair_col = p.pair_col;
+  tp.pair_len = p.pair_len;
+  tp.pair_cap = p.pair_cap;
   tp.ring_fb = p.ring_fb;
   tp.slot0_fb = p.slot0_fb;
   const int grid = tp.rows < num_sms ? tp.rows : num_sms;

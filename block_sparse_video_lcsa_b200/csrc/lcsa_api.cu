@@ -180,6 +180,10 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   ws += size_t(g.B) * g.Hn * (g.nQB + g.nKB) * size_t(c->head_dim) * 4;         // pooled
   ws += (size_t(rows) + 1) * 4 + size_t(nnz) * 4;                                // CSR
   ws += size_t(rows) * (8 + size_t(wmax) * 4);                                    // threshold reuse
+  if (nb == 64) {                                                                 // query-block pairs
+    const size_t cap = size_t(2 * wmax < g.nKB ? 2 * wmax : g.nKB);
+    ws += size_t(lcsa::pair_count(g)) * (cap + 1) * 4;
+  }
   ws += rope_n * sizeof(float2) + 256;
   ws += size_t(lcsa::kMaxK1Ctas) * (2 * size_t(g.C) * 4 + 4);                    // K1 split blocks
   if (c->host_io)
@@ -189,6 +193,13 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// pair_cap: the union of two query blocks' lists, each at most the largest
+// window (a threshold-reuse call can keep a whole window)
+int pair_capacity(const Resolved& r) {
+  const int two = 2 * r.geo.max_window;
+  return two < r.grid.nKB ? two : r.grid.nKB;
+}
 
 }  // namespace
 
@@ -212,6 +223,10 @@ struct lcsa_plan {
   unsigned* thresh = nullptr;
   int32_t* row_len = nullptr;
   int32_t* col_pad = nullptr;
+  // 64-token blocks: pairs of query blocks as one 128-row tile (union lists)
+  int32_t* pair_col = nullptr;
+  int32_t* pair_len = nullptr;
+  int npairs = 0, pair_cap = 0;
   bool reuse_mode = false;   // lcsa_plan_set_threshold_reuse
   bool have_thresh = false;  // a selecting call has recorded thresholds
   bool last_reuse = false;   // the last call kept blocks by threshold
@@ -237,7 +252,8 @@ namespace {
 void release(lcsa_plan* p) {
   void* ptrs[] = {p->v_ring, p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
                   p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
-                  p->st_v,  p->st_out,  p->st_gq,    p->st_gk,    p->thresh,     p->row_len, p->col_pad};
+                  p->st_v,  p->st_out,  p->st_gq,    p->st_gk,    p->thresh,     p->row_len, p->col_pad,
+                  p->pair_col, p->pair_len};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (auto& set : p->evsets)
@@ -256,6 +272,16 @@ lcsa_status_t dev_alloc(T** ptr, size_t bytes, const char* what) {
                 bytes, cudaGetErrorString(e));
   }
   return LCSA_OK;
+}
+
+lcsa_status_t alloc_pairs(lcsa_plan* p) {
+  const int64_t np = lcsa::pair_count(p->res.grid);
+  if (np > (int64_t(1) << 30)) return fail(LCSA_ERR_UNSUPPORTED, "%lld query-block pairs", (long long)np);
+  p->npairs = int(np);
+  p->pair_cap = pair_capacity(p->res);
+  lcsa_status_t st = dev_alloc(&p->pair_col, size_t(np) * size_t(p->pair_cap) * 4, "pair lists");
+  if (st == LCSA_OK) st = dev_alloc(&p->pair_len, size_t(np) * 4, "pair counts");
+  return st;
 }
 
 }  // namespace
@@ -327,6 +353,7 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
       (st = dev_alloc(&p->thresh, rows * 4, "thresholds")) ||
       (st = dev_alloc(&p->row_len, rows * 4, "row counts")) ||
       (st = dev_alloc(&p->col_pad, rows * size_t(p->res.geo.max_window) * 4, "padded col_idx")) ||
+      (g.nb == 64 && (st = alloc_pairs(p)) != LCSA_OK) ||
       (st = dev_alloc(&p->rope, rope_n * sizeof(float2), "rope table")) ||
       (st = dev_alloc(&p->err, 256, "error word")) ||
       (st = dev_alloc(&p->split_part, size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4, "K1 split sums")) ||
@@ -401,7 +428,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
                        void* out, cudaStream_t s, const StepBlocks& sb) {
   const lcsa::Grid& g = p->res.grid;
   cudaError_t e;
-  lcsa::K1Params k1;
+  lcsa::K1Params k1{};  // every field zero (null) unless set below
   k1.g = g;
   k1.q = static_cast<const __nv_bfloat16*>(q);
   k1.k = static_cast<const __nv_bfloat16*>(k);
@@ -429,7 +456,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k1.ss_ext = sb.ss_ext;
   k1.norm_inv_c = 1.0f / float(int64_t(p->res.heads_total) * lcsa::kHeadDim);
 
-  lcsa::K2Params k2;
+  lcsa::K2Params k2{};  // every field zero (null) unless set below
   k2.g = g;
   k2.pooled_q = p->pooled_q;
   k2.pooled_k = p->pooled_k;
@@ -449,7 +476,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k2.row_len = p->row_len;
   k2.pad_cap = p->res.geo.max_window;
 
-  lcsa::K3Params k3;
+  lcsa::K3Params k3{};  // every field zero (null) unless set below
   k3.g = g;
   k3.qhat = p->qhat;
   k3.khat = p->khat;
@@ -459,6 +486,10 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k3.col_idx = reuse ? p->col_pad : p->col_idx;
   k3.row_len = reuse ? p->row_len : nullptr;
   k3.pad_cap = p->res.geo.max_window;
+  k3.npairs = p->npairs;
+  k3.pair_col = p->pair_col;
+  k3.pair_len = p->pair_len;
+  k3.pair_cap = p->pair_cap;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
   k3.err = p->err;
   k3.ring_fb = g.Tkv / g.bt;
@@ -476,6 +507,20 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   }
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  if (p->pair_col) {
+    lcsa::PairParams pp{};
+    pp.g = g;
+    pp.npairs = p->npairs;
+    pp.row_ptr = p->row_ptr;
+    pp.col_idx = reuse ? p->col_pad : p->col_idx;
+    pp.row_len = reuse ? p->row_len : nullptr;
+    pp.pad_cap = p->res.geo.max_window;
+    pp.nkb = g.nKB;
+    pp.pair_col = p->pair_col;
+    pp.pair_len = p->pair_len;
+    pp.pair_cap = p->pair_cap;
+    if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return cuda_fail(e, "pair union launch");
+  }
   p->have_thresh = true;
   p->last_reuse = reuse;
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");

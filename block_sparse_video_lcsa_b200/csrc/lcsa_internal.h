@@ -109,6 +109,53 @@ struct K2Params {
   int pad_cap;
 };
 
+// Pairs of neighbouring 64-token query blocks (same batch, head and frame
+// group) that K3 computes as one 128-row tile over the union of their
+// selected blocks, each entry kb | (which of the two selected it) <<
+// kPairShift. Within a frame group's nHb x nWb block grid, block rows 2i and
+// 2i+1 pair column by column; an odd last block row pairs columns 2j and
+// 2j+1; an odd last column of it stays single.
+constexpr int kPairShift = 28;
+__host__ __device__ inline int pairs_per_group(const Grid& g) {
+  return (g.nHb / 2) * g.nWb + (g.nHb % 2) * ((g.nWb + 1) / 2);
+}
+__host__ __device__ inline int64_t pair_count(const Grid& g) {
+  return int64_t(g.B) * g.Hn * (g.nQB / g.bpf) * pairs_per_group(g);
+}
+// rows (batch, head, query block) of pair pr; the second is -1 for a single block
+__host__ __device__ inline void pair_rows(const Grid& g, int64_t pr, int& ra, int& rb) {
+  const int pg = pairs_per_group(g);
+  const int64_t per_bh = int64_t(g.nQB / g.bpf) * pg;
+  const int bh = int(pr / per_bh);
+  const int rem = int(pr % per_bh), tb = rem / pg, k = rem % pg;
+  int ha, wa, hb, wb;
+  if (k < (g.nHb / 2) * g.nWb) {
+    ha = 2 * (k / g.nWb);
+    hb = ha + 1;
+    wa = wb = k % g.nWb;
+  } else {
+    const int k2 = k - (g.nHb / 2) * g.nWb;
+    ha = hb = g.nHb - 1;
+    wa = 2 * k2;
+    wb = wa + 1;
+  }
+  const int base = bh * g.nQB + tb * g.bpf;
+  ra = base + ha * g.nWb + wa;
+  rb = wb < g.nWb ? base + hb * g.nWb + wb : -1;
+}
+struct PairParams {
+  Grid g;
+  int npairs;
+  const int* row_ptr;     // the rows' selections (as K3 reads them: CSR, or padded + counts)
+  const int* col_idx;
+  const int* row_len;
+  int pad_cap;
+  int nkb;                // KV blocks per (batch, head): the range of block indices
+  int* pair_col;          // [npairs][pair_cap]
+  int* pair_len;          // [npairs]
+  int pair_cap;
+};
+
 struct K3Params {
   Grid g;
   const __nv_bfloat16* qhat;
@@ -124,6 +171,11 @@ struct K3Params {
   // are col_idx[r * pad_cap ...], row_len[r] of them (threshold reuse)
   const int* row_len;
   int pad_cap;
+  // 64-token blocks: the query-block pairs' union lists (PairParams)
+  int npairs;
+  const int* pair_col;
+  const int* pair_len;
+  int pair_cap;
 };
 
 // The stateless call's block sets: every query and key block, ring = window.
@@ -143,6 +195,7 @@ cudaError_t launch_sumsq(const __nv_bfloat16* q, int64_t nq, const __nv_bfloat16
                          float* ss, cudaStream_t s);
 size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
+cudaError_t launch_pair_union(const PairParams& p, cudaStream_t s);
 
 // tcgen05 attention (128- or 64-token blocks). Tensor maps: q^ / k^ as
 // [rows][128] bf16 with boxes of 64 columns x one block of rows

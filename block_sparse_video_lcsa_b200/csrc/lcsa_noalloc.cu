@@ -207,7 +207,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   noalloc_row_ptr_kernel<<<1, 32, 0, s>>>(row_ptr, g, radius, ng.topk);
   if ((e = cudaGetLastError()) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "row offsets launch");
 
-  lcsa::K1Params k1;
+  lcsa::K1Params k1{};  // every field zero (null) unless set below
   k1.g = g;
   k1.q = static_cast<const __nv_bfloat16*>(q);
   k1.k = static_cast<const __nv_bfloat16*>(k);
@@ -234,7 +234,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
 
   int sort_n = 32;
   while (sort_n < ng.max_window) sort_n <<= 1;
-  lcsa::K2Params k2;
+  lcsa::K2Params k2{};  // every field zero (null) unless set below
   k2.g = g;
   k2.pooled_q = pooled_q;
   k2.pooled_k = pooled_k;
@@ -255,7 +255,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
 
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));
-  lcsa::K3Params k3;
+  lcsa::K3Params k3{};  // every field zero (null) unless set below
   k3.g = g;
   k3.qhat = qhat;
   k3.khat = khat;
@@ -269,6 +269,9 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.slot0_fb = 0;
   k3.row_len = nullptr;
   k3.pad_cap = 0;
+  k3.pair_col = nullptr;  // no query-block pairs without a plan: 64-token blocks run as M = 64 tiles
+  k3.pair_len = nullptr;
+  k3.npairs = 0;
   {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
