@@ -1,12 +1,13 @@
 // K3 (tcgen05 form): block-sparse flash attention over the CSR list with the
 // 5th-generation tensor cores, tensor memory and TMA, for 128- and 64-token
-// blocks. A KV tile is always 128 keys: one 128-token block, or two
-// consecutive selected 64-token blocks (an odd last tile repeats its block and
-// the softmax zeroes the copy). With 64-token blocks the query tile is 64 rows
-// and the products are M = 64 (measured on this part: M64 N128 K16 issues every
-// 64 cycles, half the rate of M128 N128 K16; M64 N64 K16 every 51), whose
-// accumulators hold row m in TMEM lane 32 (m / 16) + m % 16, so only lanes
-// 0-15 of each softmax warp carry rows.
+// blocks. Every product is M = 128 rows x N = 128: a KV tile is 128 keys
+// (one 128-token block, or two consecutive entries of a 64-token list, an odd
+// last tile repeating its entry for the softmax to mask), and a query tile is
+// 128 rows (one 128-token block, or two neighbouring 64-token query blocks
+// over the union of their selections, each KV block masked for the rows whose
+// query block did not select it). M = 64 products, measured on this part,
+// issue at the M = 128 rate for half the work (M64 N128 K16 every 64 cycles)
+// and leave half of each softmax warp's TMEM lanes empty.
 //
 // Pages: "FlashVSR: From 17.2 FPS to 57.3 FPS at 768x1408", Rebuild sparse
 // attention for Hopper: a warp-specialised producer/consumer path with TMA
@@ -280,37 +281,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       LCSA_W32(r)
       : "memory");
 }
-#define LCSA_W16(a)                                                                                               \
-  "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]), \
-      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15])
-
-// 16-lane shapes, for M = 64 accumulators (lanes 0-15 of the warp's lane
-// quarter). .16x256b.x8: for rep r, registers 4r and 4r+1 hold columns
-// 8r + 2(t%4) and 8r + 2(t%4) + 1 of lane t/4, registers 4r+2 and 4r+3 the
-// same columns of lane t/4 + 8 (t = thread of the warp).
-__device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : LCSA_R32(r)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      LCSA_W32(r)
-      : "memory");
-}
-// .16x128b.x8: for rep r, register 2r holds column 4r + t%4 of lane t/4 and
-// register 2r+1 the same column of lane t/4 + 8.
-__device__ __forceinline__ void tmem_st16x128_x8(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      LCSA_W16(r)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -368,10 +338,9 @@ __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
 
 // ---- the kernel -----------------------------------------------------------
 
-// QM = tokens per query block (128, or 64: then each KV tile holds two
-// consecutive selected 64-token blocks and the M = 64 accumulators use TMEM
-// lanes 0-15 of each lane quarter).
-template <int QM, bool PAIR>
+// PAIR: 64-token blocks, a work item is a pair of query blocks over the union
+// of their selections; otherwise 128-token blocks, a work item is one row.
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
@@ -383,9 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = p.g;
-  // tokens per query / KV block, and KV blocks per tile: 128-token blocks;
-  // 64-token blocks as M = 64 tiles; or (PAIR) 64-token blocks with two query
-  // blocks in one M = 128 tile
+  // rows per query tile (M of the products); tokens per query / KV block and
+  // KV blocks per tile: 128-token blocks, or (PAIR) 64-token blocks with two
+  // query blocks in one tile and two KV blocks per KV tile
+  constexpr int QM = 128;
   constexpr int NBLK = PAIR ? 64 : QM;
   constexpr int KB = kNB / NBLK;
 
@@ -601,183 +571,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       mbar_drain(bar(bars->mma_drain[1]), 0);
     }
-  } else if constexpr (QM == 64) {
-    // ---------------- softmax / correction / epilogue, 64-token tiles ----------------
-    // Query row m of an M = 64 accumulator sits in TMEM lane 32 * (m / 16) +
-    // m % 16, so a lane quarter holds 16 rows. The 16-lane load shapes spread
-    // them over the whole warp: thread t carries rows mA = 16 sp + t / 4 and
-    // mB = mA + 8, 16 of the half's 64 key columns each; the four threads of
-    // a row combine their maxima and sums by shuffles.
-    const int sp = warp & 3;
-    const int half = (warp - 3) >> 2;
-    const int cq = lane & 3;
-    const int mA = sp * 16 + (lane >> 2), mB = mA + 8;
-    const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
-    float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
-    float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
-    const float c = p.scale_log2;
-    int s_it = 0, xk = 0;
-    bool ok = true;
-    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
-      const int n_sel = row_count(p, rr);
-      const int n = (n_sel + 1) / 2;  // KV tiles of the row, two blocks each
-      float mu[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-      for (int j = 0; j < n && ok; ++j, ++s_it) {
-        // an odd last tile repeats its block in keys 64-127
-        const bool masked = half == 1 && 2 * j + 1 >= n_sel;
-        const int sb = s_it % kSBufs;
-        if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
-        tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld16x256_x8(lane_addr + kColS + sb * 128 + half * 64, sr);
-        tmem_wait_ld();
-        auto sv = [&](int e) { return __uint_as_float(sr[e]); };
-        float mx[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          float t[16];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            t[2 * r] = sv(4 * r + 2 * h2);
-            t[2 * r + 1] = sv(4 * r + 2 * h2 + 1);
-          }
-          const float a0 = fmax3(t[0], t[1], t[2]), a1 = fmax3(t[3], t[4], t[5]), a2 = fmax3(t[6], t[7], t[8]);
-          const float a3 = fmax3(t[9], t[10], t[11]), a4 = fmax3(t[12], t[13], t[14]);
-          float m = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, t[15]));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-          mx[h2] = masked ? -INFINITY : m;
-        }
-        float* slot = xmax + (j & 1) * 256;
-        if (cq == 0) {
-          slot[half * 128 + mA] = mx[0];
-          slot[half * 128 + mB] = mx[1];
-        }
-        mbar_arrive(bar(bars->pair[sp]));
-        if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 23))) break;
-        ++xk;
-        mx[0] = fmaxf(mx[0], slot[(half ^ 1) * 128 + mA]);
-        mx[1] = fmaxf(mx[1], slot[(half ^ 1) * 128 + mB]);
-        float alpha[2];
-        bool need_any = false;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const float m_new = fmaxf(mu[h2], mx[h2] * c);
-          const bool need = m_new > mu[h2] + kRescaleLog2;
-          alpha[h2] = 1.f;
-          if (need) {
-            alpha[h2] = exp2_mufu(mu[h2] - m_new);
-            mu[h2] = m_new;
-          }
-          l[h2] *= alpha[h2];
-          need_any |= need;
-        }
-        const bool warp_need = __any_sync(0xffffffffu, need_any);
-        uint32_t pk[16];
-        float2 rs[2][2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) rs[h2][0] = rs[h2][1] = make_float2(0.f, 0.f);
-        const float2 c2 = make_float2(c, c);
-        const float2 mneg[2] = {make_float2(-mu[0], -mu[0]), make_float2(-mu[1], -mu[1])};
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 4 * r + 2 * h2;
-            const float2 x = __ffma2_rn(make_float2(sv(e), sv(e + 1)), c2, mneg[h2]);
-            const float2 pp = ((2 * r + h2) % kPolyEvery == kPolyEvery - 1) ? exp2_poly2(x)
-                                                                           : make_float2(exp2_mufu(x.x), exp2_mufu(x.y));
-            rs[h2][r & 1] = __fadd2_rn(rs[h2][r & 1], pp);
-            pk[2 * r + h2] = pack_bf16(pp.x, pp.y);
-          }
-        }
-        if (masked) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = 0u;
-        } else {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const float2 s2 = __fadd2_rn(rs[h2][0], rs[h2][1]);
-            l[h2] += s2.x + s2.y;
-          }
-        }
-        // O is rescaled once every earlier P.V has completed (the last of them
-        // is P.V number gp = s_it - 1; P.V gp + 2 needs a P this warp has not
-        // written yet, so the parity wait on o_done[gp & 1] cannot be
-        // overtaken). P is stored only after that P.V has completed too: with
-        // M = 64 P stores overlapping an in-flight P.V, outputs varied from run
-        // to run on this part, although isolated M = 64 products read and
-        // write lanes 0-15 of each quarter only.
-        if (j >= 1) {
-          const int gp = s_it - 1;
-          if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 21))) break;
-          tc_fence_after();
-          if (warp_need) {
-            uint32_t o[32];
-            const uint32_t oa = lane_addr + kColO + half * 64;
-            tmem_ld16x256_x8(oa, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-              o[4 * r] = __float_as_uint(__uint_as_float(o[4 * r]) * alpha[0]);
-              o[4 * r + 1] = __float_as_uint(__uint_as_float(o[4 * r + 1]) * alpha[0]);
-              o[4 * r + 2] = __float_as_uint(__uint_as_float(o[4 * r + 2]) * alpha[1]);
-              o[4 * r + 3] = __float_as_uint(__uint_as_float(o[4 * r + 3]) * alpha[1]);
-            }
-            tmem_st16x256_x8(oa, o);
-          }
-        }
-        // P columns: key pair (2i, 2i+1) of this half in column half * 64 + i
-        tmem_st16x128_x8(lane_addr + kColS + sb * 128 + half * 64, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bars->p_full[sb]));
-      }
-      if (!ok) break;
-      {
-        const int gp = s_it - 1;  // the row's last P.V (completion implies all earlier ones)
-        if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 22))) break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 1);
-        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 2);
-      }
-      if (cq == 0) {
-        xsum[half * 128 + mA] = l[0];
-        xsum[half * 128 + mB] = l[1];
-      }
-      mbar_arrive(bar(bars->pair[sp]));
-      if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
-      ++xk;
-      const float invA = 1.0f / (l[0] + xsum[(half ^ 1) * 128 + mA]);
-      const float invB = 1.0f / (l[1] + xsum[(half ^ 1) * 128 + mB]);
-      const int bhh = rr / g.nQB, qb = rr % g.nQB;
-      const int b = bhh / g.Hn, h = bhh % g.Hn;
-      const int tb = qb / g.bpf, rem = qb % g.bpf;
-      auto token = [&](int m) {
-        const int tt = m / (g.bh * g.bw), yy = (m / g.bw) % g.bh, xx = m % g.bw;
-        return (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
-      };
-      const int ch = h * kD + half * 64 + 2 * cq;
-      __nv_bfloat16* dA = p.out + (int64_t(b) * g.Lq + token(mA)) * g.C + ch;
-      __nv_bfloat16* dB = p.out + (int64_t(b) * g.Lq + token(mB)) * g.C + ch;
-      uint32_t o[32];
-      tmem_ld16x256_x8(lane_addr + kColO + half * 64, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        *reinterpret_cast<uint32_t*>(dA + 8 * r) =
-            pack_bf16(__uint_as_float(o[4 * r]) * invA, __uint_as_float(o[4 * r + 1]) * invA);
-        *reinterpret_cast<uint32_t*>(dB + 8 * r) =
-            pack_bf16(__uint_as_float(o[4 * r + 2]) * invB, __uint_as_float(o[4 * r + 3]) * invB);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(bars->o_free));
-    }
   } else {
     // ---------------- softmax / correction / epilogue, 128-token tiles ----------------
     const int sp = warp & 3;                 // TMEM lane quarter of this warp
@@ -884,9 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 64-token KV blocks: P is stored only once the P.V two blocks back
           // has completed. Without this wait one lane quarter (32 rows, every
           // channel) of an occasional tile differed from run to run on this
-          // part; with it, 10 of 10 full-size runs were identical (the same
-          // effect, and the same cure one block closer, as on the M = 64 path
-          // below; the 128-token path shows neither).
+          // part; with it, 10 of 10 full-size runs were identical (an earlier
+          // M = 64 form of this path needed the same wait for the P.V just
+          // before; the 128-token path needs neither).
           if (j >= 2) {
             const int gp = s_it - 2;
             if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 26))) break;
@@ -1033,8 +826,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s) {
   if (!attention_tc_supported(p.g)) return cudaErrorInvalidValue;
   const bool paired = p.g.nb == 64 && p.pair_col != nullptr;
-  auto kern = p.g.nb == 128 ? attention_tc_kernel<128, false>
-                            : (paired ? attention_tc_kernel<128, true> : attention_tc_kernel<64, false>);
+  if (p.g.nb == 64 && !paired) return cudaErrorInvalidValue;  // 64-token blocks run as query-block pairs
+  auto kern = paired ? attention_tc_kernel<true> : attention_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
   TcParams tp{};  // every field zero unless set below

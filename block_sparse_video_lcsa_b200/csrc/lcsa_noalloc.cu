@@ -167,7 +167,12 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   const size_t off_pk = off_pq + round256(size_t(g.B) * g.Hn * g.nQB * D * 4);
   const size_t off_qh = off_pk + round256(size_t(g.B) * g.Hn * g.nKB * D * 4);
   const size_t off_kh = off_qh + round256(size_t(g.B) * g.Lq * g.C * 2);
-  const size_t need = off_kh + round256(size_t(g.B) * g.Lkv * g.C * 2);
+  // 64-token blocks: query-block pairs as 128-row tiles (union lists and counts)
+  const int64_t npairs = g.nb == 64 ? lcsa::pair_count(g) : 0;
+  const int pair_cap = 2 * ng.max_window < g.nKB ? 2 * ng.max_window : g.nKB;
+  const size_t off_pc = off_kh + round256(size_t(g.B) * g.Lkv * g.C * 2);
+  const size_t off_pl = off_pc + round256(size_t(npairs) * size_t(pair_cap) * 4);
+  const size_t need = off_pl + round256(size_t(npairs) * 4);
   if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES))
     return noalloc_fail(LCSA_ERR_UNSUPPORTED,
                         "problem needs more workspace than the static array holds (LCSA_NOALLOC_WORKSPACE_BYTES); "
@@ -199,6 +204,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   float* pooled_k = reinterpret_cast<float*>(ws + off_pk);
   __nv_bfloat16* qhat = reinterpret_cast<__nv_bfloat16*>(ws + off_qh);
   __nv_bfloat16* khat = reinterpret_cast<__nv_bfloat16*>(ws + off_kh);
+  int* pair_col = npairs ? reinterpret_cast<int*>(ws + off_pc) : nullptr;
+  int* pair_len = npairs ? reinterpret_cast<int*>(ws + off_pl) : nullptr;
 
   if ((e = cudaMemsetAsync(err, 0, off_sp - off_err, s)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "clear error word and counters");
@@ -253,6 +260,18 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.row_len = nullptr;
   k2.pad_cap = 0;
   if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
+  if (npairs) {
+    lcsa::PairParams pp{};
+    pp.g = g;
+    pp.npairs = int(npairs);
+    pp.row_ptr = row_ptr;
+    pp.col_idx = col_idx;
+    pp.nkb = g.nKB;
+    pp.pair_col = pair_col;
+    pp.pair_len = pair_len;
+    pp.pair_cap = pair_cap;
+    if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "pair union launch");
+  }
 
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));
   lcsa::K3Params k3{};  // every field zero (null) unless set below
@@ -269,9 +288,10 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.slot0_fb = 0;
   k3.row_len = nullptr;
   k3.pad_cap = 0;
-  k3.pair_col = nullptr;  // no query-block pairs without a plan: 64-token blocks run as M = 64 tiles
-  k3.pair_len = nullptr;
-  k3.npairs = 0;
+  k3.pair_col = pair_col;
+  k3.pair_len = pair_len;
+  k3.npairs = int(npairs);
+  k3.pair_cap = pair_cap;
   {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
