@@ -25,7 +25,7 @@ STREAMS = {
     # 128-token blocks, windowed selection
     "stream128": _T.replace(heads=3, q_frames=2, kv_frames=6, grid_h=24, grid_w=48, block_w=16, local_range=3,
                             topk=5, field=True, unit_gain=False, seed=8),
-    # 64-token blocks (M = 64 attention tiles), an odd top-k (a half KV tile per row)
+    # 64-token blocks (paired 128-row query tiles), an odd top-k (a half KV tile per row)
     "stream64": _T.replace(heads=2, q_frames=2, kv_frames=6, grid_h=32, grid_w=40, local_range=5, topk=7,
                            field=True, unit_gain=False, seed=9),
 }
