@@ -673,19 +673,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(oa, o);
           }
         }
-        if constexpr (PAIR) {
-          // 64-token KV blocks: P is stored only once the P.V two blocks back
-          // has completed. Without this wait one lane quarter (32 rows, every
-          // channel) of an occasional tile differed from run to run on this
-          // part; with it, 10 of 10 full-size runs were identical (an earlier
-          // M = 64 form of this path needed the same wait for the P.V just
-          // before; the 128-token path needs neither).
-          if (j >= 2) {
-            const int gp = s_it - 2;
-            if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 26))) break;
-            tc_fence_after();
-          }
-        }
         tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -696,7 +683,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue: wait for the last P.V, combine the two halves' row sums,
       // normalise and store this thread's 64 output channels
       {
-        const int gp = s_it - 1;  // the row's last P.V (completion implies all earlier ones)
+        // The row's last P.V is number gp = s_it - 1 (its completion implies
+        // all earlier ones). A parity wait is only unambiguous while its
+        // barrier is at most one phase short of the target: o_done[gp & 1]
+        // last completed for P.V gp - 2, which nothing has waited for, and if
+        // that one were still running the parity test would pass at once. So
+        // P.V gp - 1 is waited for first: its barrier's previous phase, P.V
+        // gp - 3, completed before S of block gp was issued, and its
+        // completion implies gp - 2's.
+        const int gp = s_it - 1;
+        if (gp >= 1 && !(ok = warp_wait(bar(bars->o_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, abort, p.err, 25)))
+          break;
         if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 22))) break;
       }
       tc_fence_after();
