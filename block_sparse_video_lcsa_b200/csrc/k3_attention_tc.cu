@@ -557,9 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tmem + kColO, pa + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), sdesc(va + kk * 2048, kHalfBytes, 1024),
                    id_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(bars->v_empty[vs]));
-          mma_commit(bar(bars->s_free[pb]));
+          // o_done first: the softmax's parity waits on o_done rely on a
+          // product's o_done arrival having happened once its s_free arrival
+          // (which lets S of a later block start) has been seen
           mma_commit(bar(bars->o_done[pv_it & 1]));
+          mma_commit(bar(bars->s_free[pb]));
+          mma_commit(bar(bars->v_empty[vs]));
         }
         __syncwarp();
         issued = true;
