@@ -86,7 +86,9 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
-constexpr uint32_t kOffXchg = kOffBar + 256;          // row max / sum exchange
+constexpr uint32_t kOffXchg = kOffBar + 512;          // row max / sum exchange
+constexpr int kItemSlots = 4;  // work items handed from the producer to the other roles
+constexpr int kItemReaders = 2 + kSoftmaxWarps;  // S issuer, P.V issuer, softmax warps (one arrival each)
 constexpr uint32_t kXchgBytes = (2 * 2 * 128 + 2 * 128) * 4;
 constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
 
@@ -105,10 +107,14 @@ struct Bars {
   uint64_t o_done[2];  // o_done[g & 1]: P.V number g (counted per CTA) and all before it have completed
   uint64_t o_free, mma_drain[2];
   uint64_t pair[4];  // row max / sum exchange between the two softmax warps of a lane quarter
+  // dynamic work distribution: the producer takes the next work item from
+  // the global counter and hands it to the other roles through item[]
+  uint64_t item_full[kItemSlots], item_empty[kItemSlots];
+  int item[kItemSlots];
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
 static_assert(kSoftmaxWarps == 8 && kThreads == 96 + 32 * kSoftmaxWarps, "warp roles");
 
 struct TcParams {
@@ -125,6 +131,7 @@ struct TcParams {
   float scale_log2;
   unsigned* err;
   int rows;
+  unsigned* work_counter;  // zero at launch; each CTA takes work items from it
 };
 
 // Selected blocks of row rr: col_idx[row_begin .. row_begin + row_count).
@@ -360,6 +367,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int KB = kNB / NBLK;
 
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+  // Work item number `it` of this CTA, as every role sees it: the producer
+  // takes it from the global counter and publishes it in item[it % slots];
+  // the other roles read it there (one arrival per reader frees the slot).
+  // An item >= p.rows ends the CTA's work.
+  auto take_item = [&](int it, bool& ok) -> int {
+    const int slot = it % kItemSlots;
+    if (it >= kItemSlots &&
+        !(ok = warp_wait(bar(bars->item_empty[slot]), ((it / kItemSlots) - 1) & 1, abort, p.err, 4)))
+      return p.rows;
+    int rr = 0;
+    if (lane == 0) {
+      rr = int(atomicAdd(p.work_counter, 1u));
+      bars->item[slot] = rr;
+      mbar_arrive(bar(bars->item_full[slot]));
+    }
+    return __shfl_sync(0xffffffffu, rr, 0);
+  };
+  auto read_item = [&](int it, bool& ok) -> int {
+    const int slot = it % kItemSlots;
+    if (!(ok = warp_wait(bar(bars->item_full[slot]), (it / kItemSlots) & 1, abort, p.err, 5))) return p.rows;
+    const int rr = static_cast<volatile int*>(bars->item)[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(bars->item_empty[slot]));
+    return rr;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->q_full), 1);
@@ -383,6 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(bars->mma_drain[0]), 1);
     mbar_init(bar(bars->mma_drain[1]), 1);
     for (int s = 0; s < 4; ++s) mbar_init(bar(bars->pair[s]), 64);
+    for (int s = 0; s < kItemSlots; ++s) {
+      mbar_init(bar(bars->item_full[s]), 1);
+      mbar_init(bar(bars->item_empty[s]), kItemReaders);
+    }
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -408,7 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int kv = 0, row_it = 0;
     bool ok = true;
-    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+    for (int it = 0; ok; ++it, ++row_it) {
+      const int rr = take_item(it, ok);
+      if (!ok || rr >= p.rows) break;
       const int64_t beg = list_begin<PAIR>(p, rr);
       const int n = list_count<PAIR>(p, rr);
       int ra = rr, rb = rr;  // the query block(s) of this work item
@@ -499,7 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t id_qk = idesc_bf16(0, QM);
     int kv = 0, s_it = 0, row_it = 0;
     bool ok = true, issued = false;
-    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+    for (int it = 0; ok; ++it, ++row_it) {
+      const int rr = read_item(it, ok);
+      if (!ok || rr >= p.rows) break;
       const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
       if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
       for (int j = 0; j < n; ++j, ++s_it) {
@@ -539,7 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t id_pv = idesc_bf16(1, QM);
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
-    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x, ++row_it) {
+    for (int it = 0; ok; ++it, ++row_it) {
+      const int rr = read_item(it, ok);
+      if (!ok || rr >= p.rows) break;
       const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
       for (int j = 0; j < n; ++j, ++pv_it) {
         const int pb = pv_it % kSBufs;
@@ -585,7 +627,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     int s_it = 0, xk = 0;
     bool ok = true;
-    for (int rr = blockIdx.x; rr < p.rows && ok; rr += gridDim.x) {
+    for (int it = 0; ok; ++it) {
+      const int rr = read_item(it, ok);
+      if (!ok || rr >= p.rows) break;
       const int n_sel = list_count<PAIR>(p, rr);
       const int n = (n_sel + KB - 1) / KB;  // KV tiles of the work item
       const int* lst = PAIR ? p.pair_col + list_begin<PAIR>(p, rr) : nullptr;
@@ -840,6 +884,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.scale_log2 = p.scale_log2;
   tp.err = p.err;
   tp.rows = paired ? p.npairs : p.g.B * p.g.Hn * p.g.nQB;
+  tp.work_counter = p.work_counter;
+  if (!tp.work_counter) return cudaErrorInvalidValue;
   tp.pair_col = p.pair_col;
   tp.pair_len = p.pair_len;
   tp.pair_cap = p.pair_cap;

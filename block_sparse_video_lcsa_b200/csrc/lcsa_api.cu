@@ -185,7 +185,7 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
     ws += size_t(lcsa::pair_count(g)) * (cap + 1) * 4;
   }
   ws += rope_n * sizeof(float2) + 256;
-  ws += size_t(lcsa::kMaxK1Ctas) * (2 * size_t(g.C) * 4 + 4);                    // K1 split blocks
+  ws += size_t(lcsa::kMaxK1Ctas) * 2 * size_t(g.C) * 4 + size_t(lcsa::kCounters) * 4;  // K1 split blocks, counters
   if (c->host_io)
     ws += size_t(g.B) * (2 * g.Lq + 2 * g.Lkv) * g.C * 2 + size_t(2) * g.C * 4;
   o.workspace_bytes = ws;
@@ -357,7 +357,7 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
       (st = dev_alloc(&p->rope, rope_n * sizeof(float2), "rope table")) ||
       (st = dev_alloc(&p->err, 256, "error word")) ||
       (st = dev_alloc(&p->split_part, size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4, "K1 split sums")) ||
-      (st = dev_alloc(&p->split_cnt, size_t(lcsa::kMaxK1Ctas) * 4, "K1 split counters"))) {
+      (st = dev_alloc(&p->split_cnt, size_t(lcsa::kCounters) * 4, "K1 split and K3 work counters"))) {
     release(p);
     delete p;
     return st;
@@ -376,7 +376,7 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
   }
   if ((e = cudaMemcpy(p->row_ptr, p->res.row_ptr.data(), (rows + 1) * 4, cudaMemcpyHostToDevice)) != cudaSuccess ||
       (e = cudaMemset(p->err, 0, 256)) != cudaSuccess ||
-      (e = cudaMemset(p->split_cnt, 0, size_t(lcsa::kMaxK1Ctas) * 4)) != cudaSuccess ||
+      (e = cudaMemset(p->split_cnt, 0, size_t(lcsa::kCounters) * 4)) != cudaSuccess ||
       (e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, cfg->head_dim, 0)) !=
           cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
@@ -466,7 +466,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k2.topk = p->res.geo.topk;
   k2.sort_n = p->res.sort_n;
   k2.clear_cnt = p->split_cnt;
-  k2.n_clear = lcsa::kMaxK1Ctas;
+  k2.n_clear = lcsa::kCounters;
   k2.ring_fb = g.Tkv / g.bt;
   k2.slot0_fb = sb.slot0_fb;
   const bool reuse = p->reuse_mode && p->have_thresh;
@@ -490,6 +490,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k3.pair_col = p->pair_col;
   k3.pair_len = p->pair_len;
   k3.pair_cap = p->pair_cap;
+  k3.work_counter = p->split_cnt + lcsa::kMaxK1Ctas;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
   k3.err = p->err;
   k3.ring_fb = g.Tkv / g.bt;
@@ -501,7 +502,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
   if (!sb.with_q) {
     // no K2 after this K1: clear its merge counters here
-    if ((e = cudaMemsetAsync(p->split_cnt, 0, size_t(lcsa::kMaxK1Ctas) * 4, s)) != cudaSuccess)
+    if ((e = cudaMemsetAsync(p->split_cnt, 0, size_t(lcsa::kCounters) * 4, s)) != cudaSuccess)
       return cuda_fail(e, "clear merge counters");
     return LCSA_OK;
   }

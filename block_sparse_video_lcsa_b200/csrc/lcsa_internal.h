@@ -13,6 +13,9 @@ constexpr int kHeadDim = 128;        // the only head size the kernels implement
 constexpr int kMaxHeads = 16;
 constexpr int kMaxCandidates = 4096; // admissible blocks per query block (K2 sort)
 constexpr int kMaxK1Ctas = 256;      // K1 persistent grid cap (sizes its split-block buffers)
+// The plan's counter array: K1's kMaxK1Ctas merge counters, then K3's work
+// counter; K2 zeroes all of them (after K1 has used its own, before K3 starts).
+constexpr int kCounters = kMaxK1Ctas + 1;
 
 // Device error word codes (first word of the plan's error buffer).
 constexpr unsigned kDevErrNone = 0;
@@ -176,6 +179,7 @@ struct K3Params {
   const int* pair_col;
   const int* pair_len;
   int pair_cap;
+  unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work items from it
 };
 
 // The stateless call's block sets: every query and key block, ring = window.

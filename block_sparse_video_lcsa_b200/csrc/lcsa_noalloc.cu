@@ -159,7 +159,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   const size_t rope_n = size_t(g.Tkv) * rs.pairs_t + size_t(g.gh) * rs.pairs_h + size_t(g.gw) * rs.pairs_w;
   const size_t off_err = 0;
   const size_t off_cnt = off_err + 256;  // K1 split counters, cleared together with the error word
-  const size_t off_sp = off_cnt + round256(size_t(lcsa::kMaxK1Ctas) * 4);
+  const size_t off_sp = off_cnt + round256(size_t(lcsa::kCounters) * 4);
   const size_t off_rope = off_sp + round256(size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4);
   const size_t off_rp = off_rope + round256(rope_n * sizeof(float2));
   const size_t off_ci = off_rp + round256((size_t(ng.rows) + 1) * 4);
@@ -251,7 +251,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.topk = ng.topk;
   k2.sort_n = sort_n;
   k2.clear_cnt = split_cnt;
-  k2.n_clear = lcsa::kMaxK1Ctas;
+  k2.n_clear = lcsa::kCounters;
   k2.ring_fb = g.Tkv / g.bt;
   k2.slot0_fb = 0;
   k2.thresh = nullptr;  // no threshold reuse without a plan
@@ -292,6 +292,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.pair_len = pair_len;
   k3.npairs = int(npairs);
   k3.pair_cap = pair_cap;
+  k3.work_counter = split_cnt + lcsa::kMaxK1Ctas;
   {
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
