@@ -77,7 +77,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 8;  // 128 bytes of mbarriers: full[8], done[8]
 constexpr uint32_t kSmemBudget = 220 * 1024;
 constexpr uint32_t kBarBytes = 128;  // mbarriers of the ring
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
