@@ -95,6 +95,7 @@ def _cfg(**over):
     (dict(heads=17), L.LCSA_ERR_UNSUPPORTED),
     (dict(block_w=4), L.LCSA_ERR_UNSUPPORTED),                     # 32-token blocks
     (dict(block_h=16, block_w=8, grid_h=32), L.LCSA_ERR_UNSUPPORTED),  # 16 token rows per block
+    (dict(heads=2, heads_total=1), L.LCSA_ERR_INVALID_ARG),        # a shard cannot hold more heads than its layer
 ])
 def test_bad_configs_return_their_status(over, code):
     cfg = _cfg(**over)
@@ -124,6 +125,12 @@ def test_null_arguments_never_crash():
     assert lib.lcsa_get_intermediates(None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
     assert lib.lcsa_plan_set_timing(None, 1) == L.LCSA_ERR_INVALID_ARG
     assert lib.lcsa_get_kernel_times(None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_forward_stream(None, None, None, None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_stream_push(None, None, None, None, 1, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_sumsq(None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_forward_sharded(None, None, None, None, None, None, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_plan_set_threshold_reuse(None, 1) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_selection_nnz(None, None) == L.LCSA_ERR_INVALID_ARG
     lib.lcsa_plan_destroy(None)
 
 
@@ -150,3 +157,6 @@ def test_noalloc_entry_point_rejects_before_touching_a_device():
     assert L.lcsa_forward_noalloc(_cfg(local_range=2), fake, fake, fake, fake, fake, fake, 0) == \
         L.LCSA_ERR_INVALID_ARG
     assert L.lcsa_forward_noalloc(_cfg(grid_w=20), fake, fake, fake, fake, fake, fake, 0) == L.LCSA_ERR_SHAPE
+    # head-sharded layers need a plan (lcsa_sumsq / lcsa_forward_sharded)
+    assert L.lcsa_forward_noalloc(_cfg(heads=2, heads_total=4), fake, fake, fake, fake, fake, fake, 0) == \
+        L.LCSA_ERR_UNSUPPORTED
