@@ -370,18 +370,20 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
           }
         };
         if (!HEAD) {
-          float2 ss2 = make_float2(0.f, 0.f);
+          // the order of sumsq_kernel's sums (an accumulator per qg, then the
+          // butterfly), so a one-rank sharded call equals the plain call
+          float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c4 = 0; c4 < CPL; ++c4) {
             float2 e[2], o[2];
             unpack_eo(raw[c4], e, o);
 #pragma unroll
             for (int qg = 0; qg < 2; ++qg) {
-              ss2 = __ffma2_rn(e[qg], e[qg], ss2);
-              ss2 = __ffma2_rn(o[qg], o[qg], ss2);
+              acc[qg] = __ffma2_rn(e[qg], e[qg], acc[qg]);
+              acc[qg] = __ffma2_rn(o[qg], o[qg], acc[qg]);
             }
           }
-          float ss = ss2.x + ss2.y;
+          float ss = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
           if (ss_row) ss = __ldg(ss_row + i);  // head-sharded layer: the sum over all its heads
@@ -531,7 +533,8 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
 
 // One warp per token (q tokens, then k tokens): every 16-byte chunk of the
 // token is requested before any is summed (at most 8 per lane: heads <= 16),
-// fp32 squares, then a butterfly.
+// fp32 squares, then a butterfly; the same order of additions as the
+// prologue's own sums of squares.
 __global__ void __launch_bounds__(256) sumsq_kernel(const __nv_bfloat16* xq, int64_t nq, const __nv_bfloat16* xk,
                                                     int64_t nk, int channels, float* ss) {
   const int64_t t = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
