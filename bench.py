@@ -79,9 +79,15 @@ def _kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
-def _profiled_traffic(kernel_tag, files):
+def _launches_per_call(wl):
+    """Kernels of ours in one call: prologue, selection, attention; 64-token
+    blocks add the pair-union kernel."""
+    return 3 + (1 if wl.block_t * wl.block_h * wl.block_w == 64 else 0)
+
+
+def _profiled_traffic(kernel_tag, files, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (same hash); else None."""
+    the current kernel source (same hash) and on this workload; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -89,7 +95,7 @@ def _profiled_traffic(kernel_tag, files):
     with open(path) as f:
         for line in f:
             m = re.match(r"\s*(\w+)\s+src=(\w+)\s+workload=(\S+)\s+dram_bytes_per_launch=([0-9.eE+]+)", line)
-            if m and m.group(1) == kernel_tag and m.group(2) == want:
+            if m and m.group(1) == kernel_tag and m.group(2) == want and m.group(3) == workload:
                 return float(m.group(4))
     return None
 
@@ -342,7 +348,7 @@ def run_lcsa(args):
     k3_tflops = flops / (kms[2] * 1e-3) / 1e12
     k1_gbs = geo.prologue_bytes / (kms[0] * 1e-3) / 1e9
     k3_src = "k3_attention_tc.cu"
-    traffic = _profiled_traffic("k3", [k3_src, "lcsa_internal.h"])
+    traffic = _profiled_traffic("k3", [k3_src, "lcsa_internal.h"], args.workload)
     roofline = {"bound": "tensor", "kernel": "attention (K3, %s)" % k3_src, "achieved": k3_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": k3_tflops / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_source": peaks["source"] + " burst bf16",
@@ -365,7 +371,7 @@ def run_lcsa(args):
                         "prologue_bytes": geo.prologue_bytes, "hbm_peak_gbs": peaks["hbm_gbs"]},
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": _launches_per_call(wl) * args.steps,
             "clocks": clocks.summary()}
     if world == 1 and not args.no_cpu_baseline:
         cb = _oracle_sample(wl, inp)
@@ -637,7 +643,7 @@ def run_sharded(args):
                        "l2": "256 MiB buffer written before every timed call", "parallelism": "heads%d" % world},
             "sumsq": {"ms": ss_ms, "bytes": ss_bytes, "gbs": ss_bytes / (ss_ms * 1e-3) / 1e9,
                       "hbm_frac": ss_bytes / (ss_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (1 + _launches_per_call(wl)) * args.steps,
             "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     if world > 1:
