@@ -1,0 +1,53 @@
+"""bench.py host logic on CPU: the launch count it claims per call and the
+recorded DRAM traffic it attaches to the roofline (only for the workload and
+kernel source the capture was taken on)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from block_sparse_video_lcsa_b200 import synth  # noqa: E402
+
+K3_FILES = ["k3_attention_tc.cu", "lcsa_internal.h"]
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_launch_count_per_call(name):
+    wl = synth.WORKLOADS[name]
+    nb = wl.block_t * wl.block_h * wl.block_w
+    # K1, K2, K3; 64-token blocks add the pair-union kernel between K2 and K3
+    assert bench._launches_per_call(wl) == (4 if nb == 64 else 3)
+
+
+def _records():
+    out = []
+    with open(os.path.join(ROOT, "profiles", "dram_traffic.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                fields = dict(kv.split("=", 1) for kv in line.split()[1:])
+                out.append((line.split()[0], fields["src"], fields["workload"], float(fields["dram_bytes_per_launch"])))
+    return out
+
+
+def test_recorded_traffic_is_keyed_by_workload_and_source():
+    recs = _records()
+    assert recs, "no traffic record"
+    src = bench._kernel_source_hash(K3_FILES)
+    for tag, h, wl, nbytes in recs:
+        assert wl in synth.WORKLOADS, wl
+        got = bench._profiled_traffic(tag, K3_FILES, wl)
+        assert got == (nbytes if h == src else None)
+    recorded = {wl for _, _, wl, _ in recs}
+    for wl in synth.WORKLOADS:
+        if wl not in recorded:
+            assert bench._profiled_traffic("k3", K3_FILES, wl) is None
+
+
+def test_recorded_traffic_is_dropped_once_the_source_changes(monkeypatch):
+    monkeypatch.setattr(bench, "_kernel_source_hash", lambda files: "0" * 16)
+    for wl in synth.WORKLOADS:
+        assert bench._profiled_traffic("k3", K3_FILES, wl) is None
