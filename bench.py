@@ -71,11 +71,37 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(text):
+    """C/C++/CUDA source without its comments, whitespace runs collapsed: an
+    edit that only touches comments or layout leaves it unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or character literal, kept verbatim
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def _kernel_source_hash(files):
+    """sha256 prefix of the kernel's code (comments and layout excluded)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "block_sparse_video_lcsa_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "block_sparse_video_lcsa_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

@@ -17,8 +17,11 @@
 // one thread issues the MMAs, and P goes back to tensor memory as the A
 // operand of the P.V product.
 //
-// Persistent: one CTA per SM walks rows (batch, head, query block) r =
-// blockIdx.x, blockIdx.x + gridDim.x, ... Roles (352 threads):
+// Persistent: one CTA per SM takes work items (rows (batch, head, query
+// block), or pairs of 64-token query blocks) from a global counter: the
+// producer warp draws the next item and hands it to the other roles through
+// a four-slot queue in shared memory, so CTAs that drew short items take
+// more. Roles (352 threads):
 //   warp 0  TMA producer: Q tile of the row, then K^ / V blocks of its CSR list
 //           (K^ from the block-major prologue output, V straight from the
 //           raster input through a 5-D tensor map: d, head, x, y, frame).

@@ -51,3 +51,12 @@ def test_recorded_traffic_is_dropped_once_the_source_changes(monkeypatch):
     monkeypatch.setattr(bench, "_kernel_source_hash", lambda files: "0" * 16)
     for wl in synth.WORKLOADS:
         assert bench._profiled_traffic("k3", K3_FILES, wl) is None
+
+
+def test_source_hash_ignores_comments_but_not_code():
+    a = 'int f(int x) {  // twice\n  return 2 * x; /* doubled */ }\nconst char* s = "a // b";\n'
+    b = '/* header */\nint f(int x) {\n\n  return 2 * x;\n}\nconst char* s = "a // b";  // string kept\n'
+    c = 'int f(int x) { return 3 * x; }\nconst char* s = "a // b";\n'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert '"a // b"' in bench._code_only(a)
