@@ -1,9 +1,11 @@
 """Build liblcsa.so (sm_100a) in-tree from csrc/*.cu with nvcc.
 
-    python -m block_sparse_video_lcsa_b200.build [--force] [--verbose]
+    python -m block_sparse_video_lcsa_b200.build [--force] [--verbose] [--nvtx]
 
 Objects go to _build/ (ignored by git); the library lands next to this file,
-where the binding loads it. Rebuilds only when a source or header is newer.
+where the binding loads it. Rebuilds only when a source or header is newer,
+or when the flags differ from the last build's. --nvtx compiles in NVTX
+ranges around the kernel launches of each call (csrc/nvtx_range.h).
 """
 from __future__ import annotations
 
@@ -41,9 +43,20 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, nvtx: bool = False) -> str:
     srcs = _sources()
     hdrs = _headers()
+    extra = ["-DLCSA_NVTX"] if nvtx else []
+    flags = FLAGS + extra
+    # the optional flags of the last build (no stamp: a default build)
+    stamp = os.path.join(BUILD, "extra_flags.txt")
+    want = " ".join(extra)
+    have = ""
+    if os.path.exists(stamp):
+        with open(stamp) as f:
+            have = f.read()
+    if have != want:
+        force = True  # the objects were built with other optional flags
     if not force and not _stale(LIB, srcs + hdrs + [__file__]):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
@@ -52,7 +65,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         if force or _stale(obj, [src] + hdrs + [__file__]):
-            cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+            cmd = [NVCC] + ARCH + flags + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
             r = subprocess.run(cmd, capture_output=True, text=True)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed for %s:\n%s%s" % (src, r.stdout, r.stderr))
@@ -63,13 +76,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, srcs))
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs
+    cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + (["-ldl"] if nvtx else [])
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
     os.replace(tmp, LIB)
+    with open(stamp, "w") as f:
+        f.write(want)
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, nvtx="--nvtx" in sys.argv))

@@ -12,6 +12,7 @@
 
 #include "lcsa.h"
 #include "lcsa_internal.h"
+#include "nvtx_range.h"
 
 namespace {
 
@@ -499,7 +500,10 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   cudaEvent_t* ev = nullptr;
   if (sb.with_q && !p->evsets.empty()) ev = p->evsets[size_t(p->timed % int64_t(p->evsets.size()))].data();
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
-  if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
+  {
+    LCSA_RANGE("lcsa K1 prologue");
+    if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
+  }
   if (!sb.with_q) {
     // no K2 after this K1: clear its merge counters here
     if ((e = cudaMemsetAsync(p->split_cnt, 0, size_t(lcsa::kCounters) * 4, s)) != cudaSuccess)
@@ -507,8 +511,12 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     return LCSA_OK;
   }
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
-  if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  {
+    LCSA_RANGE("lcsa K2 select");
+    if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  }
   if (p->pair_col) {
+    LCSA_RANGE("lcsa pair union");
     lcsa::PairParams pp{};
     pp.g = g;
     pp.npairs = p->npairs;
@@ -526,6 +534,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   p->last_reuse = reuse;
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
   {
+    LCSA_RANGE("lcsa K3 attention");
     CUtensorMap tm_v;
     if ((e = lcsa::make_raster_map(&tm_v, sb.v_attn, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
@@ -585,6 +594,7 @@ lcsa_status_t lcsa_sumsq(lcsa_plan_t p, const void* q, const void* k, float* ssq
   if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
   const lcsa::Grid& g = p->res.grid;
   const int64_t nq = int64_t(g.B) * g.Lq, nk = int64_t(g.B) * g.Lkv;
+  LCSA_RANGE("lcsa sumsq");
   if ((e = lcsa::launch_sumsq(static_cast<const __nv_bfloat16*>(q), nq, static_cast<const __nv_bfloat16*>(k), nk,
                               g.C, ssq, s)) != cudaSuccess)
     return cuda_fail(e, "sum of squares launch");
@@ -651,8 +661,11 @@ lcsa_status_t stream_step(lcsa_plan_t p, const void* q, const void* k, const voi
     }
   const int64_t w0_fb = after - ring;  // window frame-block 0, counted from the first push (may be < 0)
   const int t0 = p->cfg.kv_frame_offset + int(w0_fb) * g.bt;
-  if ((e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, t0, p->cfg.head_dim, s)) != cudaSuccess)
-    return cuda_fail(e, "rope table launch");
+  {
+    LCSA_RANGE("lcsa rope table");
+    if ((e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, t0, p->cfg.head_dim, s)) != cudaSuccess)
+      return cuda_fail(e, "rope table launch");
+  }
   StepBlocks sb;
   sb.with_q = q != nullptr;
   sb.k_in_fb = fb;

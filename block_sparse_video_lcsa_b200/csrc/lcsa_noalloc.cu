@@ -23,6 +23,7 @@
 
 #include "lcsa.h"
 #include "lcsa_internal.h"
+#include "nvtx_range.h"
 
 namespace {
 
@@ -209,8 +210,11 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
 
   if ((e = cudaMemsetAsync(err, 0, off_sp - off_err, s)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "clear error word and counters");
-  if ((e = lcsa::launch_rope_table(rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, D, s)) != cudaSuccess)
-    return noalloc_fail(LCSA_ERR_CUDA, "rope table launch");
+  {
+    LCSA_RANGE("lcsa rope table");
+    if ((e = lcsa::launch_rope_table(rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, D, s)) != cudaSuccess)
+      return noalloc_fail(LCSA_ERR_CUDA, "rope table launch");
+  }
   noalloc_row_ptr_kernel<<<1, 32, 0, s>>>(row_ptr, g, radius, ng.topk);
   if ((e = cudaGetLastError()) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "row offsets launch");
 
@@ -237,7 +241,10 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   lcsa::k1_all_blocks(k1);
   if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return noalloc_fail(LCSA_ERR_CUDA, "device attributes");
-  if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
+  {
+    LCSA_RANGE("lcsa K1 prologue");
+    if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
+  }
 
   int sort_n = 32;
   while (sort_n < ng.max_window) sort_n <<= 1;
@@ -259,8 +266,12 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.col_pad = nullptr;
   k2.row_len = nullptr;
   k2.pad_cap = 0;
-  if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
+  {
+    LCSA_RANGE("lcsa K2 select");
+    if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
+  }
   if (npairs) {
+    LCSA_RANGE("lcsa pair union");
     lcsa::PairParams pp{};
     pp.g = g;
     pp.npairs = int(npairs);
@@ -294,6 +305,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.pair_cap = pair_cap;
   k3.work_counter = split_cnt + lcsa::kMaxK1Ctas;
   {
+    LCSA_RANGE("lcsa K3 attention");
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
     if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||

@@ -160,3 +160,16 @@ def test_noalloc_entry_point_rejects_before_touching_a_device():
     # head-sharded layers need a plan (lcsa_sumsq / lcsa_forward_sharded)
     assert L.lcsa_forward_noalloc(_cfg(heads=2, heads_total=4), fake, fake, fake, fake, fake, fake, 0) == \
         L.LCSA_ERR_UNSUPPORTED
+
+
+def test_nvtx_ranges_compile(tmp_path):
+    """The optional NVTX ranges (build --nvtx) compile in both entry-point
+    files; the objects go to a temporary directory, the in-tree library is
+    left as built."""
+    import subprocess
+    for f in ("lcsa_api.cu", "lcsa_noalloc.cu"):
+        src = os.path.join(ROOT, "block_sparse_video_lcsa_b200", "csrc", f)
+        cmd = [lcsa_build.NVCC] + lcsa_build.ARCH + lcsa_build.FLAGS + ["-DLCSA_NVTX", "-c", src, "-o",
+                                                                       str(tmp_path / (f + ".o"))]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr[-2000:]
