@@ -13,6 +13,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -30,9 +31,12 @@ _lib = None
 
 
 def lib():
+    """The oracle's shared library: the in-tree build, or the build named by
+    LCSA_ORACLE_LIB (the mutation tests load copies of lcsa_oracle.cpp with a
+    planted mistake this way and check that the pins catch each)."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("LCSA_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         G = ctypes.POINTER(_Geom)

@@ -260,6 +260,51 @@ def test_rotation_angle_is_linear_in_position_and_first_pair_turns_one_radian():
     assert np.all(np.diff(grp) < 0)
 
 
+def test_every_axis_follows_the_rope_frequency_schedule():
+    """The RoPE reading: a step of one position along an axis of n dims turns
+    that axis' pair j by 10000^(-2j/n) radians (the standard rotary frequencies
+    per axis), with n = 44 for frames and 42 each for rows and columns at
+    head_dim 128. Measured from the turn of each pair between neighbouring
+    tokens that hold the same vector."""
+    wl, g = tiny(kv_frames=2, q_frames=2)
+    inp = _same_vector_everywhere(g, wl)
+    D = g.head_dim
+    assert D == 128
+    dims = {"t": 44, "h": 42, "w": 42}
+    first = {"t": 0, "h": 22, "w": 43}           # first pair of each axis
+
+    def tok(t, y, x):
+        return (t * g.grid_h + y) * g.grid_w + x
+
+    v0, vt, vh, vw = oracle.norm_rope(g, inp.k, inp.gamma_k, False,
+                                      [tok(0, 3, 4), tok(1, 3, 4), tok(0, 4, 4), tok(0, 3, 5)])
+    for hd in range(g.heads):
+        sl = slice(hd * D, (hd + 1) * D)
+        for axis, vec in (("t", vt), ("h", vh), ("w", vw)):
+            turn = _pair_angles(vec[sl], v0[sl])
+            n = dims[axis]
+            j = np.arange(n // 2)
+            np.testing.assert_allclose(turn[first[axis] + j], 10000.0 ** (-2.0 * j / n), rtol=0, atol=1e-11)
+
+
+def test_query_frames_are_the_last_frames_of_the_window():
+    """Queries are the last q_frames of the KV window: a query token and the
+    key token at the same place of the last KV frame, holding the same vector
+    and gains, come out of the norm and rotation identical; the same vector at
+    the same place of an earlier KV frame does not."""
+    wl, g = tiny(q_frames=1, kv_frames=3, kv_frame_offset=4)
+    inp = synth.make_inputs(wl)
+    tpf = g.grid_h * g.grid_w
+    inp.q[0, :tpf] = inp.k[0, 2 * tpf:3 * tpf]  # the query frame holds the last KV frame's vectors
+    inp.k[0, :tpf] = inp.k[0, 2 * tpf:3 * tpf]  # and so does the first KV frame
+    toks = np.arange(0, tpf, 37)
+    qh = oracle.norm_rope(g, inp.q, inp.gamma_k, True, toks)
+    k_last = oracle.norm_rope(g, inp.k, inp.gamma_k, False, 2 * tpf + toks)
+    k_first = oracle.norm_rope(g, inp.k, inp.gamma_k, False, toks)
+    np.testing.assert_array_equal(qh, k_last)
+    assert not np.allclose(qh, k_first)
+
+
 def test_scores_and_outputs_are_invariant_to_the_frame_offset():
     wl, g = tiny(q_frames=1, kv_frames=2, local_range=3)
     inp = synth.make_inputs(wl)
