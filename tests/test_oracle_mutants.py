@@ -70,6 +70,38 @@ MUTANTS = {
                                   ("int64_t xx = i % g.block_w;", "int64_t xx = (i / g.block_h) % g.block_w;")],
     # budget rule with the latent grid not scaled to pixels
     "budget_pixel_scale": [("double H = 16.0 * grid_h, W = 16.0 * grid_w;", "double H = 8.0 * grid_h, W = 8.0 * grid_w;")],
+    # budget rounded instead of floored
+    "budget_rounded": [("std::floor(num / (H * W))", "std::round(num / (H * W))")],
+    # eps dropped from the norm
+    "norm_eps_dropped": [("ss / double(d.C) + g.rms_eps", "ss / double(d.C)")],
+    # a token's row and column taken with the grid's sides exchanged
+    "token_row_from_height": [("int64_t y = (tok / g.grid_w) % g.grid_h;", "int64_t y = (tok / g.grid_h) % g.grid_w;")],
+    "token_column_from_height": [("int64_t xcol = tok % g.grid_w;", "int64_t xcol = tok % g.grid_h;")],
+    # rotation pairs (j, j + d/2) instead of (2j, 2j+1)
+    "rotation_pairs_half_split": [
+        ("double a = out[h * D + 2 * j], b = out[h * D + 2 * j + 1];",
+         "double a = out[h * D + j], b = out[h * D + j + D / 2];"),
+        ("out[h * D + 2 * j] = a * cs[j] - b * sn[j];", "out[h * D + j] = a * cs[j] - b * sn[j];"),
+        ("out[h * D + 2 * j + 1] = a * sn[j] + b * cs[j];", "out[h * D + j + D / 2] = a * sn[j] + b * cs[j];")],
+    # pooled output laid out head-major over the batch
+    "pooled_layout_head_batch": [("pooled[((b * g.heads + h) * nblk + blk) * D + e]",
+                                  "pooled[((h * g.batch + b) * nblk + blk) * D + e]")],
+    # attention rows split into (batch, head) the wrong way round
+    "attention_row_split": [("int64_t b = bh / g.heads, h = bh % g.heads;",
+                             "int64_t b = bh % g.batch, h = bh / g.batch;")],
+    # query tokens addressed with the key tensor's batch stride
+    "query_batch_stride": [("q + (b * d.Lq + tok) * d.C", "q + (b * d.Lkv + tok) * d.C")],
+    # values of head 0 for every head
+    "values_head_zero": [("v[(b * d.Lkv + tok) * d.C + h * D + e]", "v[(b * d.Lkv + tok) * d.C + e]")],
+    # pooled keys of the first (batch, head) for every row
+    "score_keys_of_head_zero": [("const double* kk = pk + (bh * d.nKB + kb) * D;", "const double* kk = pk + kb * D;")],
+    # score matrix without the window's -inf
+    "scores_unmasked": [("scores[row * d.nKB + kb] = ok ? s : -std::numeric_limits<double>::infinity();",
+                         "scores[row * d.nKB + kb] = s;")],
+    # window column distance against the key's block row
+    "window_column_index": [("dw = qrem % d.nWb - krem % d.nWb", "dw = qrem % d.nWb - krem / d.nWb")],
+    # gap measured from the best score instead of the k-th
+    "gap_from_best": [("cand[keff - 1].first - cand[keff].first", "cand[0].first - cand[keff].first")],
 }
 
 

@@ -265,8 +265,9 @@ def test_every_axis_follows_the_rope_frequency_schedule():
     that axis' pair j by 10000^(-2j/n) radians (the standard rotary frequencies
     per axis), with n = 44 for frames and 42 each for rows and columns at
     head_dim 128. Measured from the turn of each pair between neighbouring
-    tokens that hold the same vector."""
-    wl, g = tiny(kv_frames=2, q_frames=2)
+    tokens that hold the same vector, and between tokens far apart on a
+    grid wider than it is high (row and column come from the raster index)."""
+    wl, g = tiny(kv_frames=2, q_frames=2, grid_w=32)
     inp = _same_vector_everywhere(g, wl)
     D = g.head_dim
     assert D == 128
@@ -276,8 +277,8 @@ def test_every_axis_follows_the_rope_frequency_schedule():
     def tok(t, y, x):
         return (t * g.grid_h + y) * g.grid_w + x
 
-    v0, vt, vh, vw = oracle.norm_rope(g, inp.k, inp.gamma_k, False,
-                                      [tok(0, 3, 4), tok(1, 3, 4), tok(0, 4, 4), tok(0, 3, 5)])
+    v0, vt, vh, vw, vfar = oracle.norm_rope(g, inp.k, inp.gamma_k, False,
+                                            [tok(0, 3, 4), tok(1, 3, 4), tok(0, 4, 4), tok(0, 3, 5), tok(1, 11, 27)])
     for hd in range(g.heads):
         sl = slice(hd * D, (hd + 1) * D)
         for axis, vec in (("t", vt), ("h", vh), ("w", vw)):
@@ -285,6 +286,36 @@ def test_every_axis_follows_the_rope_frequency_schedule():
             n = dims[axis]
             j = np.arange(n // 2)
             np.testing.assert_allclose(turn[first[axis] + j], 10000.0 ** (-2.0 * j / n), rtol=0, atol=1e-11)
+        # (0, 3, 4) -> (1, 11, 27): 1 frame, 8 rows and 23 columns, angles modulo 2 pi
+        turn = _pair_angles(vfar[sl], v0[sl])
+        for axis, steps in (("t", 1), ("h", 8), ("w", 23)):
+            n = dims[axis]
+            j = np.arange(n // 2)
+            np.testing.assert_allclose(np.exp(1j * turn[first[axis] + j]), np.exp(1j * steps * 10000.0 ** (-2.0 * j / n)),
+                                       rtol=0, atol=1e-10)
+
+
+def test_batch_entries_are_independent():
+    """The entries of a batch do not interact: each entry of a batch-2 call
+    gives the pooled values, selection and outputs of a batch-1 call on that
+    entry alone (rows are numbered batch, then head, then query block)."""
+    over = dict(heads=3, q_frames=1, kv_frames=2, local_range=3, topk=3)
+    wl, g = tiny(batch=2, **over)
+    inp = synth.make_inputs(wl)
+    pq, pk, sel, out, _ = oracle.run(g, inp)
+    _, g1 = tiny(batch=1, **over)
+    per = g1.rows
+    for b in range(2):
+        one = synth.Inputs(q=inp.q[b:b + 1].copy(), k=inp.k[b:b + 1].copy(), v=inp.v[b:b + 1].copy(),
+                           gamma_q=inp.gamma_q, gamma_k=inp.gamma_k)
+        pq1, pk1, sel1, out1, _ = oracle.run(g1, one)
+        np.testing.assert_array_equal(pq[b], pq1[0])
+        np.testing.assert_array_equal(pk[b], pk1[0])
+        r = slice(b * per, (b + 1) * per)
+        np.testing.assert_array_equal(sel.row_len[r], sel1.row_len)
+        np.testing.assert_array_equal(sel.cols[r], sel1.cols)
+        np.testing.assert_array_equal(out[r], out1)
+    assert not np.allclose(out[:per], out[per:])  # the two entries differ
 
 
 def test_query_frames_are_the_last_frames_of_the_window():

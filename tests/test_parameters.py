@@ -44,3 +44,12 @@ def test_budget_of_the_measured_workloads():
     for name, k in want.items():
         g = oracle.Geometry.from_workload(synth.WORKLOADS[name])
         assert g.topk == k, name
+
+
+def test_budget_is_floored():
+    """The budget reading takes the floor of topk_ratio * blocks per latent
+    frame: at 768x1280 (30 blocks of 128 tokens per frame) sparse_ratio 1.55
+    gives 46.5 blocks -> 46; at 768x1408 (66 blocks of 64 tokens) sparse_ratio
+    1.01 gives 60.6 -> 60."""
+    assert oracle.resolve_topk(1.55, 48, 80, 1, 8, 16) == 46
+    assert oracle.resolve_topk(1.01, 48, 88, 1, 8, 8) == 60
