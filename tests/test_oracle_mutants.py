@@ -102,6 +102,20 @@ MUTANTS = {
     "window_column_index": [("dw = qrem % d.nWb - krem % d.nWb", "dw = qrem % d.nWb - krem / d.nWb")],
     # gap measured from the best score instead of the k-th
     "gap_from_best": [("cand[keff - 1].first - cand[keff].first", "cand[0].first - cand[keff].first")],
+    # head scope: every head takes the first head's gains
+    "head_gain_of_head_zero": [("out[h * D + e] * inv * double(gamma[h * D + e])", "out[h * D + e] * inv * double(gamma[e])")],
+    # the absolute frame offset given to the keys only
+    "frame_offset_keys_only": [("double t_abs = double(g.kv_frame_offset) + double(is_q ? (g.kv_frames - g.q_frames) : 0)",
+                                "double t_abs = double(is_q ? 0 : g.kv_frame_offset) + "
+                                "double(is_q ? (g.kv_frames - g.q_frames) : 0)")],
+    # window restricted to the query's own frame
+    "window_same_frame_only": [("if (g.local_range <= 0) return true;",
+                                "if (qb / d.bpf != kb / d.bpf) return false;\n  if (g.local_range <= 0) return true;")],
+    # pooling rotates query blocks at key positions
+    "pool_query_flag_dropped": [("norm_rope_token(g, d, x + (b * L + tok) * d.C, gamma, is_q != 0, tok, v.data());",
+                                 "norm_rope_token(g, d, x + (b * L + tok) * d.C, gamma, false, tok, v.data());")],
+    # attention rotates queries at key positions
+    "attention_query_flag_dropped": [("gamma_q, true, tok, tokvec.data());", "gamma_q, false, tok, tokvec.data());")],
 }
 
 

@@ -191,8 +191,13 @@ def test_rmsnorm_closed_form_and_direction(scope):
         assert cos == pytest.approx(1.0, abs=1e-13)
 
 
-def test_gain_scales_each_channel():
-    wl, g = tiny()
+@pytest.mark.parametrize("scope", [0, 1])
+def test_gain_scales_each_channel(scope):
+    """Each channel's gain multiplies that channel after the norm, in both
+    scopes (three heads, so the heads' gains differ)."""
+    wl, g = tiny(heads=3)
+    g.norm_scope = scope
+    g.kv_frame_offset = 0                            # token (0, 0, 0): no rotation
     inp = synth.make_inputs(wl)
     gam = (1.0 + 0.25 * np.arange(g.C) / g.C).astype(np.float32)
     a = oracle.norm_rope(g, inp.k, inp.gamma_k, False, [0])[0]
