@@ -166,10 +166,26 @@ def lcsa_config_resolve(cfg: lcsa_config_t) -> lcsa_geometry_t:
     return g
 
 
+def _expect_tensor(t, dtype, shape, name, device):
+    """`t` must be a contiguous tensor of `dtype` and `shape` (None: any) on
+    CUDA device `device` (an index) or, with device "cpu", in host memory.
+    Integers pass through as raw addresses. The C ABI cannot see dtypes,
+    strides or devices, so a mismatch is refused here before any call."""
+    if isinstance(t, int):
+        return
+    on_it = (not t.is_cuda) if device == "cpu" else (t.is_cuda and t.device.index == device)
+    if (t.dtype != dtype or not on_it or not t.is_contiguous() or
+            (shape is not None and tuple(t.shape) != tuple(shape))):
+        raise ValueError("%s: want a contiguous %s tensor%s on %s, got %s %s on %s%s" % (
+            name, dtype, "" if shape is None else " of shape %s" % (tuple(shape),),
+            "the host" if device == "cpu" else "cuda:%d" % device, t.dtype, tuple(t.shape), t.device,
+            "" if t.is_contiguous() else " (not contiguous)"))
+
+
 def lcsa_plan_create(cfg: lcsa_config_t, device: int = 0) -> "Plan":
     h = _PLAN()
     _check(lib().lcsa_plan_create(ctypes.byref(cfg), int(device), ctypes.byref(h)), "lcsa_plan_create")
-    return Plan(h, cfg)
+    return Plan(h, cfg, int(device))
 
 
 def lcsa_plan_create_stream(cfg: lcsa_config_t, device: int = 0) -> "Plan":
@@ -177,7 +193,7 @@ def lcsa_plan_create_stream(cfg: lcsa_config_t, device: int = 0) -> "Plan":
     ring; feed it with Plan.lcsa_stream_push and Plan.lcsa_forward_stream."""
     h = _PLAN()
     _check(lib().lcsa_plan_create_stream(ctypes.byref(cfg), int(device), ctypes.byref(h)), "lcsa_plan_create_stream")
-    return Plan(h, cfg)
+    return Plan(h, cfg, int(device))
 
 
 LCSA_NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -186,7 +202,17 @@ LCSA_NOALLOC_WORKSPACE_BYTES = 32 << 20
 def lcsa_forward_noalloc(cfg: lcsa_config_t, q, k, v, gamma_q, gamma_k, out, stream=None) -> int:
     """Plan-free call for callers that may not allocate device memory: every
     intermediate lives in the library's static device workspace. Returns the
-    status code (LCSA_ERR_UNSUPPORTED when the problem does not fit)."""
+    status code (LCSA_ERR_UNSUPPORTED when the problem does not fit). Tensors
+    must be contiguous, of the right dtype and on the current CUDA device;
+    their sizes are the caller's contract, as in the C ABI."""
+    if any(t is not None and not isinstance(t, int) for t in (q, k, v, gamma_q, gamma_k, out)):
+        import torch
+        dev = torch.cuda.current_device()
+        for t, dt, name in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"), (v, torch.bfloat16, "v"),
+                            (out, torch.bfloat16, "out"), (gamma_q, torch.float32, "gamma_q"),
+                            (gamma_k, torch.float32, "gamma_k")):
+            if t is not None:
+                _expect_tensor(t, dt, None, name, dev)
     return int(lib().lcsa_forward_noalloc(ctypes.byref(cfg), _addr(q), _addr(k), _addr(v), _addr(gamma_q),
                                           _addr(gamma_k), _addr(out), _stream(stream)))
 
@@ -205,9 +231,10 @@ def config_from_workload(wl, **over) -> lcsa_config_t:
 class Plan:
     """Owner of an lcsa_plan_t; every method maps to one C entry point."""
 
-    def __init__(self, handle, cfg):
+    def __init__(self, handle, cfg, device: int = 0):
         self._h = handle
         self.cfg = cfg
+        self.device = device  # the CUDA device the plan's memory and kernels live on
         g = lcsa_geometry_t()
         _check(lib().lcsa_plan_geometry(self._h, ctypes.byref(g)), "lcsa_plan_geometry")
         self.geometry = g
@@ -227,14 +254,8 @@ class Plan:
         except Exception:  # noqa: BLE001 - interpreter shutdown
             pass
 
-    def _expect(self, t, dtype, shape, name):
-        if isinstance(t, int):
-            return
-        import torch
-        if t.dtype != dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
-            raise ValueError("%s: want contiguous CUDA %s %s, got %s %s %s" % (
-                name, dtype, tuple(shape), t.dtype, tuple(t.shape), t.device))
-        _ = torch  # the check above needs torch only for real tensors
+    def _expect(self, t, dtype, shape, name, host=False):
+        _expect_tensor(t, dtype, shape, name, "cpu" if host else self.device)
 
     def lcsa_forward(self, q, k, v, gamma_q, gamma_k, out, stream=None):
         import torch
@@ -303,6 +324,14 @@ class Plan:
 
     def lcsa_forward_host(self, q, k, v, gamma_q, gamma_k, out, stream=None):
         """Host (preferably pinned) tensors in and out; copies are inside the call."""
+        import torch
+        c, g = self.cfg, self.geometry
+        self._expect(q, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "q", host=True)
+        self._expect(k, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "k", host=True)
+        self._expect(v, torch.bfloat16, (c.batch, g.kv_tokens, g.channels), "v", host=True)
+        self._expect(out, torch.bfloat16, (c.batch, g.q_tokens, g.channels), "out", host=True)
+        self._expect(gamma_q, torch.float32, (g.channels,), "gamma_q", host=True)
+        self._expect(gamma_k, torch.float32, (g.channels,), "gamma_k", host=True)
         _check(lib().lcsa_forward_host(self._h, _addr(q), _addr(k), _addr(v), _addr(gamma_q), _addr(gamma_k),
                                        _addr(out), _stream(stream)), "lcsa_forward_host")
         return out

@@ -173,3 +173,53 @@ def test_nvtx_ranges_compile(tmp_path):
                                                                        str(tmp_path / (f + ".o"))]
         r = subprocess.run(cmd, capture_output=True, text=True)
         assert r.returncode == 0, r.stderr[-2000:]
+
+
+class _FakeTensor:
+    """Just the attributes the binding's tensor checks read."""
+
+    def __init__(self, dtype, shape, cuda_index=None, contiguous=True):
+        import types
+        self.dtype, self.shape, self._c = dtype, tuple(shape), contiguous
+        self.is_cuda = cuda_index is not None
+        self.device = types.SimpleNamespace(index=cuda_index, type="cuda" if self.is_cuda else "cpu")
+
+    def is_contiguous(self):
+        return self._c
+
+
+def test_binding_refuses_tensors_it_cannot_pass_on():
+    """dtype, shape, contiguity and device (the plan's GPU, or the host for the
+    host-buffer call) are checked in Python before any C call: a tensor on
+    another GPU would have the kernels read that GPU's memory."""
+    import torch
+    t = torch.bfloat16
+    want = (1, 512, 256)
+    L._expect_tensor(_FakeTensor(t, want, 1), t, want, "q", 1)
+    L._expect_tensor(_FakeTensor(t, want), t, want, "q", "cpu")
+    L._expect_tensor(12345, t, want, "q", 0)                       # raw addresses pass through
+    for bad, dev in ((_FakeTensor(t, want, 0), 1),                 # another GPU
+                     (_FakeTensor(t, want), 0),                    # host memory for a device argument
+                     (_FakeTensor(t, want, 0), "cpu"),             # device memory for a host argument
+                     (_FakeTensor(torch.float16, want, 0), 0),     # dtype
+                     (_FakeTensor(t, (1, 512, 128), 0), 0),        # shape
+                     (_FakeTensor(t, want, 0, contiguous=False), 0)):
+        with pytest.raises(ValueError):
+            L._expect_tensor(bad, t, want, "q", dev)
+    # the host-buffer call checks before it reaches the library (here: a plan without a handle)
+    plan = L.Plan.__new__(L.Plan)
+    plan._h, plan.device = None, 0
+    plan.cfg = L.config_from_workload(synth.WORKLOADS["tiny"])
+    plan.geometry = L.lcsa_config_resolve(plan.cfg)
+    g, c = plan.geometry, plan.cfg
+    ok = [_FakeTensor(t, (c.batch, g.q_tokens, g.channels)), _FakeTensor(t, (c.batch, g.kv_tokens, g.channels)),
+          _FakeTensor(t, (c.batch, g.kv_tokens, g.channels)), _FakeTensor(torch.float32, (g.channels,)),
+          _FakeTensor(torch.float32, (g.channels,)), _FakeTensor(t, (c.batch, g.q_tokens, g.channels))]
+    wrong = list(ok)
+    wrong[1] = _FakeTensor(t, (c.batch, g.kv_tokens + 1, g.channels))
+    with pytest.raises(ValueError):
+        plan.lcsa_forward_host(*wrong, stream=0)
+    wrong = list(ok)
+    wrong[0] = _FakeTensor(t, (c.batch, g.q_tokens, g.channels), 0)
+    with pytest.raises(ValueError):
+        plan.lcsa_forward_host(*wrong, stream=0)
