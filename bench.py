@@ -259,10 +259,18 @@ def run_reference(args):
             samples.append(r)
     ms = statistics.mean(s["ms_per_call"] for s in samples)
     value = statistics.mean(s["value"] for s in samples)
+    import numpy as np
+    import oracle
+    og = oracle.Geometry.from_workload(wl)
+    kept = int(np.minimum(oracle.window_sizes(og), og.topk).sum()) * og.batch * og.heads
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name},
+            "config": {"workload": wl.name, "q_tokens": wl.q_tokens, "kv_tokens": wl.kv_tokens,
+                       "heads": wl.heads, "head_dim": wl.head_dim,
+                       "block": "%dx%dx%d" % (wl.block_t, wl.block_h, wl.block_w), "local_range": wl.local_range,
+                       "sparse_ratio": wl.sparse_ratio, "topk": og.topk, "kept_blocks": kept, "selection": "top-k",
+                       "parallelism": "rank 0 of %d, host cores" % args.gpus},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[-1]["cores"], "kind": "oracle",
                              "sample": samples[-1]["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -60,3 +60,26 @@ def test_source_hash_ignores_comments_but_not_code():
     assert bench._code_only(a) == bench._code_only(b)
     assert bench._code_only(a) != bench._code_only(c)
     assert '"a // b"' in bench._code_only(a)
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints
+    one JSON line with the contract's keys, on the same workload keys as the
+    CUDA arm's line."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "dtype", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    wl = synth.WORKLOADS[d["config"]["workload"]]
+    assert d["config"]["q_tokens"] == wl.q_tokens and d["config"]["kv_tokens"] == wl.kv_tokens
+    assert d["config"]["kept_blocks"] == 43200  # 720 rows x 60 blocks on the default workload
