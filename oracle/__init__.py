@@ -4,6 +4,10 @@ Only the tests, the smoke check and the benchmark's CPU-baseline leg may
 import this package. It wraps the C++ routines of ``lcsa_oracle.cpp`` with
 ctypes; it shares no code with the CUDA library and never calls it.
 
+Parity unpinned against the pages: the RoPE frequency schedule and the
+block-budget reading (the pages say only "factored 3D RoPE" and print the
+topk_ratio formula); the pins fix the oracle to those readings.
+
 Rows are numbered (batch, head, query block) with the query block fastest,
 blocks are numbered (frame group, block row, block column), tokens inside a
 block (frame, row, column), exactly as in the C++ file.

@@ -34,6 +34,8 @@
 //    edge, the same in every frame of the KV window; 0 means unbounded.
 //  * budget: k = floor(topk_ratio * blocks per latent frame), H = 16 H',
 //    W = 16 W' (VAE 8x and 2x2 patchify), unless an explicit k is given.
+//    Parity of this reading is unpinned against the pages beyond their
+//    printed topk_ratio formula.
 //  * query frames are the last q_frames of the KV window.
 //  * ties between equal scores go to the lower KV block index.
 #include <algorithm>
