@@ -21,7 +21,11 @@ from __future__ import annotations
 
 
 def head_slices(heads_total: int, world: int):
-    """Contiguous head ranges [h0, h1) of `world` ranks, sizes differing by at most one."""
+    """Contiguous head ranges [h0, h1) of `world` ranks, sizes differing by at
+    most one; every rank holds at least one head."""
+    if world < 1 or heads_total < world:
+        raise ValueError("cannot split %d heads over %d ranks (each rank needs at least one head)"
+                         % (heads_total, world))
     base, extra = divmod(heads_total, world)
     out, h0 = [], 0
     for r in range(world):

@@ -109,3 +109,6 @@ def test_head_slices_cover_the_layer():
             assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
             sizes = [h1 - h0 for h0, h1 in sl]
             assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    for heads, world in ((3, 4), (12, 0), (1, 2)):
+        with pytest.raises(ValueError):
+            head_slices(heads, world)
