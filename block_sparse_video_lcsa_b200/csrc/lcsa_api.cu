@@ -45,9 +45,11 @@ struct Resolved {
 // Budget in blocks: topk_ratio = sparse_ratio * 768 * 1280 / (H * W) with the
 // pixel size H = 16 grid_h, W = 16 grid_w ("FlashVSR Inference" skill,
 // Non-Negotiable Streaming Contract), times the blocks of one latent frame.
+// A budget beyond 2^30 blocks keeps every admissible block anyway.
 int budget_from_ratio(double sparse_ratio, int gh, int gw, int64_t blocks_per_frame) {
   const double pixels = (16.0 * gh) * (16.0 * gw);
-  return int(std::floor(sparse_ratio * 983040.0 * double(blocks_per_frame) / pixels));
+  const double k = std::floor(sparse_ratio * 983040.0 * double(blocks_per_frame) / pixels);
+  return k >= double(1 << 30) ? (1 << 30) : int(k);
 }
 
 lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
@@ -59,11 +61,12 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
     return fail(LCSA_ERR_INVALID_ARG, "local_range %d must be odd (a centred window diameter) or 0 (unbounded)",
                 c->local_range);
   if (c->topk < 0) return fail(LCSA_ERR_INVALID_ARG, "topk %d < 0", c->topk);
-  if (c->topk == 0 && !(c->sparse_ratio > 0.f))
-    return fail(LCSA_ERR_INVALID_ARG, "topk = 0 needs sparse_ratio > 0");
+  if (c->topk == 0 && !(c->sparse_ratio > 0.f && std::isfinite(c->sparse_ratio)))
+    return fail(LCSA_ERR_INVALID_ARG, "topk = 0 needs a finite sparse_ratio > 0");
   if (c->norm_scope != LCSA_NORM_TOKEN && c->norm_scope != LCSA_NORM_HEAD)
     return fail(LCSA_ERR_INVALID_ARG, "norm_scope %d", c->norm_scope);
-  if (!(c->rms_eps > 0.f)) return fail(LCSA_ERR_INVALID_ARG, "rms_eps must be > 0");
+  if (!(c->rms_eps > 0.f) || !std::isfinite(c->rms_eps))
+    return fail(LCSA_ERR_INVALID_ARG, "rms_eps must be finite and > 0");
   if (!(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale))
     return fail(LCSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   if (c->kv_frame_offset < 0) return fail(LCSA_ERR_INVALID_ARG, "kv_frame_offset < 0");
@@ -82,6 +85,13 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   if (c->heads_total != 0 && c->heads_total < c->heads)
     return fail(LCSA_ERR_INVALID_ARG, "heads_total %d < heads %d", c->heads_total, c->heads);
   r->heads_total = c->heads_total == 0 ? c->heads : c->heads_total;
+  // bound the sizes (in floating point, so nothing below can overflow): at
+  // most 2^40 elements per tensor, hence at most 2^33 tokens and 2^27 blocks,
+  // which every int block count and int64 token index holds
+  const double elems_max = double(c->batch) * double(c->kv_frames) * double(c->grid_h) * double(c->grid_w) *
+                           double(c->heads) * double(c->head_dim);
+  if (elems_max > double(int64_t(1) << 40))
+    return fail(LCSA_ERR_UNSUPPORTED, "tensor of %.4g elements (> 2^40)", elems_max);
 
   lcsa::Grid& g = r->grid;
   g.B = c->batch;
@@ -103,8 +113,6 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   g.Lkv = int64_t(c->kv_frames) * c->grid_h * c->grid_w;
   g.C = c->heads * c->head_dim;
 
-  const int64_t elems = int64_t(c->batch) * g.Lkv * g.C;
-  if (elems > (int64_t(1) << 40)) return fail(LCSA_ERR_UNSUPPORTED, "tensor of %lld elements", (long long)elems);
   const int64_t rows = int64_t(g.B) * g.Hn * g.nQB;
   if (rows > (int64_t(1) << 30)) return fail(LCSA_ERR_UNSUPPORTED, "%lld rows", (long long)rows);
 

@@ -73,9 +73,10 @@ lcsa_status_t noalloc_resolve(const lcsa_config_t* c, NoallocGeom* out) {
     return noalloc_fail(LCSA_ERR_INVALID_ARG, "sizes must be >= 1");
   if (c->local_range < 0 || (c->local_range != LCSA_UNBOUNDED && c->local_range % 2 == 0))
     return noalloc_fail(LCSA_ERR_INVALID_ARG, "local_range must be odd or 0 (unbounded)");
-  if (c->topk < 0 || (c->topk == 0 && !(c->sparse_ratio > 0.f)))
-    return noalloc_fail(LCSA_ERR_INVALID_ARG, "topk < 0, or topk = 0 without sparse_ratio > 0");
+  if (c->topk < 0 || (c->topk == 0 && !(c->sparse_ratio > 0.f && std::isfinite(c->sparse_ratio))))
+    return noalloc_fail(LCSA_ERR_INVALID_ARG, "topk < 0, or topk = 0 without a finite sparse_ratio > 0");
   if ((c->norm_scope != LCSA_NORM_TOKEN && c->norm_scope != LCSA_NORM_HEAD) || !(c->rms_eps > 0.f) ||
+      !std::isfinite(c->rms_eps) ||
       !(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale) || c->kv_frame_offset < 0)
     return noalloc_fail(LCSA_ERR_INVALID_ARG, "norm_scope, rms_eps, softmax_scale or kv_frame_offset out of range");
   if (c->kv_frames < c->q_frames || c->grid_h % c->block_h || c->grid_w % c->block_w || c->q_frames % c->block_t ||
@@ -85,6 +86,11 @@ lcsa_status_t noalloc_resolve(const lcsa_config_t* c, NoallocGeom* out) {
   if (c->head_dim != lcsa::kHeadDim || c->heads > lcsa::kMaxHeads || (nb != 64 && nb != 128) ||
       c->block_t * c->block_h > 8)
     return noalloc_fail(LCSA_ERR_UNSUPPORTED, "head_dim, heads or block shape outside what the kernels implement");
+  // sizes bounded in floating point before any integer product (2^40
+  // elements per tensor at most: every block count below fits an int)
+  if (double(c->batch) * double(c->kv_frames) * double(c->grid_h) * double(c->grid_w) * double(c->heads) *
+          double(c->head_dim) > double(int64_t(1) << 40))
+    return noalloc_fail(LCSA_ERR_UNSUPPORTED, "tensor of more than 2^40 elements");
   lcsa::Grid& g = out->g;
   g.B = c->batch;
   g.Hn = c->heads;
@@ -107,9 +113,11 @@ lcsa_status_t noalloc_resolve(const lcsa_config_t* c, NoallocGeom* out) {
   // budget: topk_ratio = sparse_ratio*768*1280/(H*W), H = 16 grid_h, W = 16 grid_w,
   // times the blocks of one latent frame
   int topk = c->topk;
-  if (topk == 0)
-    topk = int(std::floor(double(c->sparse_ratio) * 983040.0 * double(g.bpf) /
-                          ((16.0 * c->grid_h) * (16.0 * c->grid_w))));
+  if (topk == 0) {
+    const double k = std::floor(double(c->sparse_ratio) * 983040.0 * double(g.bpf) /
+                                ((16.0 * c->grid_h) * (16.0 * c->grid_w)));
+    topk = k >= double(1 << 30) ? (1 << 30) : int(k);  // beyond 2^30: every admissible block
+  }
   if (topk < 1) return noalloc_fail(LCSA_ERR_INVALID_ARG, "sparse_ratio gives a budget of 0 blocks");
   out->topk = topk;
   out->radius = c->local_range == LCSA_UNBOUNDED ? -1 : (c->local_range - 1) / 2;

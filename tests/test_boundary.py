@@ -108,6 +108,47 @@ def test_bad_configs_return_their_status(over, code):
     assert h.value is None
 
 
+@pytest.mark.parametrize("over,code", [
+    (dict(topk=0, sparse_ratio=float("inf")), L.LCSA_ERR_INVALID_ARG),
+    (dict(topk=0, sparse_ratio=float("nan")), L.LCSA_ERR_INVALID_ARG),
+    (dict(rms_eps=float("inf")), L.LCSA_ERR_INVALID_ARG),
+    (dict(rms_eps=float("nan")), L.LCSA_ERR_INVALID_ARG),
+    (dict(grid_h=1 << 30, grid_w=1 << 30), L.LCSA_ERR_UNSUPPORTED),    # products beyond int64 if formed
+    (dict(q_frames=1, kv_frames=1 << 30), L.LCSA_ERR_UNSUPPORTED),
+    (dict(batch=1 << 30, heads=16), L.LCSA_ERR_UNSUPPORTED),
+])
+def test_extreme_values_are_refused_by_both_entry_paths(over, code):
+    """Non-finite parameters and sizes whose products would overflow are
+    refused before any product is formed, by the plan path and by the
+    allocation-free path alike."""
+    cfg = _cfg(**over)
+    g = L.lcsa_geometry_t()
+    assert L.lib().lcsa_config_resolve(ctypes.byref(cfg), ctypes.byref(g)) == code, L.lcsa_last_error_message()
+    fake = 1 << 20
+    assert L.lcsa_forward_noalloc(cfg, fake, fake, fake, fake, fake, fake, 0) == code, L.lcsa_last_error_message()
+
+
+def test_huge_sparse_ratio_keeps_every_admissible_block():
+    cfg = _cfg(topk=0, sparse_ratio=1e30, local_range=3)
+    g = L.lcsa_config_resolve(cfg)
+    assert g.topk == 1 << 30
+    assert g.nnz == g.rows // g.q_blocks * sum(_window_sizes(cfg, g))
+
+
+def _window_sizes(cfg, g):
+    """Admissible blocks of every query block: frames x clipped row span x clipped column span."""
+    r = (cfg.local_range - 1) // 2
+    nh, nw = cfg.grid_h // cfg.block_h, cfg.grid_w // cfg.block_w
+    out = []
+    for qb in range(g.q_blocks):
+        rem = qb % (nh * nw)
+        hb, wb = divmod(rem, nw)
+        rows = min(hb + r, nh - 1) - max(hb - r, 0) + 1
+        cols = min(wb + r, nw - 1) - max(wb - r, 0) + 1
+        out.append(cfg.kv_frames // cfg.block_t * rows * cols)
+    return out
+
+
 def test_window_too_large_for_the_selection_sort():
     cfg = _cfg(grid_h=8 * 40, grid_w=8 * 40, q_frames=1, kv_frames=3, local_range=0, topk=4)
     g = L.lcsa_geometry_t()
