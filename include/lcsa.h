@@ -100,10 +100,11 @@ typedef struct lcsa_config {
                                      block_t*block_h <= 8 */
   int local_range;      /* odd window diameter in blocks, or LCSA_UNBOUNDED */
   int topk;             /* > 0: budget in blocks; 0: derive from sparse_ratio */
-  float sparse_ratio;   /* used when topk == 0 (1.5 or 2.0 on the pages) */
+  float sparse_ratio;   /* used when topk == 0 (1.5 or 2.0 on the pages): finite, > 0;
+                           a budget beyond 2^30 blocks keeps every admissible block */
   int kv_frame_offset;  /* absolute latent frame index of KV frame 0 (RoPE) */
   int norm_scope;       /* LCSA_NORM_TOKEN or LCSA_NORM_HEAD */
-  float rms_eps;        /* > 0 */
+  float rms_eps;        /* finite, > 0 */
   float softmax_scale;  /* 0: 1/sqrt(head_dim) */
   int host_io;          /* 1: also allocate device staging for lcsa_forward_host */
   int heads_total;      /* 0, or the heads of the whole layer when this plan holds
@@ -135,7 +136,15 @@ typedef struct lcsa_plan* lcsa_plan_t;
 LCSA_API void lcsa_config_default(lcsa_config_t* cfg);
 
 /* Validate *cfg and derive its sizes. Host only: touches no device.
-   Returns LCSA_ERR_INVALID_ARG / SHAPE / UNSUPPORTED on a bad config. */
+   Returns LCSA_ERR_INVALID_ARG (a size < 1, an even or negative local_range,
+   topk < 0, a non-finite or non-positive sparse_ratio (when used) or rms_eps,
+   a negative or non-finite softmax_scale, kv_frame_offset < 0, a budget of 0
+   blocks, heads_total < heads), LCSA_ERR_SHAPE (kv_frames < q_frames, or a
+   token grid the block does not divide) or LCSA_ERR_UNSUPPORTED (head_dim
+   other than 128, more heads than the kernels take, blocks of other than 64
+   or 128 tokens or more than 8 token rows, a tensor of more than 2^40
+   elements, a window larger than the selection's candidate limit). Sizes are
+   bounded before any product of them is formed. */
 LCSA_API lcsa_status_t lcsa_config_resolve(const lcsa_config_t* cfg, lcsa_geometry_t* out);
 
 /* Validate, then allocate every intermediate on `cuda_device` and build the
