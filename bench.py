@@ -105,6 +105,18 @@ def _kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
+def _spread(values):
+    """p10 / median / p90 of per-call times (linear interpolation between ranks)."""
+    xs = sorted(float(x) for x in values)
+
+    def q(f):
+        i = f * (len(xs) - 1)
+        lo = int(math.floor(i))
+        hi = min(lo + 1, len(xs) - 1)
+        return xs[lo] + (xs[hi] - xs[lo]) * (i - lo)
+    return {"p10": q(0.1), "median": q(0.5), "p90": q(0.9)}
+
+
 def _launches_per_call(wl):
     """Kernels of ours in one call: prologue, selection, attention; 64-token
     blocks add the pair-union kernel."""
@@ -345,6 +357,17 @@ def run_lcsa(args):
     plan.lcsa_plan_set_timing(0)
     kept = plan.lcsa_selection_nnz()  # the blocks the timed calls kept (threshold reuse may differ from k)
     total_ms = _max_over_ranks(sum(step_ms), dev)
+    # warm L2: the same calls without the flush between them (context for the
+    # flushed figure, which is the reported one)
+    warm_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    warm_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        warm_starts[i].record(stream)
+        plan.lcsa_forward(q, k, v, gq, gk, out, stream)
+        warm_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    plan.lcsa_check_device_error(stream)
+    warm_ms = _max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(warm_starts, warm_ends)), dev) / args.steps
 
     # end to end: pinned host buffers through lcsa_forward_host (copies inside)
     hq = torch.from_numpy(inp.q).view(torch.bfloat16).pin_memory()
@@ -392,6 +415,7 @@ def run_lcsa(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "ms_per_step_spread": _spread(step_ms), "warm_l2_ms_per_step": warm_ms,
             "config": {"workload": wl.name, "q_tokens": geo.q_tokens, "kv_tokens": geo.kv_tokens,
                        "heads": wl.heads, "head_dim": wl.head_dim,
                        "block": "%dx%dx%d" % (wl.block_t, wl.block_h, wl.block_w), "local_range": wl.local_range,

@@ -83,3 +83,9 @@ def test_reference_arm_line():
     wl = synth.WORKLOADS[d["config"]["workload"]]
     assert d["config"]["q_tokens"] == wl.q_tokens and d["config"]["kv_tokens"] == wl.kv_tokens
     assert d["config"]["kept_blocks"] == 43200  # 720 rows x 60 blocks on the default workload
+
+
+def test_spread_of_call_times():
+    d = bench._spread([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert d == {"p10": 1.4, "median": 3.0, "p90": 4.6}
+    assert bench._spread([0.41]) == {"p10": 0.41, "median": 0.41, "p90": 0.41}
