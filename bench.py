@@ -42,14 +42,18 @@ FLUSH_BYTES = 256 << 20
 
 
 def _args():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="stream_768x1280")
-    ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    from block_sparse_video_lcsa_b200 import synth
+    ap = argparse.ArgumentParser(description="Time the LCSA call on synthetic inputs; prints one JSON line.")
+    ap.add_argument("--gpus", type=int, default=1, help="ranks (one GPU each; N > 1 under torchrun)")
+    ap.add_argument("--steps", type=int, default=50, help="timed calls")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed calls before them")
+    ap.add_argument("--workload", default="stream_768x1280", choices=list(synth.WORKLOADS),
+                    help="synthetic workload (default: the 768x1280 stream chunk)")
+    ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"],
+                    help="lcsa: the CUDA library; reference: the fp64 CPU oracle on the host cores")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle sample of the CPU baseline")
+    ap.add_argument("--e2e-steps", type=int, default=10,
+                    help="calls timed end to end through host buffers (copies included)")
     ap.add_argument("--layers", type=int, default=0,
                     help="time N sequential calls (a DiT chunk's attention layers), eager and as one CUDA graph")
     ap.add_argument("--stream", action="store_true",
