@@ -80,6 +80,7 @@ SIGNATURES = [
     ("lcsa_forward", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_forward_host", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("lcsa_forward_noalloc", _I, [ctypes.POINTER(lcsa_config_t), _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    ("lcsa_noalloc_check_device_error", _I, [_VP]),
     ("lcsa_plan_create_stream", _I, [ctypes.POINTER(lcsa_config_t), _I, ctypes.POINTER(_PLAN)]),
     ("lcsa_stream_push", _I, [_PLAN, _VP, _VP, _VP, _I, _VP]),
     ("lcsa_forward_stream", _I, [_PLAN, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
@@ -215,6 +216,13 @@ def lcsa_forward_noalloc(cfg: lcsa_config_t, q, k, v, gamma_q, gamma_k, out, str
                 _expect_tensor(t, dt, None, name, dev)
     return int(lib().lcsa_forward_noalloc(ctypes.byref(cfg), _addr(q), _addr(k), _addr(v), _addr(gamma_q),
                                           _addr(gamma_k), _addr(out), _stream(stream)))
+
+
+def lcsa_noalloc_check_device_error(stream=None) -> int:
+    """Status of the device error word of lcsa_forward_noalloc's static
+    workspace in the current context (synchronises the stream, reads and
+    clears the word): LCSA_OK, LCSA_ERR_DEVICE_TIMEOUT or LCSA_ERR_DEVICE_BOUNDS."""
+    return int(lib().lcsa_noalloc_check_device_error(_stream(stream)))
 
 
 def config_from_workload(wl, **over) -> lcsa_config_t:

@@ -83,7 +83,13 @@ constexpr int kPolyEvery = 4;  // one pair of exponentials in kPolyEvery on the 
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 384, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+#ifdef LCSA_TEST_STALL
+// test-only build (liblcsa_stalltest.so): waits give up after 100 ms, so a
+// test can make one run out quickly
+constexpr unsigned long long kWaitLimitNs = 100000000ull;
+#else
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+#endif
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
@@ -113,6 +119,7 @@ struct Bars {
   // dynamic work distribution: the producer takes the next work item from
   // the global counter and hands it to the other roles through item[]
   uint64_t item_full[kItemSlots], item_empty[kItemSlots];
+  uint64_t never;  // test-only build: a barrier nothing arrives on
   int item[kItemSlots];
   uint32_t tmem_base;
   int abort;
@@ -135,6 +142,7 @@ struct TcParams {
   unsigned* err;
   int rows;
   unsigned* work_counter;  // zero at launch; each CTA takes work items from it
+  int stall_site;          // test-only build: 0, or where the first work item stalls
 };
 
 // Selected blocks of row rr: col_idx[row_begin .. row_begin + row_count).
@@ -417,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(bars->o_free), kSoftmaxWarps);
     mbar_init(bar(bars->mma_drain[0]), 1);
     mbar_init(bar(bars->mma_drain[1]), 1);
+    mbar_init(bar(bars->never), 1);
     for (int s = 0; s < 4; ++s) mbar_init(bar(bars->pair[s]), 64);
     for (int s = 0; s < kItemSlots; ++s) {
       mbar_init(bar(bars->item_full[s]), 1);
@@ -446,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int krow = 0, x0 = 0, y0 = 0, f0 = 0;
     };
     int kv = 0, row_it = 0;
+    int q_issued = 0, k_issued = 0, v_issued = 0;  // tiles whose loads this warp has issued
     bool ok = true;
     for (int it = 0; ok; ++it, ++row_it) {
       const int rr = take_item(it, ok);
@@ -474,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
+      q_issued = row_it + 1;
       const int steps = (n + KB - 1) / KB;
       auto fill = [&](Entries& e, int chunk) {
         e.chunk = chunk;
@@ -512,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         __syncwarp();
+        k_issued = kvj + 1;
         return true;
       };
       for (int st = 0; st < 2 && st < steps && ok; ++st) ok = load_k(st);
@@ -532,9 +544,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         __syncwarp();
+        v_issued = kvj + 1;
+#ifdef LCSA_TEST_STALL
+        if (p.stall_site == 1 && it == 0 && st == 0) {
+          // give up at once, with the work item's first loads just issued
+          if (lane == 0) {
+            *abort = 1;
+            if (atomicCAS(p.err, kDevErrNone, kDevErrTimeout) == kDevErrNone) {
+              p.err[1] = 91;
+              p.err[2] = blockIdx.x;
+            }
+          }
+          __syncwarp();
+          ok = false;
+          break;
+        }
+#endif
       }
       kv += steps;
     }
+    // Every load this warp issued lands before the CTA's final barrier: on a
+    // normal exit the consumers have already waited for all of them, but if
+    // any role gave up, tiles issued and not yet consumed may still be in
+    // flight into shared memory. The last phase of each barrier is the one to
+    // wait for: a stage is reloaded only after its previous tile was
+    // consumed, so that phase's completion implies the earlier ones', and no
+    // later phase exists (so the parity test is unambiguous). The waits ignore
+    // the abort flag and give up only at the wall-clock limit.
+    if (lane == 0) {
+      if (q_issued > 0) mbar_drain(bar(bars->q_full), uint32_t(q_issued - 1) & 1u);
+      for (int st = 0; st < kKStages; ++st)
+        if (k_issued > st) {
+          const int last = (k_issued - 1) - ((k_issued - 1 - st) % kKStages);
+          mbar_drain(bar(bars->k_full[st]), uint32_t(last / kKStages) & 1u);
+        }
+      for (int st = 0; st < kVStages; ++st)
+        if (v_issued > st) {
+          const int last = (v_issued - 1) - ((v_issued - 1 - st) % kVStages);
+          mbar_drain(bar(bars->v_full[st]), uint32_t(last / kVStages) & 1u);
+        }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------- S issuer (converged warp, lane 0 issues) ----------------
     constexpr uint32_t id_qk = idesc_bf16(0, QM);
@@ -647,6 +697,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           masked = e >= n_sel || !((__ldg(lst + e) >> kPairShift) & (sp < 2 ? 1 : 2));
         }
         const int sb = s_it % kSBufs;
+#ifdef LCSA_TEST_STALL
+        // a wait that nothing ends: it runs out after the (test) limit
+        if (p.stall_site == 2 && warp == 3 && it == 0 && j == 0 &&
+            !(ok = warp_wait(bar(bars->never), 0, abort, p.err, 92)))
+          break;
+#endif
         if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
         uint32_t sr[2][32];
@@ -869,6 +925,12 @@ cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+#ifdef LCSA_TEST_STALL
+namespace {
+int g_stall_site = 0;  // consumed by the next attention launch
+}
+#endif
+
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s) {
   if (!attention_tc_supported(p.g)) return cudaErrorInvalidValue;
@@ -894,9 +956,22 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.pair_cap = p.pair_cap;
   tp.ring_fb = p.ring_fb;
   tp.slot0_fb = p.slot0_fb;
+#ifdef LCSA_TEST_STALL
+  tp.stall_site = g_stall_site;
+  g_stall_site = 0;
+#endif
   const int grid = tp.rows < num_sms ? tp.rows : num_sms;
   kern<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();
 }
 
 }  // namespace lcsa
+
+#ifdef LCSA_TEST_STALL
+// Test-only build: make the next attention launch give up a wait in its
+// first work item. site 1: the TMA producer aborts right after issuing the
+// item's first loads (they are still in flight); site 2: a softmax warp waits
+// on a barrier nothing arrives on until the (100 ms) limit. Either records
+// LCSA_ERR_DEVICE_TIMEOUT (error sites 91 / 92) and the kernel winds down.
+extern "C" LCSA_API void lcsa_test_arm_stall(int site) { lcsa::g_stall_site = site; }
+#endif

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -42,125 +43,31 @@ struct Resolved {
   int heads_total;     // heads of the whole (possibly head-sharded) layer
 };
 
-// Budget in blocks: topk_ratio = sparse_ratio * 768 * 1280 / (H * W) with the
-// pixel size H = 16 grid_h, W = 16 grid_w ("FlashVSR Inference" skill,
-// Non-Negotiable Streaming Contract), times the blocks of one latent frame.
-// A budget beyond 2^30 blocks keeps every admissible block anyway.
-int budget_from_ratio(double sparse_ratio, int gh, int gw, int64_t blocks_per_frame) {
-  const double pixels = (16.0 * gh) * (16.0 * gw);
-  const double k = std::floor(sparse_ratio * 983040.0 * double(blocks_per_frame) / pixels);
-  return k >= double(1 << 30) ? (1 << 30) : int(k);
-}
-
+// Checks and sizes come from lcsa::resolve_config (lcsa_config.cu), which the
+// allocation-free entry point shares; the plan path adds the CSR row offsets
+// (they depend on the geometry only) and the workspace size.
 lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
-  if (!c) return fail(LCSA_ERR_INVALID_ARG, "config is null");
-  if (c->batch < 1 || c->heads < 1 || c->head_dim < 1 || c->q_frames < 1 || c->kv_frames < 1 || c->grid_h < 1 ||
-      c->grid_w < 1 || c->block_t < 1 || c->block_h < 1 || c->block_w < 1)
-    return fail(LCSA_ERR_INVALID_ARG, "sizes must be >= 1");
-  if (c->local_range < 0 || (c->local_range != LCSA_UNBOUNDED && c->local_range % 2 == 0))
-    return fail(LCSA_ERR_INVALID_ARG, "local_range %d must be odd (a centred window diameter) or 0 (unbounded)",
-                c->local_range);
-  if (c->topk < 0) return fail(LCSA_ERR_INVALID_ARG, "topk %d < 0", c->topk);
-  if (c->topk == 0 && !(c->sparse_ratio > 0.f && std::isfinite(c->sparse_ratio)))
-    return fail(LCSA_ERR_INVALID_ARG, "topk = 0 needs a finite sparse_ratio > 0");
-  if (c->norm_scope != LCSA_NORM_TOKEN && c->norm_scope != LCSA_NORM_HEAD)
-    return fail(LCSA_ERR_INVALID_ARG, "norm_scope %d", c->norm_scope);
-  if (!(c->rms_eps > 0.f) || !std::isfinite(c->rms_eps))
-    return fail(LCSA_ERR_INVALID_ARG, "rms_eps must be finite and > 0");
-  if (!(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale))
-    return fail(LCSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
-  if (c->kv_frame_offset < 0) return fail(LCSA_ERR_INVALID_ARG, "kv_frame_offset < 0");
-  if (c->kv_frames < c->q_frames)
-    return fail(LCSA_ERR_SHAPE, "kv_frames %d < q_frames %d (queries are the last frames of the KV window)",
-                c->kv_frames, c->q_frames);
-  if (c->grid_h % c->block_h || c->grid_w % c->block_w || c->q_frames % c->block_t || c->kv_frames % c->block_t)
-    return fail(LCSA_ERR_SHAPE, "token grid %dx%dx%d (q %d) not divisible by block %dx%dx%d", c->kv_frames,
-                c->grid_h, c->grid_w, c->q_frames, c->block_t, c->block_h, c->block_w);
-  if (c->head_dim != lcsa::kHeadDim) return fail(LCSA_ERR_UNSUPPORTED, "head_dim %d (only 128)", c->head_dim);
-  if (c->heads > lcsa::kMaxHeads) return fail(LCSA_ERR_UNSUPPORTED, "heads %d > %d", c->heads, lcsa::kMaxHeads);
-  const int nb = c->block_t * c->block_h * c->block_w;
-  if (nb != 64 && nb != 128) return fail(LCSA_ERR_UNSUPPORTED, "block of %d tokens (64 or 128)", nb);
-  if (c->block_t * c->block_h > 8)
-    return fail(LCSA_ERR_UNSUPPORTED, "block_t*block_h = %d > 8 token rows", c->block_t * c->block_h);
-  if (c->heads_total != 0 && c->heads_total < c->heads)
-    return fail(LCSA_ERR_INVALID_ARG, "heads_total %d < heads %d", c->heads_total, c->heads);
-  r->heads_total = c->heads_total == 0 ? c->heads : c->heads_total;
-  // bound the sizes (in floating point, so nothing below can overflow): at
-  // most 2^40 elements per tensor, hence at most 2^33 tokens and 2^27 blocks,
-  // which every int block count and int64 token index holds
-  const double elems_max = double(c->batch) * double(c->kv_frames) * double(c->grid_h) * double(c->grid_w) *
-                           double(c->heads) * double(c->head_dim);
-  if (elems_max > double(int64_t(1) << 40))
-    return fail(LCSA_ERR_UNSUPPORTED, "tensor of %.4g elements (> 2^40)", elems_max);
-
-  lcsa::Grid& g = r->grid;
-  g.B = c->batch;
-  g.Hn = c->heads;
-  g.Tq = c->q_frames;
-  g.Tkv = c->kv_frames;
-  g.gh = c->grid_h;
-  g.gw = c->grid_w;
-  g.bt = c->block_t;
-  g.bh = c->block_h;
-  g.bw = c->block_w;
-  g.nb = nb;
-  g.nHb = c->grid_h / c->block_h;
-  g.nWb = c->grid_w / c->block_w;
-  g.bpf = g.nHb * g.nWb;
-  g.nQB = (c->q_frames / c->block_t) * g.bpf;
-  g.nKB = (c->kv_frames / c->block_t) * g.bpf;
-  g.Lq = int64_t(c->q_frames) * c->grid_h * c->grid_w;
-  g.Lkv = int64_t(c->kv_frames) * c->grid_h * c->grid_w;
-  g.C = c->heads * c->head_dim;
-
-  const int64_t rows = int64_t(g.B) * g.Hn * g.nQB;
-  if (rows > (int64_t(1) << 30)) return fail(LCSA_ERR_UNSUPPORTED, "%lld rows", (long long)rows);
-
-  int topk = c->topk;
-  if (topk == 0) {
-    topk = budget_from_ratio(double(c->sparse_ratio), c->grid_h, c->grid_w, g.bpf);
-    if (topk < 1)
-      return fail(LCSA_ERR_INVALID_ARG, "sparse_ratio %g gives a budget of %d blocks", double(c->sparse_ratio), topk);
-  }
-  r->radius = c->local_range == LCSA_UNBOUNDED ? -1 : (c->local_range - 1) / 2;
-
-  // admissible-set size per query block: frame groups x clipped window
-  const int groups = g.nKB / g.bpf;
-  auto span = [](int center, int rad, int n) {
-    if (rad < 0) return n;
-    const int lo = center - rad < 0 ? 0 : center - rad;
-    const int hi = center + rad > n - 1 ? n - 1 : center + rad;
-    return hi - lo + 1;
-  };
-  int wmin = 1 << 30, wmax = 0;
-  int64_t nnz_per_head = 0;
-  std::vector<int32_t> keff(g.nQB);
-  for (int qb = 0; qb < g.nQB; ++qb) {
-    const int rem = qb % g.bpf;
-    const int a = groups * span(rem / g.nWb, r->radius, g.nHb) * span(rem % g.nWb, r->radius, g.nWb);
-    wmin = a < wmin ? a : wmin;
-    wmax = a > wmax ? a : wmax;
-    keff[qb] = topk < a ? topk : a;
-    nnz_per_head += keff[qb];
-  }
-  if (wmax > lcsa::kMaxCandidates)
-    return fail(LCSA_ERR_UNSUPPORTED, "window holds %d blocks (> %d)", wmax, lcsa::kMaxCandidates);
-  int sort_n = 32;
-  while (sort_n < wmax) sort_n <<= 1;
-  r->sort_n = sort_n;
-
-  const int64_t nnz = nnz_per_head * g.B * g.Hn;
-  if (nnz > (int64_t(1) << 31) - 1) return fail(LCSA_ERR_UNSUPPORTED, "%lld kept blocks", (long long)nnz);
+  lcsa::ConfigCore core;
+  char why[256];
+  const lcsa_status_t st = lcsa::resolve_config(c, &core, why, sizeof(why));
+  if (st != LCSA_OK) return fail(st, "%s", why);
+  const lcsa::Grid& g = core.grid;
+  r->grid = g;
+  r->radius = core.radius;
+  r->sort_n = core.sort_n;
+  r->scale = core.scale;
+  r->heads_total = core.heads_total;
+  const int64_t rows = core.rows, nnz = core.nnz;
+  const int nb = g.nb, wmin = core.min_window, wmax = core.max_window, topk = core.topk;
   if (want_rows) {
     r->row_ptr.assign(size_t(rows) + 1, 0);
     int64_t acc = 0;
     for (int64_t row = 0; row < rows; ++row) {
       r->row_ptr[size_t(row)] = int32_t(acc);
-      acc += keff[size_t(row % g.nQB)];
+      acc += lcsa::kept_blocks(core, int(row % g.nQB));
     }
     r->row_ptr[size_t(rows)] = int32_t(acc);
   }
-  r->scale = c->softmax_scale > 0.f ? c->softmax_scale : float(1.0 / std::sqrt(double(c->head_dim)));
 
   lcsa_geometry_t& o = r->geo;
   std::memset(&o, 0, sizeof(o));
@@ -252,6 +159,8 @@ struct lcsa_plan {
   // tcgen05 attention: tensor maps of the plan-owned q^ / k^; SM count (persistent grids)
   CUtensorMap tm_q, tm_k;
   int num_sms = 0;
+  unsigned fault_launch = 0;                       // LCSA_FAULT launch:K (kFault* bits)
+  bool fault_copy = false;                         // LCSA_FAULT copy
   std::vector<std::array<cudaEvent_t, 4>> evsets;  // timing ring
   int64_t timed = 0;                                // forwards recorded
 };
@@ -271,8 +180,62 @@ void release(lcsa_plan* p) {
   p->evsets.clear();
 }
 
+// Host-side fault injection for tests of the error paths (no GPU fault is
+// involved): LCSA_FAULT, read when a plan is created, holds one of
+//   alloc:N   the N-th device allocation of that plan's creation fails (OOM)
+//   launch:K  every call of the plan reports a failed launch of kernel K
+//             (K1, K2, PAIR, K3 or ROPE) instead of launching it
+//   copy      lcsa_forward_host reports a failed host-to-device copy
+// A value that is none of these refuses the plan (LCSA_ERR_INVALID_ARG), so a
+// misspelt injection is never silently ignored.
+constexpr unsigned kFaultK1 = 1, kFaultK2 = 2, kFaultPair = 4, kFaultK3 = 8, kFaultRope = 16;
+struct Faults {
+  int alloc_at = 0;
+  unsigned launch = 0;
+  bool copy = false;
+};
+thread_local int t_alloc_countdown = 0;  // > 0 while a plan with alloc:N is being created
+
+lcsa_status_t parse_faults(Faults* f) {
+  *f = Faults{};
+  const char* v = std::getenv("LCSA_FAULT");
+  if (!v || !*v) return LCSA_OK;
+  const std::string s(v);
+  if (s == "copy") {
+    f->copy = true;
+    return LCSA_OK;
+  }
+  if (s.rfind("alloc:", 0) == 0) {
+    char* end = nullptr;
+    const long n = std::strtol(s.c_str() + 6, &end, 10);
+    if (end && *end == 0 && n >= 1 && n <= 1000) {
+      f->alloc_at = int(n);
+      return LCSA_OK;
+    }
+  }
+  const struct {
+    const char* name;
+    unsigned bit;
+  } kernels[] = {{"launch:K1", kFaultK1}, {"launch:K2", kFaultK2}, {"launch:PAIR", kFaultPair},
+                 {"launch:K3", kFaultK3}, {"launch:ROPE", kFaultRope}};
+  for (const auto& k : kernels)
+    if (s == k.name) {
+      f->launch = k.bit;
+      return LCSA_OK;
+    }
+  return fail(LCSA_ERR_INVALID_ARG, "LCSA_FAULT=%s not understood (alloc:N, launch:K1|K2|PAIR|K3|ROPE, copy)", v);
+}
+
+lcsa_status_t injected_launch_failure(const lcsa_plan* p, unsigned bit, const char* what) {
+  return (p->fault_launch & bit) ? fail(LCSA_ERR_CUDA, "%s launch: injected failure (LCSA_FAULT)", what) : LCSA_OK;
+}
+
 template <class T>
 lcsa_status_t dev_alloc(T** ptr, size_t bytes, const char* what) {
+  if (t_alloc_countdown > 0 && --t_alloc_countdown == 0) {
+    *ptr = nullptr;
+    return fail(LCSA_ERR_OOM, "cudaMalloc(%s, %zu bytes): injected failure (LCSA_FAULT)", what, bytes);
+  }
   cudaError_t e = cudaMalloc(reinterpret_cast<void**>(ptr), bytes < 16 ? 16 : bytes);
   if (e != cudaSuccess) {
     *ptr = nullptr;
@@ -291,6 +254,19 @@ lcsa_status_t alloc_pairs(lcsa_plan* p) {
   lcsa_status_t st = dev_alloc(&p->pair_col, size_t(np) * size_t(p->pair_cap) * 4, "pair lists");
   if (st == LCSA_OK) st = dev_alloc(&p->pair_len, size_t(np) * 4, "pair counts");
   return st;
+}
+
+// Read the plan's device error word (the stream is already synchronised),
+// clear it if set, and map it to a status.
+lcsa_status_t take_device_error(lcsa_plan* p) {
+  unsigned word[4] = {0, 0, 0, 0};
+  cudaError_t e = cudaMemcpy(word, p->err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (word[0] == lcsa::kDevErrNone) return LCSA_OK;
+  if ((e = cudaMemset(p->err, 0, 256)) != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (word[0] == lcsa::kDevErrTimeout)
+    return fail(LCSA_ERR_DEVICE_TIMEOUT, "kernel gave up a bounded wait (site %u, block %u)", word[1], word[2]);
+  return fail(LCSA_ERR_DEVICE_BOUNDS, "kernel index check failed (site %u, value %u)", word[1], word[2]);
 }
 
 }  // namespace
@@ -328,9 +304,13 @@ lcsa_status_t lcsa_config_resolve(const lcsa_config_t* cfg, lcsa_geometry_t* out
   return st;
 }
 
-lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out) {
-  if (!out) return fail(LCSA_ERR_INVALID_ARG, "plan output is null");
-  *out = nullptr;
+}  // extern "C"
+
+namespace {
+
+// Validate, allocate and set up a plan (the allocations count down
+// t_alloc_countdown, set by the callers from LCSA_FAULT).
+lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Faults& faults, lcsa_plan_t* out) {
   lcsa_plan* p = new (std::nothrow) lcsa_plan();
   if (!p) return fail(LCSA_ERR_OOM, "host allocation of the plan");
   lcsa_status_t st = resolve(cfg, &p->res, true);
@@ -340,6 +320,8 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
   }
   p->cfg = *cfg;
   p->device = cuda_device;
+  p->fault_launch = faults.launch;
+  p->fault_copy = faults.copy;
   cudaError_t e = cudaSetDevice(cuda_device);
   if (e != cudaSuccess) {
     delete p;
@@ -408,6 +390,22 @@ lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_p
   }
   *out = p;
   return LCSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lcsa_status_t lcsa_plan_create(const lcsa_config_t* cfg, int cuda_device, lcsa_plan_t* out) {
+  if (!out) return fail(LCSA_ERR_INVALID_ARG, "plan output is null");
+  *out = nullptr;
+  Faults faults;
+  lcsa_status_t st = parse_faults(&faults);
+  if (st != LCSA_OK) return st;
+  t_alloc_countdown = faults.alloc_at;
+  st = create_plan(cfg, cuda_device, faults, out);
+  t_alloc_countdown = 0;
+  return st;
 }
 
 void lcsa_plan_destroy(lcsa_plan_t p) {
@@ -510,6 +508,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
   {
     LCSA_RANGE("lcsa K1 prologue");
+    if (lcsa_status_t st = injected_launch_failure(p, kFaultK1, "prologue")) return st;
     if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return cuda_fail(e, "prologue launch");
   }
   if (!sb.with_q) {
@@ -521,6 +520,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
   {
     LCSA_RANGE("lcsa K2 select");
+    if (lcsa_status_t st = injected_launch_failure(p, kFaultK2, "select")) return st;
     if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   }
   if (p->pair_col) {
@@ -536,6 +536,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     pp.pair_col = p->pair_col;
     pp.pair_len = p->pair_len;
     pp.pair_cap = p->pair_cap;
+    if (lcsa_status_t st = injected_launch_failure(p, kFaultPair, "pair union")) return st;
     if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return cuda_fail(e, "pair union launch");
   }
   p->have_thresh = true;
@@ -545,6 +546,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     LCSA_RANGE("lcsa K3 attention");
     CUtensorMap tm_v;
     if ((e = lcsa::make_raster_map(&tm_v, sb.v_attn, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
+    if (lcsa_status_t st = injected_launch_failure(p, kFaultK3, "attention")) return st;
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
       return cuda_fail(e, "attention launch");
   }
@@ -624,11 +626,22 @@ lcsa_status_t lcsa_plan_create_stream(const lcsa_config_t* cfg, int cuda_device,
   if (cfg && cfg->host_io) return fail(LCSA_ERR_INVALID_ARG, "stream plans take device tensors (host_io = 0)");
   if (cfg && cfg->heads_total != 0 && cfg->heads_total != cfg->heads)
     return fail(LCSA_ERR_UNSUPPORTED, "stream plans are not head-sharded");
-  lcsa_status_t st = lcsa_plan_create(cfg, cuda_device, out);
+  if (!out) return fail(LCSA_ERR_INVALID_ARG, "plan output is null");
+  *out = nullptr;
+  Faults faults;
+  lcsa_status_t st = parse_faults(&faults);
   if (st != LCSA_OK) return st;
+  t_alloc_countdown = faults.alloc_at;
+  st = create_plan(cfg, cuda_device, faults, out);
+  if (st != LCSA_OK) {
+    t_alloc_countdown = 0;
+    return st;
+  }
   lcsa_plan* p = *out;
   const lcsa::Grid& g = p->res.grid;
-  if ((st = dev_alloc(&p->v_ring, size_t(g.B) * g.Lkv * g.C * 2, "v ring")) != LCSA_OK) {
+  st = dev_alloc(&p->v_ring, size_t(g.B) * g.Lkv * g.C * 2, "v ring");
+  t_alloc_countdown = 0;
+  if (st != LCSA_OK) {
     lcsa_plan_destroy(p);
     *out = nullptr;
     return st;
@@ -671,6 +684,7 @@ lcsa_status_t stream_step(lcsa_plan_t p, const void* q, const void* k, const voi
   const int t0 = p->cfg.kv_frame_offset + int(w0_fb) * g.bt;
   {
     LCSA_RANGE("lcsa rope table");
+    if (lcsa_status_t st = injected_launch_failure(p, kFaultRope, "rope table")) return st;
     if ((e = lcsa::launch_rope_table(p->rope, g.Tkv, g.gh, g.gw, t0, p->cfg.head_dim, s)) != cudaSuccess)
       return cuda_fail(e, "rope table launch");
   }
@@ -718,6 +732,7 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
   if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
   const lcsa::Grid& g = p->res.grid;
   const size_t qb = size_t(g.B) * g.Lq * g.C * 2, kb = size_t(g.B) * g.Lkv * g.C * 2, gb = size_t(g.C) * 4;
+  if (p->fault_copy) return fail(LCSA_ERR_CUDA, "host-to-device copy: injected failure (LCSA_FAULT)");
   if ((e = cudaMemcpyAsync(p->st_q, q, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
       (e = cudaMemcpyAsync(p->st_k, k, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
       (e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
@@ -729,7 +744,7 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
   if ((e = cudaMemcpyAsync(out, p->st_out, qb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
     return cuda_fail(e, "device-to-host copy");
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  return LCSA_OK;
+  return take_device_error(p);
 }
 
 lcsa_status_t lcsa_plan_geometry(lcsa_plan_t p, lcsa_geometry_t* out) {
@@ -822,14 +837,7 @@ lcsa_status_t lcsa_check_device_error(lcsa_plan_t p, void* stream) {
   cudaError_t e = cudaSetDevice(p->device);
   if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream");
-  unsigned word[4] = {0, 0, 0, 0};
-  if ((e = cudaMemcpy(word, p->err, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
-    return cuda_fail(e, "read error word");
-  if (word[0] == lcsa::kDevErrNone) return LCSA_OK;
-  cudaMemset(p->err, 0, 256);
-  if (word[0] == lcsa::kDevErrTimeout)
-    return fail(LCSA_ERR_DEVICE_TIMEOUT, "kernel gave up a bounded wait (site %u, block %u)", word[1], word[2]);
-  return fail(LCSA_ERR_DEVICE_BOUNDS, "kernel index check failed (site %u, value %u)", word[1], word[2]);
+  return take_device_error(p);
 }
 
 lcsa_status_t lcsa_plan_set_timing(lcsa_plan_t p, int capacity) {

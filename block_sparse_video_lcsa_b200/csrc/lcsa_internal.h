@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lcsa.h"
+
 namespace lcsa {
 
 constexpr int kHeadDim = 128;        // the only head size the kernels implement
@@ -181,6 +183,29 @@ struct K3Params {
   int pair_cap;
   unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work items from it
 };
+
+// Sizes of one configuration (lcsa_config.cu), derived without touching the
+// heap or a device, so the plan path and the allocation-free path apply the
+// same rules.
+struct ConfigCore {
+  Grid grid;
+  int topk;                  // resolved budget in blocks
+  int radius;                // window radius in blocks, -1 when unbounded
+  int sort_n;                // power of two >= max_window (K2's candidate slots)
+  int min_window, max_window;  // smallest / largest admissible set
+  int64_t rows, nnz;         // CSR rows (b, h, qb) and kept blocks in all
+  int heads_total;           // heads of the whole (possibly head-sharded) layer
+  float scale;               // softmax scale
+};
+// Validate *c and fill *out. On failure, msg (if not null) receives a
+// one-line reason; with msg null nothing is formatted.
+lcsa_status_t resolve_config(const lcsa_config_t* c, ConfigCore* out, char* msg, size_t msg_cap);
+// Budget in blocks from sparse_ratio (the topk_ratio formula, floored; a
+// budget beyond 2^30 blocks is capped there and keeps every admissible block).
+int budget_from_ratio(double sparse_ratio, int gh, int gw, int64_t blocks_per_frame);
+// Admissible blocks of query block qb, and how many of them are kept.
+int window_blocks(const ConfigCore& r, int qb);
+int kept_blocks(const ConfigCore& r, int qb);
 
 // The stateless call's block sets: every query and key block, ring = window.
 inline void k1_all_blocks(K1Params& k1) {

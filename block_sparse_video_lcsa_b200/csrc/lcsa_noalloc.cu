@@ -8,16 +8,26 @@
 // and stall the decode, encode and render streams that share it, and because
 // a late allocation can fail when another allocator already owns the memory.
 // Those callers cannot create an lcsa_plan_t (which allocates its workspace).
-// This entry point runs the same three kernels with every intermediate placed
-// in a file-scope static device array of LCSA_NOALLOC_WORKSPACE_BYTES, which
-// each GPU that loads the library holds until the process exits.
+// This entry point runs the same kernels with every intermediate placed in a
+// file-scope static device array of LCSA_NOALLOC_WORKSPACE_BYTES, and the
+// configuration goes through the same checks as a plan's (resolve_config).
 //
-// The first call on a device looks up the array's device address there
-// (cudaGetSymbolAddress with that device current); make that first call
-// before any stream capture. All calls share the one array and it keeps the
-// last call's contents, so calls that overlap on the GPU (other streams, other
-// host threads) race; serialise them. The kernels overwrite every byte they
-// read except the error word, which each call clears first.
+// Set-up: the first call in a CUDA context looks up the array's device address
+// there (cudaGetSymbolAddress with that context current) and clears its error
+// word. Under CUDA's default lazy module loading that lookup is also what
+// loads this file's module, and loading it reserves the array on the device:
+// make the first call at start-up, before any stream capture (or load every
+// module at start-up with CUDA_MODULE_LOADING=EAGER). Later calls allocate
+// nothing. The address is cached per context (by its unique context ID), so a
+// context created later on the same device, for instance after
+// cudaDeviceReset, looks it up again.
+//
+// All calls share the one array and it keeps the last call's contents, so
+// calls that overlap on the GPU (other streams, other host threads) race;
+// serialise them. Each call clears the counters its kernels start from; the
+// kernels overwrite every other byte they read. The error word is not
+// cleared by a call: a kernel's timeout or bounds record stays until
+// lcsa_noalloc_check_device_error reads it.
 #include <cmath>
 #include <mutex>
 
@@ -29,184 +39,178 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_ws[LCSA_NOALLOC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
+// Layout of the array's first bytes: the error word (kept across calls),
+// then K1's merge counters and K3's work counter (cleared by every call).
+constexpr size_t kOffErr = 0;
+constexpr size_t kOffCnt = 256;
+constexpr size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+constexpr size_t kOffAfterCnt = kOffCnt + round256(size_t(lcsa::kCounters) * 4);
+
+// Workspace address per CUDA context, keyed by the context's unique ID
+// (cuCtxGetId; IDs are never reused within a process).
+constexpr int kMaxContexts = 64;
+struct WsEntry {
+  unsigned long long ctx_id;
+  unsigned char* addr;
+};
 std::mutex g_ws_mutex;
-void* g_ws_addr[kMaxDevices] = {};
+WsEntry g_ws[kMaxContexts] = {};
+int g_ws_n = 0;
 
-// Failures are reported by status code only: composing a message string could
-// allocate host memory, which this entry point never does.
-lcsa_status_t noalloc_fail(lcsa_status_t st, const char* /*why*/) { return st; }
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
 
-size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
-
-// k_eff of every (b, h, qb) row and the row offsets, from the geometry alone.
-__global__ void noalloc_row_ptr_kernel(int* row_ptr, lcsa::Grid g, int radius, int topk) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  const int groups = g.nKB / g.bpf;
-  int acc = 0;
-  const int rows = g.B * g.Hn * g.nQB;
-  for (int row = 0; row < rows; ++row) {
-    row_ptr[row] = acc;
-    const int rem = (row % g.nQB) % g.bpf;
-    const int hb = rem / g.nWb, wb = rem % g.nWb;
-    int nh = g.nHb, nw = g.nWb;
-    if (radius >= 0) {
-      nh = min(hb + radius, g.nHb - 1) - max(hb - radius, 0) + 1;
-      nw = min(wb + radius, g.nWb - 1) - max(wb - radius, 0) + 1;
-    }
-    const int a = groups * nh * nw;
-    acc += topk < a ? topk : a;
+// ID of the calling thread's current context (false if there is none).
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrent get_current = nullptr;
+  static CtxGetId get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return false;
+    get_current = reinterpret_cast<CtxGetCurrent>(f1);
+    get_id = reinterpret_cast<CtxGetId>(f2);
   }
-  row_ptr[rows] = acc;
+  CUcontext ctx = nullptr;
+  return get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, id) == CUDA_SUCCESS;
 }
 
-// Sizes of one problem, checked without touching the heap.
-struct NoallocGeom {
-  lcsa::Grid g;
-  int radius, topk, max_window;
-  int64_t rows, nnz;
-};
+// The array's address in the current context, looked up (and its error word
+// cleared on `s`) the first time. Caller holds g_ws_mutex. Null on failure.
+unsigned char* workspace_here(cudaStream_t s, bool set_up) {
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) return nullptr;
+  for (int i = 0; i < g_ws_n; ++i)
+    if (g_ws[i].ctx_id == id) return g_ws[i].addr;
+  if (!set_up || g_ws_n == kMaxContexts) return nullptr;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_ws) != cudaSuccess || !ptr) return nullptr;
+  if (cudaMemsetAsync(static_cast<unsigned char*>(ptr) + kOffErr, 0, kOffCnt - kOffErr, s) != cudaSuccess)
+    return nullptr;
+  g_ws[g_ws_n++] = WsEntry{id, static_cast<unsigned char*>(ptr)};
+  return static_cast<unsigned char*>(ptr);
+}
 
-lcsa_status_t noalloc_resolve(const lcsa_config_t* c, NoallocGeom* out) {
-  if (c->batch < 1 || c->heads < 1 || c->head_dim < 1 || c->q_frames < 1 || c->kv_frames < 1 || c->grid_h < 1 ||
-      c->grid_w < 1 || c->block_t < 1 || c->block_h < 1 || c->block_w < 1)
-    return noalloc_fail(LCSA_ERR_INVALID_ARG, "sizes must be >= 1");
-  if (c->local_range < 0 || (c->local_range != LCSA_UNBOUNDED && c->local_range % 2 == 0))
-    return noalloc_fail(LCSA_ERR_INVALID_ARG, "local_range must be odd or 0 (unbounded)");
-  if (c->topk < 0 || (c->topk == 0 && !(c->sparse_ratio > 0.f && std::isfinite(c->sparse_ratio))))
-    return noalloc_fail(LCSA_ERR_INVALID_ARG, "topk < 0, or topk = 0 without a finite sparse_ratio > 0");
-  if ((c->norm_scope != LCSA_NORM_TOKEN && c->norm_scope != LCSA_NORM_HEAD) || !(c->rms_eps > 0.f) ||
-      !std::isfinite(c->rms_eps) ||
-      !(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale) || c->kv_frame_offset < 0)
-    return noalloc_fail(LCSA_ERR_INVALID_ARG, "norm_scope, rms_eps, softmax_scale or kv_frame_offset out of range");
-  if (c->kv_frames < c->q_frames || c->grid_h % c->block_h || c->grid_w % c->block_w || c->q_frames % c->block_t ||
-      c->kv_frames % c->block_t)
-    return noalloc_fail(LCSA_ERR_SHAPE, "kv_frames < q_frames, or the token grid is not divisible by the block");
-  const int nb = c->block_t * c->block_h * c->block_w;
-  if (c->head_dim != lcsa::kHeadDim || c->heads > lcsa::kMaxHeads || (nb != 64 && nb != 128) ||
-      c->block_t * c->block_h > 8)
-    return noalloc_fail(LCSA_ERR_UNSUPPORTED, "head_dim, heads or block shape outside what the kernels implement");
-  // sizes bounded in floating point before any integer product (2^40
-  // elements per tensor at most: every block count below fits an int)
-  if (double(c->batch) * double(c->kv_frames) * double(c->grid_h) * double(c->grid_w) * double(c->heads) *
-          double(c->head_dim) > double(int64_t(1) << 40))
-    return noalloc_fail(LCSA_ERR_UNSUPPORTED, "tensor of more than 2^40 elements");
-  lcsa::Grid& g = out->g;
-  g.B = c->batch;
-  g.Hn = c->heads;
-  g.Tq = c->q_frames;
-  g.Tkv = c->kv_frames;
-  g.gh = c->grid_h;
-  g.gw = c->grid_w;
-  g.bt = c->block_t;
-  g.bh = c->block_h;
-  g.bw = c->block_w;
-  g.nb = nb;
-  g.nHb = c->grid_h / c->block_h;
-  g.nWb = c->grid_w / c->block_w;
-  g.bpf = g.nHb * g.nWb;
-  g.nQB = (c->q_frames / c->block_t) * g.bpf;
-  g.nKB = (c->kv_frames / c->block_t) * g.bpf;
-  g.Lq = int64_t(c->q_frames) * c->grid_h * c->grid_w;
-  g.Lkv = int64_t(c->kv_frames) * c->grid_h * c->grid_w;
-  g.C = c->heads * c->head_dim;
-  // budget: topk_ratio = sparse_ratio*768*1280/(H*W), H = 16 grid_h, W = 16 grid_w,
-  // times the blocks of one latent frame
-  int topk = c->topk;
-  if (topk == 0) {
-    const double k = std::floor(double(c->sparse_ratio) * 983040.0 * double(g.bpf) /
-                                ((16.0 * c->grid_h) * (16.0 * c->grid_w)));
-    topk = k >= double(1 << 30) ? (1 << 30) : int(k);  // beyond 2^30: every admissible block
-  }
-  if (topk < 1) return noalloc_fail(LCSA_ERR_INVALID_ARG, "sparse_ratio gives a budget of 0 blocks");
-  out->topk = topk;
-  out->radius = c->local_range == LCSA_UNBOUNDED ? -1 : (c->local_range - 1) / 2;
-  const int groups = g.nKB / g.bpf;
-  int wmax = 0;
-  int64_t per_head = 0;
-  for (int qb = 0; qb < g.nQB; ++qb) {
-    const int rem = qb % g.bpf, hb = rem / g.nWb, wb = rem % g.nWb;
-    int nh = g.nHb, nw = g.nWb;
-    if (out->radius >= 0) {
-      const int r = out->radius;
-      nh = (hb + r < g.nHb - 1 ? hb + r : g.nHb - 1) - (hb - r > 0 ? hb - r : 0) + 1;
-      nw = (wb + r < g.nWb - 1 ? wb + r : g.nWb - 1) - (wb - r > 0 ? wb - r : 0) + 1;
+// CSR row offsets from the geometry alone. A query block's kept count
+// depends only on its place in its frame, so the block first scans the kept
+// counts of one frame's places into pre[0..bpf] (1024 at a time, warp scans
+// and a carry), then writes row (bh, qb) = bh * per_head + (qb / bpf) *
+// per_frame + pre[qb % bpf].
+__global__ void __launch_bounds__(1024) noalloc_row_ptr_kernel(int* row_ptr, int* pre, lcsa::ConfigCore r) {
+  __shared__ int warp_incl[32];
+  __shared__ int carry;
+  const lcsa::Grid& g = r.grid;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < g.bpf; base += 1024) {
+    const int place = base + tid;
+    int v = 0;
+    if (place < g.bpf) {
+      const int hb = place / g.nWb, wb = place % g.nWb;
+      int nh = g.nHb, nw = g.nWb;
+      if (r.radius >= 0) {
+        nh = min(hb + r.radius, g.nHb - 1) - max(hb - r.radius, 0) + 1;
+        nw = min(wb + r.radius, g.nWb - 1) - max(wb - r.radius, 0) + 1;
+      }
+      const int a = (g.nKB / g.bpf) * nh * nw;
+      v = r.topk < a ? r.topk : a;
     }
-    const int a = groups * nh * nw;
-    wmax = a > wmax ? a : wmax;
-    per_head += topk < a ? topk : a;
+    int x = v;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_incl[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = warp_incl[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      warp_incl[lane] = t;
+    }
+    __syncthreads();
+    const int excl = carry + (w > 0 ? warp_incl[w - 1] : 0) + x - v;
+    if (place < g.bpf) pre[place] = excl;
+    __syncthreads();  // every thread has read carry
+    if (tid == 1023) carry = excl + v;
+    __syncthreads();
   }
-  if (wmax > lcsa::kMaxCandidates) return noalloc_fail(LCSA_ERR_UNSUPPORTED, "window holds too many blocks");
-  out->max_window = wmax;
-  out->rows = int64_t(g.B) * g.Hn * g.nQB;
-  out->nnz = per_head * g.B * g.Hn;
-  return LCSA_OK;
+  const int per_frame = carry;
+  const int64_t per_head = int64_t(per_frame) * (g.nQB / g.bpf);
+  const int rows = g.B * g.Hn * g.nQB;
+  for (int row = tid; row < rows; row += 1024) {
+    const int bh = row / g.nQB, qb = row % g.nQB;
+    row_ptr[row] = int(bh * per_head + int64_t(qb / g.bpf) * per_frame + pre[qb % g.bpf]);
+  }
+  if (tid == 0) row_ptr[rows] = int(int64_t(g.B) * g.Hn * per_head);
 }
 
 }  // namespace
 
 extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const void* q, const void* k, const void* v,
                                               const float* gamma_q, const float* gamma_k, void* out, void* stream) {
-  if (!cfg) return noalloc_fail(LCSA_ERR_INVALID_ARG, "config is null");
-  if (cfg->host_io) return noalloc_fail(LCSA_ERR_INVALID_ARG, "host_io needs staging buffers; use a plan");
+  // Failures are reported by status code only: composing a message string
+  // could allocate host memory, which this entry point never does.
+  if (!cfg) return LCSA_ERR_INVALID_ARG;
+  if (cfg->host_io) return LCSA_ERR_INVALID_ARG;  // host buffers need staging: use a plan
   if (cfg->heads_total != 0 && cfg->heads_total != cfg->heads)
-    return noalloc_fail(LCSA_ERR_UNSUPPORTED, "head-sharded layers need a plan (lcsa_forward_sharded)");
-  NoallocGeom ng;
-  lcsa_status_t st = noalloc_resolve(cfg, &ng);
+    return LCSA_ERR_UNSUPPORTED;  // head-sharded layers need a plan (lcsa_forward_sharded)
+  lcsa::ConfigCore core;
+  lcsa_status_t st = lcsa::resolve_config(cfg, &core, nullptr, 0);
   if (st != LCSA_OK) return st;
-  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return noalloc_fail(LCSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return LCSA_ERR_INVALID_ARG;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out) |
                         reinterpret_cast<uintptr_t>(gamma_q) | reinterpret_cast<uintptr_t>(gamma_k);
-  if (mis & 15u) return noalloc_fail(LCSA_ERR_ALIGNMENT, "tensor pointers must be 16-byte aligned");
-  const lcsa::Grid& g = ng.g;
-  const int radius = ng.radius;
+  if (mis & 15u) return LCSA_ERR_ALIGNMENT;
+  const lcsa::Grid& g = core.grid;
   const int D = cfg->head_dim;
 
   // carve the static workspace
   const lcsa::RopeSplit rs = lcsa::rope_split(D);
   const size_t rope_n = size_t(g.Tkv) * rs.pairs_t + size_t(g.gh) * rs.pairs_h + size_t(g.gw) * rs.pairs_w;
-  const size_t off_err = 0;
-  const size_t off_cnt = off_err + 256;  // K1 split counters, cleared together with the error word
-  const size_t off_sp = off_cnt + round256(size_t(lcsa::kCounters) * 4);
+  const size_t off_sp = kOffAfterCnt;
   const size_t off_rope = off_sp + round256(size_t(lcsa::kMaxK1Ctas) * 2 * g.C * 4);
-  const size_t off_rp = off_rope + round256(rope_n * sizeof(float2));
-  const size_t off_ci = off_rp + round256((size_t(ng.rows) + 1) * 4);
-  const size_t off_pq = off_ci + round256(size_t(ng.nnz) * 4);
+  const size_t off_pre = off_rope + round256(rope_n * sizeof(float2));
+  const size_t off_rp = off_pre + round256((size_t(g.bpf) + 1) * 4);
+  const size_t off_ci = off_rp + round256((size_t(core.rows) + 1) * 4);
+  const size_t off_pq = off_ci + round256(size_t(core.nnz) * 4);
   const size_t off_pk = off_pq + round256(size_t(g.B) * g.Hn * g.nQB * D * 4);
   const size_t off_qh = off_pk + round256(size_t(g.B) * g.Hn * g.nKB * D * 4);
   const size_t off_kh = off_qh + round256(size_t(g.B) * g.Lq * g.C * 2);
   // 64-token blocks: query-block pairs as 128-row tiles (union lists and counts)
   const int64_t npairs = g.nb == 64 ? lcsa::pair_count(g) : 0;
-  const int pair_cap = 2 * ng.max_window < g.nKB ? 2 * ng.max_window : g.nKB;
+  const int pair_cap = 2 * core.max_window < g.nKB ? 2 * core.max_window : g.nKB;
   const size_t off_pc = off_kh + round256(size_t(g.B) * g.Lkv * g.C * 2);
   const size_t off_pl = off_pc + round256(size_t(npairs) * size_t(pair_cap) * 4);
   const size_t need = off_pl + round256(size_t(npairs) * 4);
-  if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES))
-    return noalloc_fail(LCSA_ERR_UNSUPPORTED,
-                        "problem needs more workspace than the static array holds (LCSA_NOALLOC_WORKSPACE_BYTES); "
-                        "create a plan instead");
+  if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES)) return LCSA_ERR_UNSUPPORTED;  // create a plan instead
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return noalloc_fail(LCSA_ERR_UNSUPPORTED, "device index out of range");
+  if (e != cudaSuccess) return LCSA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_ws_mutex);
-    if (!g_ws_addr[dev]) {
-      void* ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, g_noalloc_ws);
-      if (e != cudaSuccess || !ptr) return noalloc_fail(LCSA_ERR_CUDA, "cudaGetSymbolAddress of the static workspace");
-      g_ws_addr[dev] = ptr;
-    }
-    ws = static_cast<unsigned char*>(g_ws_addr[dev]);
+    ws = workspace_here(s, true);
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  unsigned* err = reinterpret_cast<unsigned*>(ws + off_err);
-  unsigned* split_cnt = reinterpret_cast<unsigned*>(ws + off_cnt);
+  if (!ws) return LCSA_ERR_CUDA;
+  unsigned* err = reinterpret_cast<unsigned*>(ws + kOffErr);
+  unsigned* split_cnt = reinterpret_cast<unsigned*>(ws + kOffCnt);
   float* split_part = reinterpret_cast<float*>(ws + off_sp);
   float2* rope = reinterpret_cast<float2*>(ws + off_rope);
+  int* pre = reinterpret_cast<int*>(ws + off_pre);
   int* row_ptr = reinterpret_cast<int*>(ws + off_rp);
   int* col_idx = reinterpret_cast<int*>(ws + off_ci);
   float* pooled_q = reinterpret_cast<float*>(ws + off_pq);
@@ -216,15 +220,15 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   int* pair_col = npairs ? reinterpret_cast<int*>(ws + off_pc) : nullptr;
   int* pair_len = npairs ? reinterpret_cast<int*>(ws + off_pl) : nullptr;
 
-  if ((e = cudaMemsetAsync(err, 0, off_sp - off_err, s)) != cudaSuccess)
-    return noalloc_fail(LCSA_ERR_CUDA, "clear error word and counters");
+  // the counters start at zero (an aborted call may have left them set)
+  if ((e = cudaMemsetAsync(split_cnt, 0, kOffAfterCnt - kOffCnt, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   {
     LCSA_RANGE("lcsa rope table");
     if ((e = lcsa::launch_rope_table(rope, g.Tkv, g.gh, g.gw, cfg->kv_frame_offset, D, s)) != cudaSuccess)
-      return noalloc_fail(LCSA_ERR_CUDA, "rope table launch");
+      return LCSA_ERR_CUDA;
   }
-  noalloc_row_ptr_kernel<<<1, 32, 0, s>>>(row_ptr, g, radius, ng.topk);
-  if ((e = cudaGetLastError()) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "row offsets launch");
+  noalloc_row_ptr_kernel<<<1, 1024, 0, s>>>(row_ptr, pre, core);
+  if ((e = cudaGetLastError()) != cudaSuccess) return LCSA_ERR_CUDA;
 
   lcsa::K1Params k1{};  // every field zero (null) unless set below
   k1.g = g;
@@ -248,23 +252,21 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.norm_inv_c = 1.0f / float(g.C);
   lcsa::k1_all_blocks(k1);
   if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return noalloc_fail(LCSA_ERR_CUDA, "device attributes");
+    return LCSA_ERR_CUDA;
   {
     LCSA_RANGE("lcsa K1 prologue");
-    if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "prologue launch");
+    if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
 
-  int sort_n = 32;
-  while (sort_n < ng.max_window) sort_n <<= 1;
   lcsa::K2Params k2{};  // every field zero (null) unless set below
   k2.g = g;
   k2.pooled_q = pooled_q;
   k2.pooled_k = pooled_k;
   k2.row_ptr = row_ptr;
   k2.col_idx = col_idx;
-  k2.radius = radius;
-  k2.topk = ng.topk;
-  k2.sort_n = sort_n;
+  k2.radius = core.radius;
+  k2.topk = core.topk;
+  k2.sort_n = core.sort_n;
   k2.clear_cnt = split_cnt;
   k2.n_clear = lcsa::kCounters;
   k2.ring_fb = g.Tkv / g.bt;
@@ -276,7 +278,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k2.pad_cap = 0;
   {
     LCSA_RANGE("lcsa K2 select");
-    if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "select launch");
+    if ((e = lcsa::launch_select(k2, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
   if (npairs) {
     LCSA_RANGE("lcsa pair union");
@@ -289,10 +291,9 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
     pp.pair_col = pair_col;
     pp.pair_len = pair_len;
     pp.pair_cap = pair_cap;
-    if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return noalloc_fail(LCSA_ERR_CUDA, "pair union launch");
+    if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
 
-  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : float(1.0 / std::sqrt(double(D)));
   lcsa::K3Params k3{};  // every field zero (null) unless set below
   k3.g = g;
   k3.qhat = qhat;
@@ -301,7 +302,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.out = static_cast<__nv_bfloat16*>(out);
   k3.row_ptr = row_ptr;
   k3.col_idx = col_idx;
-  k3.scale_log2 = scale * 1.4426950408889634f;
+  k3.scale_log2 = core.scale * 1.4426950408889634f;
   k3.err = err;
   k3.ring_fb = g.Tkv / g.bt;
   k3.slot0_fb = 0;
@@ -319,9 +320,24 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
     if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||
         (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb)) != cudaSuccess ||
         (e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess)
-      return noalloc_fail(LCSA_ERR_CUDA, "tensor maps");
-    if ((e = lcsa::launch_attention_tc(k3, tm_q, tm_k, tm_v, num_sms, s)) != cudaSuccess)
-      return noalloc_fail(LCSA_ERR_CUDA, "attention launch");
+      return LCSA_ERR_CUDA;
+    if ((e = lcsa::launch_attention_tc(k3, tm_q, tm_k, tm_v, num_sms, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
   return LCSA_OK;
+}
+
+extern "C" lcsa_status_t lcsa_noalloc_check_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    ws = workspace_here(s, false);
+  }
+  if (!ws) return LCSA_OK;  // no call has run in this context
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LCSA_ERR_CUDA;
+  unsigned word[4] = {0, 0, 0, 0};  // host stack: no allocation
+  if (cudaMemcpy(word, ws + kOffErr, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return LCSA_ERR_CUDA;
+  if (word[0] == lcsa::kDevErrNone) return LCSA_OK;
+  if (cudaMemset(ws + kOffErr, 0, sizeof(word)) != cudaSuccess) return LCSA_ERR_CUDA;
+  return word[0] == lcsa::kDevErrTimeout ? LCSA_ERR_DEVICE_TIMEOUT : LCSA_ERR_DEVICE_BOUNDS;
 }

@@ -164,7 +164,9 @@ LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void*
 /* Same call from HOST buffers: copies q, k, v and the gains into plan-owned
    device staging, runs lcsa_forward and copies out back, all on `stream`.
    Needs a plan created with host_io = 1. Host buffers should be pinned for
-   asynchronous copies; the call returns once `out` holds the result. */
+   asynchronous copies; the call returns once `out` holds the result, after
+   reading the plan's device error word as lcsa_check_device_error does
+   (LCSA_ERR_DEVICE_TIMEOUT / LCSA_ERR_DEVICE_BOUNDS: `out` is not valid). */
 LCSA_API lcsa_status_t lcsa_forward_host(lcsa_plan_t plan, const void* q, const void* k, const void* v,
                                 const float* gamma_q, const float* gamma_k, void* out, void* stream);
 
@@ -232,7 +234,8 @@ LCSA_API lcsa_status_t lcsa_plan_set_threshold_reuse(lcsa_plan_t plan, int on);
 LCSA_API lcsa_status_t lcsa_selection_nnz(lcsa_plan_t plan, int64_t* nnz);
 
 /* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
-   Every GPU that loads the library holds this array until the process exits. */
+   A GPU holds this array from the first lcsa_forward_noalloc call made on it
+   (when the CUDA module that holds it is loaded) until the process exits. */
 #define LCSA_NOALLOC_WORKSPACE_BYTES (32u << 20)
 
 /* The LCSA call without a plan and without any allocation, for callers that
@@ -241,18 +244,37 @@ LCSA_API lcsa_status_t lcsa_selection_nnz(lcsa_plan_t plan, int64_t* nnz);
    where cudaMalloc/cudaFree would synchronise the device and stall the other
    streams, or could fail). This entry point has no counterpart in the paper.
    Arguments are those of lcsa_forward, with the configuration passed directly
-   (host_io must be 0). All intermediates live in one file-scope static device
-   array of LCSA_NOALLOC_WORKSPACE_BYTES; the first call on a device looks up
-   that array's address on the current device, so make the first call before
-   any stream capture. All calls share the array and it keeps the last call's
-   contents: calls that overlap on the GPU race and must be serialised by the
-   caller. Returns LCSA_ERR_UNSUPPORTED when the problem's intermediates do not
-   fit in the array (create a plan instead), and the codes of
-   lcsa_config_resolve for a bad configuration; no detail message is set. No
-   device or host memory is allocated and no allocating library routine is
-   called. Asynchronous on `stream`. */
+   (host_io must be 0; the checks are lcsa_config_resolve's, shared code).
+   All intermediates live in one file-scope static device array of
+   LCSA_NOALLOC_WORKSPACE_BYTES.
+   Set-up: the first call in a CUDA context looks up that array's address in
+   that context and clears its error word. Under CUDA's default lazy module
+   loading this first call also loads the module that holds the array, which
+   reserves its device memory: make it at start-up, before any stream capture
+   (or set CUDA_MODULE_LOADING=EAGER so every module loads with the context).
+   Later calls allocate nothing. Addresses are kept per context (by its
+   unique ID), so a new context on the same device (after cudaDeviceReset,
+   say) repeats the set-up.
+   All calls share the array and it keeps the last call's contents: calls that
+   overlap on the GPU race and must be serialised by the caller. Returns
+   LCSA_ERR_UNSUPPORTED when the problem's intermediates do not fit in the
+   array (create a plan instead), and the codes of lcsa_config_resolve for a
+   bad configuration; no detail message is set. No device or host memory is
+   allocated and no allocating library routine is called. Asynchronous on
+   `stream`. A kernel's bounded-wait timeout or index-check failure is kept in
+   the array's error word (calls do not clear it) until
+   lcsa_noalloc_check_device_error reads it. */
 LCSA_API lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const void* q, const void* k, const void* v,
                                             const float* gamma_q, const float* gamma_k, void* out, void* stream);
+
+/* Device-error status of the lcsa_forward_noalloc calls made in the current
+   context since the last check: synchronises `stream`, reads the static
+   array's error word into host stack memory and clears it. Returns LCSA_OK,
+   LCSA_ERR_DEVICE_TIMEOUT (a kernel gave up a bounded wait; that call's output
+   is incomplete), LCSA_ERR_DEVICE_BOUNDS, or LCSA_ERR_CUDA (the stream or the
+   copy failed). LCSA_OK too when no call has run in this context. Allocates
+   nothing. No counterpart in the paper, like lcsa_forward_noalloc. */
+LCSA_API lcsa_status_t lcsa_noalloc_check_device_error(void* stream);
 
 /* Resolved geometry of a plan. */
 LCSA_API lcsa_status_t lcsa_plan_geometry(lcsa_plan_t plan, lcsa_geometry_t* out);

@@ -203,6 +203,37 @@ def test_noalloc_entry_point_rejects_before_touching_a_device():
         L.LCSA_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("value", ["alloc", "alloc:0", "alloc:x", "launch:K9", "launch:", "oom", "copy:1"])
+def test_a_malformed_fault_injection_value_is_refused(value, monkeypatch):
+    """LCSA_FAULT is read before any device call, so a misspelt injection is
+    refused (never silently ignored), with or without a GPU."""
+    monkeypatch.setenv("LCSA_FAULT", value)
+    cfg = _cfg()
+    for create in (L.lib().lcsa_plan_create, L.lib().lcsa_plan_create_stream):
+        h = ctypes.c_void_p()
+        assert create(ctypes.byref(cfg), 0, ctypes.byref(h)) == L.LCSA_ERR_INVALID_ARG
+        assert "LCSA_FAULT" in L.lcsa_last_error_message()
+        assert h.value is None
+
+
+@pytest.mark.parametrize("value", ["alloc:3", "launch:K1", "launch:K2", "launch:PAIR", "launch:K3", "launch:ROPE",
+                                   "copy"])
+def test_well_formed_fault_injection_values_pass_the_parser(value, monkeypatch):
+    monkeypatch.setenv("LCSA_FAULT", value)
+    cfg = _cfg()
+    h = ctypes.c_void_p()
+    st = L.lib().lcsa_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h))
+    # no GPU here: the plan fails at the device (or, on a GPU, at the injected allocation)
+    assert st in (L.LCSA_ERR_CUDA, L.LCSA_ERR_OOM, L.LCSA_OK), st
+    assert "not understood" not in L.lcsa_last_error_message()
+    if st == L.LCSA_OK:
+        L.lib().lcsa_plan_destroy(h)
+
+
+def test_noalloc_status_call_without_any_call_is_clean():
+    assert L.lcsa_noalloc_check_device_error(0) == L.LCSA_OK
+
+
 def test_nvtx_ranges_compile(tmp_path):
     """The optional NVTX ranges (build --nvtx) compile in both entry-point
     files; the objects go to a temporary directory, the in-tree library is

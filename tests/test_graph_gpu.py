@@ -1,15 +1,18 @@
 """Several lcsa_forward calls captured in one CUDA graph (the 30 attention
 calls of a DiT chunk share one geometry) replay bit-identically to the same
-calls made eagerly. lcsa_forward does no host synchronisation and no
-allocation, so it can be captured; the plan is not re-entrant, so the calls
-of one plan are ordered on one stream inside the graph."""
+calls made eagerly, and each replayed output matches the fp64 oracle of its
+own inputs within the parity tolerance. lcsa_forward does no host
+synchronisation and no allocation, so it can be captured; the plan is not
+re-entrant, so the calls of one plan are ordered on one stream inside the
+graph."""
 import numpy as np
 import pytest
 
 import block_sparse_video_lcsa_b200 as L
+import oracle
 from block_sparse_video_lcsa_b200 import synth
 
-from lcsa_harness import torch_inputs
+from lcsa_harness import OUT_MAX_ABS, OUT_MEAN_ABS, block_rows_to_raster, torch_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +30,8 @@ LAYERS = 3
 def test_graph_replay_equals_eager_calls(name):
     import torch
     wl = WL[name]
-    layers = [torch_inputs(synth.make_inputs(wl.replace(seed=10 + i))) for i in range(LAYERS)]
+    host = [synth.make_inputs(wl.replace(seed=10 + i)) for i in range(LAYERS)]
+    layers = [torch_inputs(inp) for inp in host]
     plan = L.lcsa_plan_create(L.config_from_workload(wl), 0)
     try:
         eager = []
@@ -50,6 +54,15 @@ def test_graph_replay_equals_eager_calls(name):
         plan.lcsa_check_device_error()
         for a, b in zip(eager, outs):
             np.testing.assert_array_equal(a.view(torch.int16).cpu().numpy(), b.view(torch.int16).cpu().numpy())
+        # each replayed layer against the oracle of its own inputs
+        og = oracle.Geometry.from_workload(wl)
+        D = og.head_dim
+        for inp, out in zip(host, outs):
+            _, _, _, ref, _ = oracle.run(og, inp)
+            got = synth.bf16_bits_to_f64(out.view(torch.int16).cpu().numpy().view(np.uint16))
+            err = np.concatenate([np.abs(got[b, tok, h * D:(h + 1) * D] - ref[n, i])
+                                  for b, tok, h, n, i in block_rows_to_raster(og, np.arange(og.rows), ref)])
+            assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (err.max(), err.mean())
         del graph
     finally:
         plan.destroy()

@@ -1,5 +1,6 @@
-"""Pins of the parameter contract against values the pages print
-(tests/golden/lcsa_parameters.txt), and of the block budget reading."""
+"""Pins of the parameter contract against the pages
+(tests/golden/lcsa_parameters.txt: the printed topk_ratio formula evaluated at
+four sizes, and the printed latent geometry), and of the block budget reading."""
 import os
 
 import pytest

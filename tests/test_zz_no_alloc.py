@@ -3,17 +3,21 @@ device memory while they run (for example a real-time video pipeline or a
 plugin whose device memory is reserved at start-up: a cudaMalloc there would
 synchronise the device and stall the other streams, or fail outright).
 
-It must give the plan path's result, within the parity tolerance, on two
-calls in a row with different inputs (the shared static workspace keeps the
-previous call's contents). This file is collected last on purpose.
+It runs the plan path's kernels on the same inputs, so its output must equal
+the plan path's bit for bit, on two calls in a row with different inputs (the
+shared static workspace keeps the previous call's contents); one case is also
+compared with the fp64 oracle at the parity tolerance, and the static
+workspace's error word must read clean afterwards. This file is collected
+last on purpose.
 """
 import numpy as np
 import pytest
 
 import block_sparse_video_lcsa_b200 as L
+import oracle
 from block_sparse_video_lcsa_b200 import synth
 
-from lcsa_harness import OUT_MAX_ABS, OUT_MEAN_ABS, torch_inputs
+from lcsa_harness import OUT_MAX_ABS, OUT_MEAN_ABS, block_rows_to_raster, torch_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +37,7 @@ def _plan_output(wl, inp):
         out = torch.empty_like(q)
         plan.lcsa_forward(q, k, v, gq, gk, out)
         plan.lcsa_check_device_error()
-        return out.float().cpu().numpy()
+        return out.view(torch.int16).cpu().numpy()
     finally:
         plan.destroy()
 
@@ -49,12 +53,19 @@ def test_noalloc_matches_the_plan_path_on_two_calls_in_a_row(name):
     outs = [torch.full_like(t[0], float("nan")) for t in tensors]
     for (q, k, v, gq, gk), out in zip(tensors, outs):          # back to back on one stream
         assert L.lcsa_forward_noalloc(cfg, q, k, v, gq, gk, out) == L.LCSA_OK
-    torch.cuda.synchronize()
-    for out, ref in zip(outs, want):
-        got = out.float().cpu().numpy()
-        assert np.all(np.isfinite(got))
-        diff = np.abs(got - ref)
-        assert diff.max() <= OUT_MAX_ABS and diff.mean() <= OUT_MEAN_ABS, (diff.max(), diff.mean())
+    assert L.lcsa_noalloc_check_device_error() == L.LCSA_OK
+    for call, (out, ref) in enumerate(zip(outs, want)):
+        got = out.view(torch.int16).cpu().numpy()
+        diff = int(np.count_nonzero(got != ref))
+        assert diff == 0, "call %d: %d output elements differ from the plan path" % (call, diff)
+    # the second call against the fp64 oracle as well (parity tolerance)
+    og = oracle.Geometry.from_workload(wl)
+    _, _, _, ref, _ = oracle.run(og, loads[1])
+    got = synth.bf16_bits_to_f64(outs[1].view(torch.int16).cpu().numpy().view(np.uint16))
+    D = og.head_dim
+    err = np.concatenate([np.abs(got[b, tok, h * D:(h + 1) * D] - ref[n, i])
+                          for b, tok, h, n, i in block_rows_to_raster(og, np.arange(og.rows), ref)])
+    assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (err.max(), err.mean())
 
 
 def test_noalloc_rejects_problems_larger_than_its_workspace():
@@ -63,3 +74,4 @@ def test_noalloc_rejects_problems_larger_than_its_workspace():
     x = torch.empty(16, dtype=torch.bfloat16, device="cuda:0")
     g = torch.ones(16, dtype=torch.float32, device="cuda:0")
     assert L.lcsa_forward_noalloc(cfg, x, x, x, g, g, x) == L.LCSA_ERR_UNSUPPORTED
+    assert L.lcsa_noalloc_check_device_error() == L.LCSA_OK
