@@ -29,29 +29,33 @@
 //           of three TMEM S buffers, running up to three KV blocks ahead of
 //           the softmax; also owns the TMEM allocation.
 //   warp 2  P.V issuer: O += P V with P read from TMEM.
-//           Each issuer is a converged warp (every lane waits, lane 0
-//           issues), so each feeds the tensor pipe one kind of product: a
-//           single thread that alternates the two kinds with barrier waits in
-//           between was measured to issue at half the pipe's rate. The two
-//           streams are ordered only through mbarriers: S of block j+3 waits
-//           until P.V of block j (which reads P_j from the same buffer) has
-//           completed.
-//   warps 3-10 softmax, two warpgroups: a query row (TMEM lane) is shared by
-//           lane i of warp w and of warp w+4, each owning 64 of its 128 key
-//           columns. The pair trades row maxima (and at the end row sums)
-//           through shared memory, ordered by an mbarrier of 64 arrivals. Online
-//           softmax in the exp2 domain (scale folded into log2 e), P written
-//           to TMEM as bf16 pairs, O rescaled only when the running max grew
-//           by more than 2^8 (exact: O and the row sum use the same stale
-//           max); only a rescale waits for the preceding P.V, so the softmax
-//           of block j overlaps P.V of block j-1. Finally each thread
-//           normalises and stores 64 of the row's output channels.
-//           Independent accumulators break the max and sum chains, and every
-//           fourth exponential runs on the FMA pipe (Cody-Waite reduction
-//           2^x = 2^n 2^f, |f| <= 1/2, and a degree-3 minimax polynomial for
-//           2^f fitted for this kernel, relative error below 7.5e-5) so the
-//           MUFU unit is not the bottleneck (the pages' "FFMA-form softmax
-//           math").
+//           Each issuer is a converged warp (every lane waits, one lane
+//           chosen by elect.sync issues), so each feeds the tensor pipe one
+//           kind of product: a single thread that alternates the two kinds
+//           with barrier waits in between was measured to issue at half the
+//           pipe's rate, and issuing from an elected lane instead of a lane-0
+//           branch measured 1.5-3.5 % faster. The two streams are ordered
+//           only through mbarriers: S of block j+3 waits until P.V of block
+//           j (which reads P_j from the same buffer) has completed.
+//   warps 3-10 softmax, two groups of four (one warp per TMEM lane quarter):
+//           the KV tiles of the CTA's work go to the groups in turn, and a
+//           group's warp handles all 128 keys of its quarter's 32 rows, so
+//           the two warps of a sub-partition work on different tiles at
+//           different times. The row's running maximum passes from tile to
+//           tile through a slot and an mbarrier per tile parity; a tile's
+//           maximum is published before its exponentials are computed, and
+//           it is raised only when the block maximum exceeds it by more than
+//           2^8 (exact: O and the row sums use the same stale maximum), so
+//           only such a tile waits for the preceding P.V to rescale O. Each
+//           group keeps its own partial row sum; the two are added once at
+//           the end of the row. Online softmax in the exp2 domain (scale
+//           folded into log2 e), P written to TMEM as bf16 pairs; finally each
+//           thread normalises and stores 64 of its row's output channels.
+//           Every fourth exponential runs on the FMA pipe (Cody-Waite
+//           reduction 2^x = 2^n 2^f, |f| <= 1/2, and a degree-3 minimax
+//           polynomial for 2^f fitted for this kernel, relative error below
+//           7.5e-5) so the MUFU unit is not the bottleneck (the pages'
+//           "FFMA-form softmax math").
 // TMEM columns: S ring [0,128) [128,256) [256,384), O [384,512). P of block j
 // is written back into S buffer j % 3 (bf16 pairs; keys 0-63 in its columns
 // 0-31, keys 64-127 in columns 64-95, each half inside the columns its own
@@ -98,7 +102,7 @@ constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffXchg = kOffBar + 512;          // row max / sum exchange
 constexpr int kItemSlots = 4;  // work items handed from the producer to the other roles
 constexpr int kItemReaders = 2 + kSoftmaxWarps;  // S issuer, P.V issuer, softmax warps (one arrival each)
-constexpr uint32_t kXchgBytes = (2 * 2 * 128 + 2 * 128) * 4;
+constexpr uint32_t kXchgBytes = (2 * 128 + 2 * 2 * 128) * 4;
 constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
 
 // 2^f on [-1/2, 1/2]: degree-3 minimax coefficients (relative error 7.49e-5),
@@ -115,7 +119,8 @@ struct Bars {
   uint64_t s_full[kSBufs], p_full[kSBufs], s_free[kSBufs];
   uint64_t o_done[2];  // o_done[g & 1]: P.V number g (counted per CTA) and all before it have completed
   uint64_t o_free, mma_drain[2];
-  uint64_t pair[4];  // row max / sum exchange between the two softmax warps of a lane quarter
+  uint64_t pair[4];  // end-of-row sum exchange between the two softmax warps of a lane quarter
+  uint64_t dec[4][2];  // maximum in use after a tile published, per lane quarter and tile parity
   // dynamic work distribution: the producer takes the next work item from
   // the global counter and hands it to the other roles through item[]
   uint64_t item_full[kItemSlots], item_empty[kItemSlots];
@@ -242,6 +247,11 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -291,6 +301,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
       : LCSA_R32(r)
       : "r"(taddr));
+}
+// tmem_ld32 that cannot be issued before `after` is computed (an unused asm input)
+__device__ __forceinline__ void tmem_ld32_after(uint32_t taddr, uint32_t (&r)[32], float after) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : LCSA_R32(r)
+      : "r"(taddr), "f"(after));
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -417,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(bars->s_full[s]), 1);
-      mbar_init(bar(bars->p_full[s]), kSoftmaxWarps);
+      mbar_init(bar(bars->p_full[s]), kSoftmaxWarps / 2);
       mbar_init(bar(bars->s_free[s]), 1);
     }
     mbar_init(bar(bars->o_done[0]), 1);
@@ -426,7 +444,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(bars->mma_drain[0]), 1);
     mbar_init(bar(bars->mma_drain[1]), 1);
     mbar_init(bar(bars->never), 1);
-    for (int s = 0; s < 4; ++s) mbar_init(bar(bars->pair[s]), 64);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar(bars->pair[s]), 64);
+      mbar_init(bar(bars->dec[s][0]), 32);
+      mbar_init(bar(bars->dec[s][1]), 32);
+    }
     for (int s = 0; s < kItemSlots; ++s) {
       mbar_init(bar(bars->item_full[s]), 1);
       mbar_init(bar(bars->item_empty[s]), kItemReaders);
@@ -604,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         if (!(ok = warp_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
           const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
@@ -623,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       kv += n;
     }
     if (issued) {
-      if (lane == 0) mma_commit(bar(bars->mma_drain[0]));
+      if (elect_one()) mma_commit(bar(bars->mma_drain[0]));
       __syncwarp();
       mbar_drain(bar(bars->mma_drain[0]), 0);
     }
@@ -644,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j == 0 && row_it > 0 && !(ok = warp_wait(bar(bars->o_free), (row_it - 1) & 1, abort, p.err, 15)))
           break;
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
           const uint32_t va = base + kOffV + vs * kTileBytes;
           const uint32_t pa = tmem + kColS + pb * 128;
 #pragma unroll
@@ -665,36 +687,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       kv += n;
     }
     if (issued) {
-      if (lane == 0) mma_commit(bar(bars->mma_drain[1]));
+      if (elect_one()) mma_commit(bar(bars->mma_drain[1]));
       __syncwarp();
       mbar_drain(bar(bars->mma_drain[1]), 0);
     }
   } else {
-    // ---------------- softmax / correction / epilogue, 128-token tiles ----------------
+    // ---------------- softmax / correction / epilogue ----------------
+    // The KV tiles of the CTA's work are numbered s = 0, 1, ... in order; tile
+    // s goes to group s & 1 (warps 3-6 or 7-10), whose warp for TMEM lane
+    // quarter sp handles all 128 keys of that quarter's 32 rows. The two
+    // warps of a sub-partition thus work on different tiles at different
+    // times, so one's exponentials overlap the other's other work. The row's
+    // running maximum passes from tile to tile: the warp of tile s waits for
+    // the maximum in use after tile s - 1 (a slot and an mbarrier per tile
+    // parity), takes the block maximum, decides the maximum in use after
+    // tile s (raised only if the block's exceeds it by more than 2^8: O and
+    // the row sums then use the same stale maximum exactly), publishes it, and
+    // only then computes the exponentials. Each group keeps its own partial
+    // row sum, brought to the current maximum when it next works on the row,
+    // and the two are added once at the end of the row.
     const int sp = warp & 3;                 // TMEM lane quarter of this warp
-    const int half = (warp - 3) >> 2;        // which 64 key columns / channels
+    const int grp = (warp - 3) >> 2;         // which tiles (s & 1) and, at the end, which 64 channels
     const int row_in_tile = sp * 32 + lane;  // query token of this lane's row
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
-    float* xmax = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 parity][2 half][128]
-    float* xsum = xmax + 2 * 2 * 128;                          // [2 half][128]
+    float* xdec = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 tile parity][128] maximum in use
+    float* xsum = xdec + 2 * 128;                              // [2 row parity][2 group][128]
     const float c = p.scale_log2;
     int s_it = 0, xk = 0;
     bool ok = true;
+    // the maximum in use after tile s has been published
+    auto wait_dec = [&](int s) { return warp_wait(bar(bars->dec[sp][s & 1]), (s >> 1) & 1, abort, p.err, 26); };
     for (int it = 0; ok; ++it) {
       const int rr = read_item(it, ok);
       if (!ok || rr >= p.rows) break;
       const int n_sel = list_count<PAIR>(p, rr);
       const int n = (n_sel + KB - 1) / KB;  // KV tiles of the work item
       const int* lst = PAIR ? p.pair_col + list_begin<PAIR>(p, rr) : nullptr;
-      float m_used = -INFINITY, l = 0.f;
+      float m_g = -INFINITY, l = 0.f;  // this group's partial row sum, scaled by 2^-m_g
       for (int j = 0; j < n && ok; ++j, ++s_it) {
-        // paired 64-token blocks: this warp's 64 keys are one KV block and its
-        // rows one query block; the block counts for these rows only if their
-        // query block selected it (and exists: an odd last tile repeats it)
-        bool masked = false;
+        if ((s_it & 1) != grp) continue;
+        // paired 64-token blocks: keys 0-63 and 64-127 are two KV blocks and
+        // this quarter's rows one query block; a block counts for these rows
+        // only if their query block selected it (and exists: an odd last tile
+        // repeats it)
+        bool mask0 = false, mask1 = false;
         if constexpr (PAIR) {
-          const int e = KB * j + half;
-          masked = e >= n_sel || !((__ldg(lst + e) >> kPairShift) & (sp < 2 ? 1 : 2));
+          const int bit = sp < 2 ? 1 : 2;
+          mask0 = !((__ldg(lst + KB * j) >> kPairShift) & bit);
+          mask1 = KB * j + 1 >= n_sel || !((__ldg(lst + KB * j + 1) >> kPairShift) & bit);
         }
         const int sb = s_it % kSBufs;
 #ifdef LCSA_TEST_STALL
@@ -705,73 +745,105 @@ __global__ void __launch_bounds__(kThreads, 1)
 #endif
         if (!(ok = warp_wait(bar(bars->s_full[sb]), (s_it / kSBufs) & 1, abort, p.err, 20))) break;
         tc_fence_after();
+        // one 64-key half in registers at a time: both halves are read for
+        // the block maximum, then half 1's exponentials come from the
+        // registers and half 0 is read again (keeps the warp under its
+        // register share without spills)
         uint32_t sr[2][32];
-        tmem_ld32(lane_addr + kColS + sb * 128 + half * 64, sr[0]);
-        tmem_ld32(lane_addr + kColS + sb * 128 + half * 64 + 32, sr[1]);
-        tmem_wait_ld();
-        // row maximum of this half: 8 independent chains of three-input max
-        auto sv = [&](int e) { return __uint_as_float(sr[e >> 5][e & 31]); };
-        float mk[8];
+        // `after`: a value the load must wait for (an asm input), so the
+        // compiler cannot issue it while the previous half is still needed
+        auto load_half = [&](int hh, float after) {
+          tmem_ld32_after(lane_addr + kColS + sb * 128 + hh * 64, sr[0], after);
+          tmem_ld32(lane_addr + kColS + sb * 128 + hh * 64 + 32, sr[1]);
+          tmem_wait_ld();
+        };
+        // 8 independent chains of three-input max over the half in registers
+        auto half_max = [&]() {
+          auto sv = [&](int e) { return __uint_as_float(sr[e >> 5][e & 31]); };
+          float mk[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          mk[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
-          mk[a] = fmax3(mk[a], sv(a + 24), sv(a + 32));
-          mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
-          mk[a] = fmaxf(mk[a], sv(a + 56));
+          for (int a = 0; a < 8; ++a) {
+            mk[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
+            mk[a] = fmax3(mk[a], sv(a + 24), sv(a + 32));
+            mk[a] = fmax3(mk[a], sv(a + 40), sv(a + 48));
+            mk[a] = fmaxf(mk[a], sv(a + 56));
+          }
+          return fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+        };
+        float mx = -INFINITY;
+        if (!mask0) {
+          load_half(0, 0.f);
+          mx = half_max();
         }
-        const float mpart =
-            masked ? -INFINITY : fmax3(fmax3(mk[0], mk[1], mk[2]), fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
-        float* slot = xmax + (j & 1) * 256;
-        slot[half * 128 + row_in_tile] = mpart;
-        mbar_arrive(bar(bars->pair[sp]));
-        if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 23))) break;
-        ++xk;
-        const float mx = fmaxf(mpart, slot[(half ^ 1) * 128 + row_in_tile]);
-        const float m_new = fmaxf(m_used, mx * c);
-        const bool need = m_new > m_used + kRescaleLog2;
-        const bool warp_need = __any_sync(0xffffffffu, need);
-        float alpha = 1.f;
-        if (need) {
-          alpha = exp2_mufu(m_used - m_new);
-          m_used = m_new;
+        if (!mask1) {
+          load_half(1, mx);
+          mx = fmaxf(mx, half_max());
         }
-        l *= alpha;
-        const float mneg = -m_used;
-        uint32_t pk[32];
+        // the maximum in use so far (tile s - 1 belongs to the other group;
+        // every tile waits for it, even at a row start, which keeps the
+        // barrier phases in step)
+        float m_prev = -INFINITY;
+        if (s_it > 0) {
+          if (!(ok = wait_dec(s_it - 1))) break;
+          if (j > 0) m_prev = xdec[((s_it - 1) & 1) * 128 + row_in_tile];
+        }
+        const float m_new = fmaxf(m_prev, mx * c);
+        const bool need = m_new > m_prev + kRescaleLog2;
+        const float m_used = need ? m_new : m_prev;
+        xdec[(s_it & 1) * 128 + row_in_tile] = m_used;
+        mbar_arrive(bar(bars->dec[sp][s_it & 1]));
+        if (m_g != m_used) {
+          if (l != 0.f) l *= exp2_mufu(m_g - m_used);
+          m_g = m_used;
+        }
+        const float2 c2 = make_float2(c, c), m2 = make_float2(-m_used, -m_used);
         float2 rs2[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) rs2[a] = make_float2(0.f, 0.f);
-        const float2 c2 = make_float2(c, c), m2 = make_float2(mneg, mneg);
+        // half 1 (in registers unless masked), then half 0 (read again)
+        uint32_t pk_prev = 0u;
+#pragma unroll 1
+        for (int step = 0; step < 2; ++step) {
+          const int hh = 1 - step;
+          uint32_t pk[32];
+          if (hh == 0 ? mask0 : mask1) {
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
+          } else {
+            if (hh == 0 && !mask1) load_half(0, __uint_as_float(pk_prev));  // (half 1 masked: half 0 still in registers)
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[q2][e]), __uint_as_float(sr[q2][e + 1])), c2, m2);
-            const float2 pp = ((e >> 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly2(x)
-                                                                         : make_float2(exp2_mufu(x.x), exp2_mufu(x.y));
-            rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], pp);
-            pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
+            for (int q2 = 0; q2 < 2; ++q2) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float2 x =
+                    __ffma2_rn(make_float2(__uint_as_float(sr[q2][e]), __uint_as_float(sr[q2][e + 1])), c2, m2);
+                const float2 pp = ((e >> 1) % kPolyEvery == kPolyEvery - 1)
+                                      ? exp2_poly2(x)
+                                      : make_float2(exp2_mufu(x.x), exp2_mufu(x.y));
+                rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], pp);
+                pk[q2 * 16 + (e >> 1)] = pack_bf16(pp.x, pp.y);
+              }
+            }
           }
+          // P of keys 64 hh .. 64 hh + 63 into columns 64 hh .. 64 hh + 31 (already read)
+          tmem_st32(lane_addr + kColS + sb * 128 + hh * 64, pk);
+          pk_prev = pk[31];
         }
-        if (masked) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = 0u;
-        } else {
-          const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-          l += rsum.x + rsum.y;
-        }
-        // O is touched only to rescale it, once every earlier P.V has
-        // completed; the last of them is P.V number gp = s_it - 1. P.V number
-        // gp + 2 needs a P this warp has not written yet, so the parity wait
-        // on o_done[gp & 1] cannot be overtaken.
-        if (j >= 1 && warp_need) {
+        const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        l += rsum.x + rsum.y;
+        // O is rescaled when this tile raised the maximum, once every earlier
+        // P.V of the row has completed; the last of them is P.V number
+        // gp = s_it - 1, and P.V gp - 2 has completed (S of this tile was
+        // issued only after it), so the parity wait is unambiguous
+        if (j >= 1 && __any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2_mufu(m_prev - m_used) : 1.f;
           const int gp = s_it - 1;
           if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 21))) break;
           tc_fence_after();
 #pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
+          for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
-            const uint32_t oa = lane_addr + kColO + half * 64 + q2 * 32;
+            const uint32_t oa = lane_addr + kColO + q * 32;
             tmem_ld32(oa, o);
             tmem_wait_ld();
 #pragma unroll
@@ -779,35 +851,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(oa, o);
           }
         }
-        tmem_st32(lane_addr + kColS + sb * 128 + half * 64, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->p_full[sb]));
       }
       if (!ok) break;
-      // epilogue: wait for the last P.V, combine the two halves' row sums,
-      // normalise and store this thread's 64 output channels
+      // epilogue: the row's final maximum, the two groups' sums brought to it
+      // and added, then each group normalises and stores 64 output channels
+      const int s_last = s_it - 1;
+      float m_final = m_g;
+      if ((s_last & 1) != grp) {
+        if (!(ok = wait_dec(s_last))) break;  // waited for again by this warp's next tile: harmless
+        m_final = xdec[(s_last & 1) * 128 + row_in_tile];
+      }
+      if (m_g != m_final && l != 0.f) l *= exp2_mufu(m_g - m_final);
       {
-        // The row's last P.V is number gp = s_it - 1 (its completion implies
+        // The row's last P.V is number gp = s_last (its completion implies
         // all earlier ones). A parity wait is only unambiguous while its
         // barrier is at most one phase short of the target: o_done[gp & 1]
-        // last completed for P.V gp - 2, which nothing has waited for, and if
-        // that one were still running the parity test would pass at once. So
-        // P.V gp - 1 is waited for first: its barrier's previous phase, P.V
-        // gp - 3, completed before S of block gp was issued, and its
+        // last completed for P.V gp - 2, which nothing may have waited for.
+        // So P.V gp - 1 is waited for first: its barrier's previous phase,
+        // P.V gp - 3, completed before S of tile gp was issued, and its
         // completion implies gp - 2's.
-        const int gp = s_it - 1;
+        const int gp = s_last;
         if (gp >= 1 && !(ok = warp_wait(bar(bars->o_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, abort, p.err, 25)))
           break;
         if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 22))) break;
       }
       tc_fence_after();
-      xsum[half * 128 + row_in_tile] = l;
+      // row sums, double-buffered by row: a group can start the next row's
+      // epilogue before its partner has read this row's sum
+      float* xs = xsum + (xk & 1) * 256;
+      xs[grp * 128 + row_in_tile] = l;
       mbar_arrive(bar(bars->pair[sp]));
       if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
       ++xk;
-      const float inv = 1.0f / (l + xsum[(half ^ 1) * 128 + row_in_tile]);
+      const float inv = 1.0f / (l + xs[(grp ^ 1) * 128 + row_in_tile]);
       int qrow = rr, m_tok = row_in_tile;  // query block (row) and token of this lane's row
       bool store = true;
       if constexpr (PAIR) {
@@ -823,11 +903,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tb = qb / g.bpf, rem = qb % g.bpf;
       const int tt = m_tok / (g.bh * g.bw), yy = (m_tok / g.bw) % g.bh, xx = m_tok % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
-      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + half * 64;
+      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + grp * 64;
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t o[32];
-        tmem_ld32(lane_addr + kColO + half * 64 + q2 * 32, o);
+        tmem_ld32(lane_addr + kColO + grp * 64 + q2 * 32, o);
         tmem_wait_ld();
         uint4 v[4];
         uint32_t* w = reinterpret_cast<uint32_t*>(v);
@@ -843,11 +923,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bars->o_free));
-      // xsum is rewritten only after this row's next exchanges, which need the
-      // partner's arrival, so the partner has read it by then
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
