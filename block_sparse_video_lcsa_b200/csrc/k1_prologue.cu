@@ -12,7 +12,7 @@
 // Work split: a persistent grid of one CTA per SM (8 compute warps and one
 // copy warp); CTA c owns a contiguous range of the combined row list (query
 // blocks, then key blocks; a block is bt * bh rows of bw tokens). Each row is
-// one contiguous run of bw * heads * 128 bf16 in the raster input, so the
+// one contiguous run of bw * heads * head_dim bf16 in the raster input, so the
 // copy warp streams the rows into a ring of shared-memory stages with bulk
 // asynchronous copies (cp.async.bulk, completion counted on a "full"
 // mbarrier per stage) several rows ahead. Warp w takes tokens w, w+8, ... of
@@ -153,16 +153,17 @@ __device__ __forceinline__ BlockRef block_ref(const K1Params& p, int bid) {
   return r;
 }
 
-// CPL = 16-byte chunks per lane per token = ceil(heads * 16 / 32); FULL: every
-// lane's CPL chunks exist (even head count); HEAD: per-head norm scope.
+// D = head_dim (64 or 128); CPL = 16-byte chunks per lane per token =
+// ceil(heads * D / 8 / 32); FULL: every lane's CPL chunks exist; HEAD:
+// per-head norm scope.
 // Warps per CTA. (16, one token of a 16-token row each, measured slower: a
 // lane's pooled sums and token do not fit 128 registers without spills.)
 template <int CPL>
 __host__ __device__ constexpr int k1_warps() { return 8; }
 
-// A processed row (bw tokens x heads x 128, token-major as it arrived) goes
-// from its ring stage to q^ / k^ in one bulk tensor store: the map's box is
-// (128 channels, all heads, bw tokens of one block) over the head-major
+// A processed row (bw tokens x heads x head_dim, token-major as it arrived)
+// goes from its ring stage to q^ / k^ in one bulk tensor store: the map's box
+// is (head_dim channels, all heads, bw tokens of one block) over the head-major
 // layout, so the shared-memory side is exactly the raster row.
 __device__ __forceinline__ void store_row(const CUtensorMap* map, uint32_t src, int r_tok, int blk, int b) {
   asm volatile(
@@ -196,7 +197,7 @@ __device__ __forceinline__ void record_timeout(unsigned* err, unsigned site) {
 
 // Warps 0..NW-1 compute; warp NW is the copy warp (one lane issues every bulk
 // copy, so the compute warps never block on the copy engine).
-template <int CPL, bool FULL, bool HEAD>
+template <int D, int CPL, bool FULL, bool HEAD>
 __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
     prologue_kernel(const __grid_constant__ CUtensorMap tm_qhat, const __grid_constant__ CUtensorMap tm_khat,
                     const K1Params p, int stages, uint32_t row_bytes) {
@@ -219,7 +220,9 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
   const int64_t nrows = int64_t(total) * R;
   const int64_t lo = nrows * blockIdx.x / gridDim.x, hi = nrows * (blockIdx.x + 1) / gridDim.x;
   const int my_rows = int(hi - lo);
-  constexpr int PT = 22, PH = 21;  // RoPE pairs on the frame / row axes (head_dim 128)
+  // RoPE pairs on the frame / row / column axes of a head: (22, 21, 21) for
+  // head_dim 128, (12, 10, 10) for 64
+  constexpr int PH = D / 6, PT = D / 2 - 2 * PH;
 
   // full[s]: the stage's row has landed; done[s]: every compute warp has
   // finished the stage's row in place
@@ -305,7 +308,8 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
   }
   compute_sync(NT);
 
-  const int jb = 4 * (lane & 15);  // first RoPE pair of this lane (same in every head)
+  constexpr int kChunksPerHead = D / 8;
+  const int jb = 4 * (lane & (kChunksPerHead - 1));  // first RoPE pair of this lane (same in every head)
   float2 ae[CPL][2], ao[CPL][2];  // pooled sums, e / o layout of unpack_eo
   __shared__ int combine;
   int gi = 0;  // rows of this CTA consumed so far
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
           const int j = jb + qd;
           const int idx = j < PT        ? t * PT + j
                           : j < PT + PH ? p.rope_h_off + y * PH + (j - PT)
-                                        : p.rope_w_off + xc * (kHeadDim / 2 - PT - PH) + (j - PT - PH);
+                                        : p.rope_w_off + xc * (D / 2 - PT - PH) + (j - PT - PH);
           cs[qd] = __ldg(p.rope + idx);
         }
         // RMSNorm scale(s), folded into the rotation: x^ = rot(rs * (x * gamma)).
@@ -401,8 +405,9 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
             }
             float ss = ss2.x + ss2.y;
 #pragma unroll
-            for (int o2 = 8; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
-            rr_h[c4] = rsqrtf(ss * (1.0f / float(kHeadDim)) + p.eps);
+            // the lanes of one head: 16 (head_dim 128) or 8 (64)
+            for (int o2 = kChunksPerHead / 2; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
+            rr_h[c4] = rsqrtf(ss * (1.0f / float(D)) + p.eps);
           }
         }
 #pragma unroll
@@ -465,8 +470,8 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
       compute_sync(NT);
     }
     const float inv_nb = 1.0f / float(g.nb);
-    float* pooled_row = pooled + (int64_t(br.b) * g.Hn * br.nblk + br.blk) * kHeadDim;  // + head * nblk * d + dd
-    const int64_t head_stride = int64_t(br.nblk) * kHeadDim;
+    float* pooled_row = pooled + (int64_t(br.b) * g.Hn * br.nblk + br.blk) * D;  // + head * nblk * d + dd
+    const int64_t head_stride = int64_t(br.nblk) * D;
     auto warp_sum = [&](int e) {
       float sum = red[e];
 #pragma unroll
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
     };
     if (r_begin == 0 && r_end == R) {
       for (int e = threadIdx.x; e < g.C; e += NT)
-        pooled_row[(e / kHeadDim) * head_stride + e % kHeadDim] = warp_sum(e) * inv_nb;
+        pooled_row[(e / D) * head_stride + e % D] = warp_sum(e) * inv_nb;
     } else {
       // A block cut between CTA c and c + 1: CTA c holds its first rows (part
       // 0), CTA c + 1 the rest (part 1). Each writes its part to the cut's
@@ -498,7 +503,7 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
       compute_sync(NT);
       if (combine) {
         for (int e = threadIdx.x; e < g.C; e += NT)
-          pooled_row[(e / kHeadDim) * head_stride + e % kHeadDim] =
+          pooled_row[(e / D) * head_stride + e % D] =
               (__ldcg(part + e) + __ldcg(part + g.C + e)) * inv_nb;
       }
     }
@@ -508,7 +513,7 @@ __global__ void __launch_bounds__((k1_warps<CPL>() + 1) * 32, 1)
   if (!ok && threadIdx.x == 0) record_timeout(p.err, 1);
 }
 
-template <int CPL, bool FULL, bool HEAD>
+template <int D, int CPL, bool FULL, bool HEAD>
 cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   const int nblocks = p.n_qblk + p.g.B * p.k_in_fb * p.g.bpf;
   if (nblocks <= 0) return cudaSuccess;
@@ -518,7 +523,8 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2 || p.num_sms <= 0) return cudaErrorInvalidValue;
   const size_t smem = kBarBytes + 128 + size_t(stages) * row_bytes + red_bytes;  // + alignment of the ring
-  cudaError_t e = cudaFuncSetAttribute(prologue_kernel<CPL, FULL, HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e =
+      cudaFuncSetAttribute(prologue_kernel<D, CPL, FULL, HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   int grid = nblocks < p.num_sms ? nblocks : p.num_sms;
   if (grid > kMaxK1Ctas) grid = kMaxK1Ctas;
@@ -526,8 +532,8 @@ cudaError_t launch_cpl(const K1Params& p, cudaStream_t s) {
   if ((e = make_xhat_row_map(&tm_qhat, p.qhat, p.g, p.g.nQB)) != cudaSuccess ||
       (e = make_xhat_row_map(&tm_khat, p.khat, p.g, p.g.nKB)) != cudaSuccess)
     return e;
-  prologue_kernel<CPL, FULL, HEAD><<<grid, (k1_warps<CPL>() + 1) * 32, smem, s>>>(tm_qhat, tm_khat, p, stages,
-                                                                                 row_bytes);
+  prologue_kernel<D, CPL, FULL, HEAD><<<grid, (k1_warps<CPL>() + 1) * 32, smem, s>>>(tm_qhat, tm_khat, p, stages,
+                                                                                    row_bytes);
   return cudaGetLastError();
 }
 
@@ -583,22 +589,35 @@ cudaError_t launch_sumsq(const __nv_bfloat16* q, int64_t nq, const __nv_bfloat16
 }
 
 cudaError_t launch_prologue(const K1Params& p, cudaStream_t s) {
-  const bool full = p.g.Hn % 2 == 0, head = p.norm_scope != 0;
-#define LCSA_K1_CASE(n)                                                              \
-  case n:                                                                            \
-    if (full) return head ? launch_cpl<n, true, true>(p, s) : launch_cpl<n, true, false>(p, s); \
-    return head ? launch_cpl<n, false, true>(p, s) : launch_cpl<n, false, false>(p, s);
-  switch ((p.g.Hn + 1) / 2) {
-    LCSA_K1_CASE(1)
-    LCSA_K1_CASE(2)
-    LCSA_K1_CASE(3)
-    LCSA_K1_CASE(4)
-    LCSA_K1_CASE(5)
-    LCSA_K1_CASE(6)
-    LCSA_K1_CASE(7)
-    LCSA_K1_CASE(8)
-    default: return cudaErrorInvalidValue;
+  const int nchunks = p.g.C / 8;
+  const bool full = nchunks % 32 == 0, head = p.norm_scope != 0;
+#define LCSA_K1_CASE(d, n)                                                                          \
+  case n:                                                                                           \
+    if (full) return head ? launch_cpl<d, n, true, true>(p, s) : launch_cpl<d, n, true, false>(p, s); \
+    return head ? launch_cpl<d, n, false, true>(p, s) : launch_cpl<d, n, false, false>(p, s);
+  if (p.g.D == 128) {
+    switch ((nchunks + 31) / 32) {
+      LCSA_K1_CASE(128, 1)
+      LCSA_K1_CASE(128, 2)
+      LCSA_K1_CASE(128, 3)
+      LCSA_K1_CASE(128, 4)
+      LCSA_K1_CASE(128, 5)
+      LCSA_K1_CASE(128, 6)
+      LCSA_K1_CASE(128, 7)
+      LCSA_K1_CASE(128, 8)
+      default: return cudaErrorInvalidValue;
+    }
   }
+  if (p.g.D == 64) {
+    switch ((nchunks + 31) / 32) {
+      LCSA_K1_CASE(64, 1)
+      LCSA_K1_CASE(64, 2)
+      LCSA_K1_CASE(64, 3)
+      LCSA_K1_CASE(64, 4)
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  return cudaErrorInvalidValue;
 #undef LCSA_K1_CASE
 }
 

@@ -42,6 +42,9 @@ __device__ __forceinline__ unsigned order_bits(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// D: head_dim (64 or 128); the first D / 4 lanes hold a pooled vector's
+// float4s, the others add zeros.
+template <int D>
 __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   extern __shared__ __align__(16) unsigned long long keys[];  // [sort_n], then flags [sort_n] bytes
   unsigned char* flag = reinterpret_cast<unsigned char*>(keys + p.sort_n);
@@ -78,8 +81,10 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
     return slot * g.bpf + (h0 + hr) * g.nWb + (w0 + wr);
   };
 
-  const float4 qv = reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * kHeadDim)[lane];
-  const float4* pk = reinterpret_cast<const float4*>(p.pooled_k + int64_t(bh) * g.nKB * kHeadDim);
+  constexpr int kLanes = D / 4;  // lanes that hold part of a pooled vector
+  const float4 qv = lane < kLanes ? reinterpret_cast<const float4*>(p.pooled_q + int64_t(rr) * D)[lane]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* pk = reinterpret_cast<const float4*>(p.pooled_k + int64_t(bh) * g.nKB * D);
 
   if (blockIdx.x == 0)
     for (int c = threadIdx.x; c < p.n_clear; c += kThreads) p.clear_cnt[c] = 0u;
@@ -91,7 +96,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
       const int c = c0 + u;
-      kv[u] = c < nc ? pk[int64_t(cand_block(c, true)) * (kHeadDim / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+      kv[u] = (c < nc && lane < kLanes) ? pk[int64_t(cand_block(c, true)) * kLanes + lane]
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kCandPerIter; ++u) {
@@ -285,15 +291,24 @@ cudaError_t launch_pair_union(const PairParams& p, cudaStream_t s) {
 
 size_t select_smem_bytes(int sort_n) { return size_t(sort_n) * (sizeof(unsigned long long) + 1); }
 
-cudaError_t launch_select(const K2Params& p, cudaStream_t s) {
+namespace {
+template <int D>
+cudaError_t launch_select_d(const K2Params& p, cudaStream_t s) {
   const size_t smem = select_smem_bytes(p.sort_n);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
   const int rows = p.g.B * p.g.Hn * p.g.nQB;
-  select_kernel<<<rows, kThreads, smem, s>>>(p);
+  select_kernel<D><<<rows, kThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_select(const K2Params& p, cudaStream_t s) {
+  if (p.g.D == 128) return launch_select_d<128>(p, s);
+  if (p.g.D == 64) return launch_select_d<64>(p, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace lcsa

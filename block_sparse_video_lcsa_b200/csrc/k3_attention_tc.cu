@@ -76,11 +76,11 @@ namespace lcsa {
 namespace {
 
 constexpr int kNB = 128;                    // keys per KV tile (one 128-token block or two 64-token blocks)
-constexpr int kD = 128;                     // head_dim
 constexpr int kKStages = 2;
 constexpr int kVStages = 3;
-constexpr uint32_t kTileBytes = kNB * kD * 2;   // 32 KB
-constexpr uint32_t kHalfBytes = kTileBytes / 2; // 64 columns of a tile
+// A tile (Q, K^ or V) is 128 rows x head_dim bf16, stored as head_dim / 64
+// blocks of 64 columns (one 128-byte swizzle atom wide), 16 KB each.
+constexpr uint32_t kHalfBytes = kNB * 64 * 2;
 constexpr int kThreads = 352;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kPolyEvery = 4;  // one pair of exponentials in kPolyEvery on the FMA pipe
@@ -95,15 +95,22 @@ constexpr unsigned long long kWaitLimitNs = 100000000ull;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 #endif
 
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;
-constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
-constexpr uint32_t kOffXchg = kOffBar + 512;          // row max / sum exchange
 constexpr int kItemSlots = 4;  // work items handed from the producer to the other roles
 constexpr int kItemReaders = 2 + kSoftmaxWarps;  // S issuer, P.V issuer, softmax warps (one arrival each)
 constexpr uint32_t kXchgBytes = (2 * 128 + 2 * 2 * 128) * 4;
-constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
+
+// Shared-memory layout for head_dim D (64 or 128): the Q tile, the K^ and V
+// rings, the barrier block and the row maximum / sum exchange.
+template <int D>
+struct Smem {
+  static constexpr uint32_t tile = kNB * D * 2;
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t k = q + tile;
+  static constexpr uint32_t v = k + kKStages * tile;
+  static constexpr uint32_t bar = v + kVStages * tile;
+  static constexpr uint32_t xchg = bar + 512;
+  static constexpr uint32_t bytes = xchg + kXchgBytes + 1024;  // + alignment slack
+};
 
 // 2^f on [-1/2, 1/2]: degree-3 minimax coefficients (relative error 7.49e-5),
 // fitted by csrc/fit_exp2_poly.py.
@@ -262,9 +269,10 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,
-// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), N = 128, M = 128 or 64.
-__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t b_mn, uint32_t m = 128) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((128u >> 3) << 17) | ((m >> 4) << 24);
+// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M = 128 or 64,
+// N = 128 or 64.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t b_mn, uint32_t m = 128, uint32_t n = 128) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -376,7 +384,8 @@ __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
 
 // PAIR: 64-token blocks, a work item is a pair of query blocks over the union
 // of their selections; otherwise 128-token blocks, a work item is one row.
-template <bool PAIR>
+// D: head_dim (64 or 128).
+template <bool PAIR, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
@@ -384,7 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  Bars* bars = reinterpret_cast<Bars*>(gbase + kOffBar);
+  using L = Smem<D>;
+  constexpr int kHalves = D / 64;  // 64-column blocks of a tile
+  Bars* bars = reinterpret_cast<Bars*>(gbase + L::bar);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = p.g;
@@ -493,16 +504,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = bhh / g.Hn, h = bhh % g.Hn;
       if (row_it > 0 && !(ok = warp_wait(bar(bars->q_empty), (row_it - 1) & 1, abort, p.err, 1))) break;
       if (lane == 0) {
-        mbar_expect_tx(bar(bars->q_full), QM * kD * 2);
-        if constexpr (PAIR) {
+        mbar_expect_tx(bar(bars->q_full), L::tile);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            tma_load_2d(base + kOffQ + hh * QM * 128, &tm_q, hh * 64, ra * NBLK, bar(bars->q_full));
-            tma_load_2d(base + kOffQ + hh * QM * 128 + NBLK * 128, &tm_q, hh * 64, rb * NBLK, bar(bars->q_full));
+        for (int hh = 0; hh < kHalves; ++hh) {
+          if constexpr (PAIR) {
+            tma_load_2d(base + L::q + hh * kHalfBytes, &tm_q, hh * 64, ra * NBLK, bar(bars->q_full));
+            tma_load_2d(base + L::q + hh * kHalfBytes + NBLK * 128, &tm_q, hh * 64, rb * NBLK, bar(bars->q_full));
+          } else {
+            tma_load_2d(base + L::q + hh * kHalfBytes, &tm_q, hh * 64, rr * QM, bar(bars->q_full));
           }
-        } else {
-          tma_load_2d(base + kOffQ, &tm_q, 0, rr * QM, bar(bars->q_full));
-          tma_load_2d(base + kOffQ + QM * 128, &tm_q, 64, rr * QM, bar(bars->q_full));
         }
       }
       __syncwarp();
@@ -533,15 +543,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_k = [&](int st) -> bool {
         const int kvj = kv + st, ks = kvj % kKStages, ku = kvj / kKStages;
         if (ku > 0 && !warp_wait(bar(bars->k_empty[ks]), (ku - 1) & 1, abort, p.err, 2)) return false;
-        const uint32_t kdst = base + kOffK + ks * kTileBytes;
-        if (lane == 0) mbar_expect_tx(bar(bars->k_full[ks]), kTileBytes);
+        const uint32_t kdst = base + L::k + ks * L::tile;
+        if (lane == 0) mbar_expect_tx(bar(bars->k_full[ks]), L::tile);
 #pragma unroll
         for (int i = 0; i < KB; ++i) {
           const int src = entry(ke, st, i);
           const int krow = __shfl_sync(0xffffffffu, ke.krow, src);
           if (lane == 0) {
-            tma_load_2d(kdst + i * NBLK * 128, &tm_k, 0, krow, bar(bars->k_full[ks]));
-            tma_load_2d(kdst + kHalfBytes + i * NBLK * 128, &tm_k, 64, krow, bar(bars->k_full[ks]));
+#pragma unroll
+            for (int hh = 0; hh < kHalves; ++hh)
+              tma_load_2d(kdst + hh * kHalfBytes + i * NBLK * 128, &tm_k, hh * 64, krow, bar(bars->k_full[ks]));
           }
         }
         __syncwarp();
@@ -553,16 +564,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (st + 2 < steps && !(ok = load_k(st + 2))) break;
         const int kvj = kv + st, vs = kvj % kVStages, vu = kvj / kVStages;
         if (vu > 0 && !(ok = warp_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
-        const uint32_t vdst = base + kOffV + vs * kTileBytes;
-        if (lane == 0) mbar_expect_tx(bar(bars->v_full[vs]), kTileBytes);
+        const uint32_t vdst = base + L::v + vs * L::tile;
+        if (lane == 0) mbar_expect_tx(bar(bars->v_full[vs]), L::tile);
 #pragma unroll
         for (int i = 0; i < KB; ++i) {
           const int src = entry(ve, st, i);
           const int x0 = __shfl_sync(0xffffffffu, ve.x0, src), y0 = __shfl_sync(0xffffffffu, ve.y0, src);
           const int f0 = __shfl_sync(0xffffffffu, ve.f0, src);
           if (lane == 0) {
-            tma_load_5d(vdst + i * NBLK * 128, &tm_v, 0, h, x0, y0, f0, bar(bars->v_full[vs]));
-            tma_load_5d(vdst + kHalfBytes + i * NBLK * 128, &tm_v, 64, h, x0, y0, f0, bar(bars->v_full[vs]));
+#pragma unroll
+            for (int hh = 0; hh < kHalves; ++hh)
+              tma_load_5d(vdst + hh * kHalfBytes + i * NBLK * 128, &tm_v, hh * 64, h, x0, y0, f0, bar(bars->v_full[vs]));
           }
         }
         __syncwarp();
@@ -627,9 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = warp_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t qa = base + kOffQ, ka = base + kOffK + ks * kTileBytes;
+          const uint32_t qa = base + L::q, ka = base + L::k + ks * L::tile;
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
+          for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
             const uint32_t qoff = (kk >> 2) * (QM * 128) + (kk & 3) * 32;
             mma_ss(tmem + kColS + sb * 128, sdesc(qa + qoff, 16, 1024), sdesc(ka + koff, 16, 1024), id_qk,
@@ -651,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ---------------- P.V issuer (converged warp, lane 0 issues) ----------------
-    constexpr uint32_t id_pv = idesc_bf16(1, QM);
+    constexpr uint32_t id_pv = idesc_bf16(1, QM, D);
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int it = 0; ok; ++it, ++row_it) {
@@ -667,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t va = base + kOffV + vs * kTileBytes;
+          const uint32_t va = base + L::v + vs * L::tile;
           const uint32_t pa = tmem + kColS + pb * 128;
 #pragma unroll
           for (int kk = 0; kk < kNB / 16; ++kk) {
@@ -710,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - 3) >> 2;         // which tiles (s & 1) and, at the end, which 64 channels
     const int row_in_tile = sp * 32 + lane;  // query token of this lane's row
     const uint32_t lane_addr = tmem + (uint32_t(sp * 32) << 16);
-    float* xdec = reinterpret_cast<float*>(gbase + kOffXchg);  // [2 tile parity][128] maximum in use
+    float* xdec = reinterpret_cast<float*>(gbase + L::xchg);  // [2 tile parity][128] maximum in use
     float* xsum = xdec + 2 * 128;                              // [2 row parity][2 group][128]
     const float c = p.scale_log2;
     int s_it = 0, xk = 0;
@@ -841,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = warp_wait(bar(bars->o_done[gp & 1]), (gp >> 1) & 1, abort, p.err, 21))) break;
           tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
             const uint32_t oa = lane_addr + kColO + q * 32;
             tmem_ld32(oa, o);
@@ -903,11 +915,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tb = qb / g.bpf, rem = qb % g.bpf;
       const int tt = m_tok / (g.bh * g.bw), yy = (m_tok / g.bw) % g.bh, xx = m_tok % g.bw;
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
-      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * kD + grp * 64;
+      // this group's half of the row's D output channels, 32 at a time
+      __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * D + grp * (D / 2);
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
+      for (int q2 = 0; q2 < D / 64; ++q2) {
         uint32_t o[32];
-        tmem_ld32(lane_addr + kColO + grp * 64 + q2 * 32, o);
+        tmem_ld32(lane_addr + kColO + grp * (D / 2) + q2 * 32, o);
         tmem_wait_ld();
         uint4 v[4];
         uint32_t* w = reinterpret_cast<uint32_t*>(v);
@@ -960,11 +973,11 @@ cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s
   return cudaGetLastError();
 }
 
-cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows, int head_dim) {
   EncodeTiled enc = encoder();
   if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kD * 2)};
+  const cuuint64_t dims[2] = {cuuint64_t(head_dim), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(head_dim) * 2};
   const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -976,10 +989,10 @@ cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int
 cudaError_t make_xhat_row_map(CUtensorMap* map, void* base, const Grid& g, int nblk) {
   EncodeTiled enc = encoder();
   if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t tok = cuuint64_t(kD) * 2, blk = tok * cuuint64_t(g.nb), head = blk * cuuint64_t(nblk);
-  const cuuint64_t dims[5] = {cuuint64_t(kD), cuuint64_t(g.Hn), cuuint64_t(g.nb), cuuint64_t(nblk), cuuint64_t(g.B)};
+  const cuuint64_t tok = cuuint64_t(g.D) * 2, blk = tok * cuuint64_t(g.nb), head = blk * cuuint64_t(nblk);
+  const cuuint64_t dims[5] = {cuuint64_t(g.D), cuuint64_t(g.Hn), cuuint64_t(g.nb), cuuint64_t(nblk), cuuint64_t(g.B)};
   const cuuint64_t strides[4] = {head, tok, blk, head * cuuint64_t(g.Hn)};
-  const cuuint32_t box[5] = {cuuint32_t(kD), cuuint32_t(g.Hn), cuuint32_t(g.bw), 1, 1};
+  const cuuint32_t box[5] = {cuuint32_t(g.D), cuuint32_t(g.Hn), cuuint32_t(g.bw), 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -991,9 +1004,9 @@ cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g) {
   EncodeTiled enc = encoder();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t row = cuuint64_t(g.C) * 2;  // bytes per token
-  const cuuint64_t dims[5] = {cuuint64_t(kD), cuuint64_t(g.Hn), cuuint64_t(g.gw), cuuint64_t(g.gh),
+  const cuuint64_t dims[5] = {cuuint64_t(g.D), cuuint64_t(g.Hn), cuuint64_t(g.gw), cuuint64_t(g.gh),
                               cuuint64_t(g.B) * cuuint64_t(g.Tkv)};
-  const cuuint64_t strides[4] = {cuuint64_t(kD * 2), row, row * cuuint64_t(g.gw), row * cuuint64_t(g.gw) * g.gh};
+  const cuuint64_t strides[4] = {cuuint64_t(g.D) * 2, row, row * cuuint64_t(g.gw), row * cuuint64_t(g.gw) * g.gh};
   const cuuint32_t box[5] = {64, 1, cuuint32_t(g.bw), cuuint32_t(g.bh), cuuint32_t(g.bt)};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
@@ -1013,8 +1026,11 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   if (!attention_tc_supported(p.g)) return cudaErrorInvalidValue;
   const bool paired = p.g.nb == 64 && p.pair_col != nullptr;
   if (p.g.nb == 64 && !paired) return cudaErrorInvalidValue;  // 64-token blocks run as query-block pairs
-  auto kern = paired ? attention_tc_kernel<true> : attention_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  if (p.g.D != 64 && p.g.D != 128) return cudaErrorInvalidValue;
+  auto kern = p.g.D == 128 ? (paired ? attention_tc_kernel<true, 128> : attention_tc_kernel<false, 128>)
+                           : (paired ? attention_tc_kernel<true, 64> : attention_tc_kernel<false, 64>);
+  const uint32_t smem = p.g.D == 128 ? Smem<128>::bytes : Smem<64>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   TcParams tp{};  // every field zero unless set below
   tp.g = p.g;
@@ -1038,7 +1054,7 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   g_stall_site = 0;
 #endif
   const int grid = tp.rows < num_sms ? tp.rows : num_sms;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_k, tm_v, tp);
+  kern<<<grid, kThreads, smem, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();
 }
 

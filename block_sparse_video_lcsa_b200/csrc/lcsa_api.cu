@@ -381,8 +381,8 @@ lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Fault
     return cuda_fail(e, "device attributes");
   }
   {
-    if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&p->tm_k, p->khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb)) != cudaSuccess) {
+    if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb, g.D)) != cudaSuccess ||
+        (e = lcsa::make_block_map(&p->tm_k, p->khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb, g.D)) != cudaSuccess) {
       release(p);
       delete p;
       return cuda_fail(e, "tensor maps");
@@ -461,7 +461,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k1.slot0_fb = sb.slot0_fb;
   k1.Lk_in = int64_t(sb.k_in_fb) * g.bt * g.gh * g.gw;
   k1.ss_ext = sb.ss_ext;
-  k1.norm_inv_c = 1.0f / float(int64_t(p->res.heads_total) * lcsa::kHeadDim);
+  k1.norm_inv_c = 1.0f / float(int64_t(p->res.heads_total) * g.D);
 
   lcsa::K2Params k2{};  // every field zero (null) unless set below
   k2.g = g;
@@ -826,9 +826,9 @@ lcsa_status_t lcsa_get_intermediates(lcsa_plan_t p, void* qhat, void* khat, floa
   if (e == cudaSuccess && qhat) e = cudaMemcpy(qhat, p->qhat, size_t(g.B) * g.Lq * g.C * 2, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && khat) e = cudaMemcpy(khat, p->khat, size_t(g.B) * g.Lkv * g.C * 2, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && pooled_q)
-    e = cudaMemcpy(pooled_q, p->pooled_q, size_t(g.B) * g.Hn * g.nQB * lcsa::kHeadDim * 4, cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(pooled_q, p->pooled_q, size_t(g.B) * g.Hn * g.nQB * g.D * 4, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && pooled_k)
-    e = cudaMemcpy(pooled_k, p->pooled_k, size_t(g.B) * g.Hn * g.nKB * lcsa::kHeadDim * 4, cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(pooled_k, p->pooled_k, size_t(g.B) * g.Hn * g.nKB * g.D * 4, cudaMemcpyDeviceToHost);
   return e == cudaSuccess ? LCSA_OK : cuda_fail(e, "copy intermediates");
 }
 

@@ -83,7 +83,8 @@ lcsa_status_t resolve_config(const lcsa_config_t* c, ConfigCore* r, char* msg, s
   if (c->grid_h % c->block_h || c->grid_w % c->block_w || c->q_frames % c->block_t || c->kv_frames % c->block_t)
     return refuse(msg, cap, LCSA_ERR_SHAPE, "token grid %dx%dx%d (q %d) not divisible by block %dx%dx%d",
                   c->kv_frames, c->grid_h, c->grid_w, c->q_frames, c->block_t, c->block_h, c->block_w);
-  if (c->head_dim != kHeadDim) return refuse(msg, cap, LCSA_ERR_UNSUPPORTED, "head_dim %d (only 128)", c->head_dim);
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return refuse(msg, cap, LCSA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", c->head_dim);
   if (c->heads > kMaxHeads) return refuse(msg, cap, LCSA_ERR_UNSUPPORTED, "heads %d > %d", c->heads, kMaxHeads);
   const int nb = c->block_t * c->block_h * c->block_w;
   if (nb != 64 && nb != 128) return refuse(msg, cap, LCSA_ERR_UNSUPPORTED, "block of %d tokens (64 or 128)", nb);
@@ -117,6 +118,7 @@ lcsa_status_t resolve_config(const lcsa_config_t* c, ConfigCore* r, char* msg, s
   g.nKB = (c->kv_frames / c->block_t) * g.bpf;
   g.Lq = int64_t(c->q_frames) * c->grid_h * c->grid_w;
   g.Lkv = int64_t(c->kv_frames) * c->grid_h * c->grid_w;
+  g.D = c->head_dim;
   g.C = c->heads * c->head_dim;
   r->heads_total = c->heads_total == 0 ? c->heads : c->heads_total;
 

@@ -11,7 +11,7 @@
 
 namespace lcsa {
 
-constexpr int kHeadDim = 128;        // the only head size the kernels implement
+constexpr int kMaxHeadDim = 128;     // head sizes the kernels implement: 64 and 128
 constexpr int kMaxHeads = 16;
 constexpr int kMaxCandidates = 4096; // admissible blocks per query block (K2 sort)
 constexpr int kMaxK1Ctas = 256;      // K1 persistent grid cap (sizes its split-block buffers)
@@ -51,6 +51,7 @@ struct Grid {
   int nHb, nWb, bpf;    // block rows / columns / blocks per frame group
   int nQB, nKB;         // blocks per (batch, head)
   int64_t Lq, Lkv;      // tokens per batch element
+  int D;                // head_dim (64 or 128)
   int C;                // heads * head_dim
 };
 
@@ -226,15 +227,15 @@ size_t select_smem_bytes(int sort_n);
 cudaError_t launch_select(const K2Params& p, cudaStream_t s);
 cudaError_t launch_pair_union(const PairParams& p, cudaStream_t s);
 
-// tcgen05 attention (128- or 64-token blocks). Tensor maps: q^ / k^ as
-// [rows][128] bf16 with boxes of 64 columns x one block of rows
+// tcgen05 attention (128- or 64-token blocks, head_dim 128 or 64). Tensor
+// maps: q^ / k^ as [rows][head_dim] bf16 with boxes of 64 columns x one block of rows
 // (make_block_map, box_rows = tokens per block), V through its raster layout
 // (make_raster_map). The kernel is persistent over min(rows, num_sms) CTAs.
 bool attention_tc_supported(const Grid& g);
-cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
+cudaError_t make_block_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows, int head_dim);
 cudaError_t make_raster_map(CUtensorMap* map, const void* base, const Grid& g);
-// q^ / k^ ([B][Hn][nblk][nb][128]) seen as (channel, head, token of the block,
-// block, batch) with boxes of (128, Hn, bw, 1, 1): one box is one raster row of
+// q^ / k^ ([B][Hn][nblk][nb][head_dim]) seen as (channel, head, token of the
+// block, block, batch) with boxes of (head_dim, Hn, bw, 1, 1): one box is one raster row of
 // bw tokens with all heads, token-major in shared memory (K1's bulk stores).
 cudaError_t make_xhat_row_map(CUtensorMap* map, void* base, const Grid& g, int nblk);
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);

@@ -317,8 +317,8 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
     LCSA_RANGE("lcsa K3 attention");
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
     const int num_sms = k1.num_sms;
-    if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb)) != cudaSuccess ||
-        (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb)) != cudaSuccess ||
+    if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb, g.D)) != cudaSuccess ||
+        (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb, g.D)) != cudaSuccess ||
         (e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess)
       return LCSA_ERR_CUDA;
     if ((e = lcsa::launch_attention_tc(k3, tm_q, tm_k, tm_v, num_sms, s)) != cudaSuccess) return LCSA_ERR_CUDA;

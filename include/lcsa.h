@@ -26,7 +26,8 @@
  * Readings where the pages are silent: the RMSNorm spans heads*head_dim
  * (LCSA_NORM_TOKEN; LCSA_NORM_HEAD is offered), eps 1e-6; RoPE rotates pairs
  * (2i, 2i+1), first d-4*(d/6) dims by frame, next 2*(d/6) by token row, last
- * 2*(d/6) by token column, pair j of an n-dim axis turning by
+ * 2*(d/6) by token column (44/42/42 for d = 128, 24/20/20 for d = 64), pair
+ * j of an n-dim axis turning by
  * pos * 10000^(-2j/n); the block score is the raw dot product of block means;
  * local_range is an odd window diameter in blocks applied as a Chebyshev
  * distance over (block row, block column), clipped at the frame edge and the
@@ -92,7 +93,7 @@ typedef enum {
 typedef struct lcsa_config {
   int batch;            /* >= 1 */
   int heads;            /* 1 .. 16 */
-  int head_dim;         /* 128 */
+  int head_dim;         /* 128 (the pages' size) or 64 */
   int q_frames;         /* >= 1; the last q_frames of the KV window */
   int kv_frames;        /* >= q_frames (equal: self-attention over the chunk) */
   int grid_h, grid_w;   /* latent token grid per frame (H' = H/16, W' = W/16) */
@@ -141,7 +142,7 @@ LCSA_API void lcsa_config_default(lcsa_config_t* cfg);
    a negative or non-finite softmax_scale, kv_frame_offset < 0, a budget of 0
    blocks, heads_total < heads), LCSA_ERR_SHAPE (kv_frames < q_frames, or a
    token grid the block does not divide) or LCSA_ERR_UNSUPPORTED (head_dim
-   other than 128, more heads than the kernels take, blocks of other than 64
+   other than 64 or 128, more heads than the kernels take, blocks of other than 64
    or 128 tokens or more than 8 token rows, a tensor of more than 2^40
    elements, a window larger than the selection's candidate limit). Sizes are
    bounded before any product of them is formed. */

@@ -62,6 +62,17 @@ def test_resolved_geometry_matches_the_oracle(name):
     assert geo.selected_flops == geo.nnz * 4 * og.nb * og.nb * og.head_dim
 
 
+def test_head_dim_64_resolves():
+    """head_dim 64 (the ABI's other head size): 24 / 20 / 20 RoPE dims, the
+    softmax scale 1/8, the budget and window as for 128."""
+    cfg = _cfg(head_dim=64)
+    g = L.lcsa_config_resolve(cfg)
+    ref = L.lcsa_config_resolve(_cfg())
+    assert g.channels == cfg.heads * 64
+    assert (g.topk, g.nnz, g.rows, g.max_window) == (ref.topk, ref.nnz, ref.rows, ref.max_window)
+    assert g.selected_flops * 2 == ref.selected_flops
+
+
 def test_stream_chunk_numbers():
     geo = L.lcsa_config_resolve(L.config_from_workload(synth.WORKLOADS["stream_768x1280"]))
     assert (geo.q_tokens, geo.kv_tokens, geo.q_blocks, geo.kv_blocks, geo.topk) == (7680, 23040, 60, 180, 60)
@@ -91,7 +102,8 @@ def _cfg(**over):
     (dict(grid_w=20), L.LCSA_ERR_SHAPE),                           # ragged block column
     (dict(grid_h=12), L.LCSA_ERR_SHAPE),                           # ragged block row
     (dict(block_t=2, q_frames=1, kv_frames=2), L.LCSA_ERR_SHAPE),
-    (dict(head_dim=64), L.LCSA_ERR_UNSUPPORTED),
+    (dict(head_dim=96), L.LCSA_ERR_UNSUPPORTED),                   # head_dim 64 and 128 only
+    (dict(head_dim=256), L.LCSA_ERR_UNSUPPORTED),
     (dict(heads=17), L.LCSA_ERR_UNSUPPORTED),
     (dict(block_w=4), L.LCSA_ERR_UNSUPPORTED),                     # 32-token blocks
     (dict(block_h=16, block_w=8, grid_h=32), L.LCSA_ERR_UNSUPPORTED),  # 16 token rows per block

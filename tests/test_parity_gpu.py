@@ -37,8 +37,18 @@ SMALL = {
                                   local_range=3, topk=4, kv_frame_offset=1, field=True, unit_gain=False, seed=5),
     "budget_from_ratio": _T.replace(heads=2, q_frames=2, kv_frames=6, grid_h=48, grid_w=80, block_w=16,
                                     local_range=11, topk=0, sparse_ratio=0.25, field=True, unit_gain=False, seed=4),
+    # head_dim 64: RoPE dims 24 / 20 / 20, a tile one 64-column swizzle block wide
+    "d64_tiny": _T.replace(head_dim=64),
+    "d64_head_scope": _T.replace(head_dim=64, heads=4, field=True, unit_gain=False, seed=8),
+    "d64_blocks128": _T.replace(head_dim=64, heads=4, q_frames=1, kv_frames=3, grid_h=24, grid_w=48, block_w=16,
+                                local_range=3, topk=5, kv_frame_offset=2, field=True, unit_gain=False, seed=9),
+    "d64_blocks64_odd_heads": _T.replace(head_dim=64, heads=5, q_frames=2, kv_frames=4, grid_h=32, grid_w=40,
+                                         local_range=5, topk=9, field=True, unit_gain=False, seed=10),
+    "d64_k1_split_blocks": _T.replace(head_dim=64, heads=2, q_frames=1, kv_frames=2, grid_h=64, grid_w=128,
+                                      block_w=16, local_range=3, topk=4, kv_frame_offset=1, field=True,
+                                      unit_gain=False, seed=11),
 }
-OVERRIDES = {"tiny_head_scope": dict(norm_scope=1)}
+OVERRIDES = {"tiny_head_scope": dict(norm_scope=1), "d64_head_scope": dict(norm_scope=1)}
 
 _inputs = {}
 

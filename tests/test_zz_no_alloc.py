@@ -26,6 +26,8 @@ CASES = {
     "tiny": _T,
     "stream_small": _T.replace(heads=3, q_frames=1, kv_frames=3, grid_h=24, grid_w=48, block_w=16, local_range=3,
                                topk=5, kv_frame_offset=2, field=True, unit_gain=False),
+    "blocks64_d64": _T.replace(head_dim=64, heads=4, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5,
+                               topk=9, field=True, unit_gain=False, seed=13),
 }
 
 
