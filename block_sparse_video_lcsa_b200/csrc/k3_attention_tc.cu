@@ -154,6 +154,7 @@ struct TcParams {
   unsigned* err;
   int rows;
   unsigned* work_counter;  // zero at launch; each CTA takes work items from it
+  int item_lo, item_hi;    // this launch's work items (rows or pairs item_lo .. item_hi - 1)
   int stall_site;          // test-only build: 0, or where the first work item stalls
 };
 
@@ -418,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       return p.rows;
     int rr = 0;
     if (lane == 0) {
-      rr = int(atomicAdd(p.work_counter, 1u));
+      rr = p.item_lo + int(atomicAdd(p.work_counter, 1u));
+      if (rr >= p.item_hi) rr = p.rows;  // past this launch's items: the end
       bars->item[slot] = rr;
       mbar_arrive(bar(bars->item_full[slot]));
     }
@@ -1042,6 +1044,9 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.scale_log2 = p.scale_log2;
   tp.err = p.err;
   tp.rows = paired ? p.npairs : p.g.B * p.g.Hn * p.g.nQB;
+  tp.item_lo = p.item_lo;
+  tp.item_hi = p.item_hi > 0 ? p.item_hi : tp.rows;
+  if (tp.item_lo < 0 || tp.item_hi > tp.rows || tp.item_lo >= tp.item_hi) return cudaErrorInvalidValue;
   tp.work_counter = p.work_counter;
   if (!tp.work_counter) return cudaErrorInvalidValue;
   tp.pair_col = p.pair_col;
@@ -1053,7 +1058,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.stall_site = g_stall_site;
   g_stall_site = 0;
 #endif
-  const int grid = tp.rows < num_sms ? tp.rows : num_sms;
+  const int items = tp.item_hi - tp.item_lo;
+  const int grid = items < num_sms ? items : num_sms;
   kern<<<grid, kThreads, smem, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();
 }

@@ -159,6 +159,11 @@ struct lcsa_plan {
   // tcgen05 attention: tensor maps of the plan-owned q^ / k^; SM count (persistent grids)
   CUtensorMap tm_q, tm_k;
   int num_sms = 0;
+  // host-IO plans: a copy stream and the events that order it against the
+  // call's stream (q/k uploaded, V uploaded, first attention half done,
+  // first half of the output downloaded)
+  cudaStream_t io_stream = nullptr;
+  cudaEvent_t ev_qk = nullptr, ev_v = nullptr, ev_k3a = nullptr, ev_outa = nullptr;
   unsigned fault_launch = 0;                       // LCSA_FAULT launch:K (kFault* bits)
   bool fault_copy = false;                         // LCSA_FAULT copy
   std::vector<std::array<cudaEvent_t, 4>> evsets;  // timing ring
@@ -178,6 +183,9 @@ void release(lcsa_plan* p) {
     for (auto e : set)
       if (e) cudaEventDestroy(e);
   p->evsets.clear();
+  for (cudaEvent_t e : {p->ev_qk, p->ev_v, p->ev_k3a, p->ev_outa})
+    if (e) cudaEventDestroy(e);
+  if (p->io_stream) cudaStreamDestroy(p->io_stream);
 }
 
 // Host-side fault injection for tests of the error paths (no GPU fault is
@@ -364,6 +372,15 @@ lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Fault
       delete p;
       return st;
     }
+    if ((e = cudaStreamCreateWithFlags(&p->io_stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&p->ev_qk, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&p->ev_v, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&p->ev_k3a, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&p->ev_outa, cudaEventDisableTiming)) != cudaSuccess) {
+      release(p);
+      delete p;
+      return cuda_fail(e, "host-IO stream and events");
+    }
   }
   if ((e = cudaMemcpy(p->row_ptr, p->res.row_ptr.data(), (rows + 1) * 4, cudaMemcpyHostToDevice)) != cudaSuccess ||
       (e = cudaMemset(p->err, 0, 256)) != cudaSuccess ||
@@ -429,6 +446,9 @@ struct StepBlocks {
   int slot0_fb = 0;     // ring slot of window frame-block 0
   const void* v_attn = nullptr;  // raster v seen by K3 (caller's tensor or the ring)
   const float* ss_ext = nullptr; // head-sharded token-scope norm: reduced per-token sums of squares
+  cudaEvent_t k3_wait = nullptr; // an event K3 waits for (the host-IO call's V upload)
+  int k3_split = 0;              // > 0: K3 as two launches, work items [0, k3_split) and the rest,
+  cudaEvent_t k3_first_done = nullptr;  // recorded between them
 };
 
 lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float* gamma_q, const float* gamma_k,
@@ -547,6 +567,20 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     CUtensorMap tm_v;
     if ((e = lcsa::make_raster_map(&tm_v, sb.v_attn, g)) != cudaSuccess) return cuda_fail(e, "V tensor map");
     if (lcsa_status_t st = injected_launch_failure(p, kFaultK3, "attention")) return st;
+    if (sb.k3_wait && (e = cudaStreamWaitEvent(s, sb.k3_wait, 0)) != cudaSuccess) return cuda_fail(e, "wait for V");
+    if (sb.k3_split > 0) {
+      // two launches over the two halves of the work items, each with its own
+      // zeroed work counter; the event between them lets the caller start on
+      // the first half's output
+      k3.item_lo = 0;
+      k3.item_hi = sb.k3_split;
+      if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
+        return cuda_fail(e, "attention launch");
+      if ((e = cudaEventRecord(sb.k3_first_done, s)) != cudaSuccess) return cuda_fail(e, "event");
+      k3.item_lo = sb.k3_split;
+      k3.item_hi = 0;  // to the end
+      k3.work_counter += 1;
+    }
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
       return cuda_fail(e, "attention launch");
   }
@@ -726,6 +760,8 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
                                 const float* gamma_k, void* out, void* stream) {
   if (!p) return fail(LCSA_ERR_INVALID_ARG, "plan is null");
   if (!p->cfg.host_io) return fail(LCSA_ERR_INVALID_ARG, "plan was created without host_io");
+  if (sharded_token_norm(p))
+    return fail(LCSA_ERR_INVALID_ARG, "a head-sharded plan with token-scope norm takes lcsa_forward_sharded");
   if (!q || !k || !v || !gamma_q || !gamma_k || !out) return fail(LCSA_ERR_INVALID_ARG, "null host pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSetDevice(p->device);
@@ -733,16 +769,49 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
   const lcsa::Grid& g = p->res.grid;
   const size_t qb = size_t(g.B) * g.Lq * g.C * 2, kb = size_t(g.B) * g.Lkv * g.C * 2, gb = size_t(g.C) * 4;
   if (p->fault_copy) return fail(LCSA_ERR_CUDA, "host-to-device copy: injected failure (LCSA_FAULT)");
-  if ((e = cudaMemcpyAsync(p->st_q, q, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+  // The copies share one link, so they go in the order the kernels need
+  // them: gains, q and k on the call's stream (K1 and K2 start as soon as
+  // they are in), then v on the plan's copy stream while K1 and K2 run.
+  if ((e = cudaMemcpyAsync(p->st_gq, gamma_q, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_gk, gamma_k, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_q, q, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
       (e = cudaMemcpyAsync(p->st_k, k, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(p->st_gq, gamma_q, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(p->st_gk, gamma_k, gb, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+      (e = cudaEventRecord(p->ev_qk, s)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(p->io_stream, p->ev_qk, 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, p->io_stream)) != cudaSuccess ||
+      (e = cudaEventRecord(p->ev_v, p->io_stream)) != cudaSuccess)
     return cuda_fail(e, "host-to-device copy");
-  lcsa_status_t st = lcsa_forward(p, p->st_q, p->st_k, p->st_v, p->st_gq, p->st_gk, p->st_out, stream);
+  // K3 waits for v. With one batch element and at least two heads it runs as
+  // two launches over the first and the second half of the heads (rows, or
+  // query-block pairs, are numbered head-major), and the first half's output
+  // channels go back on the copy stream while the second half computes.
+  StepBlocks sb;
+  sb.k_in_fb = g.Tkv / g.bt;
+  sb.v_attn = p->st_v;
+  sb.k3_wait = p->ev_v;
+  const int heads_a = g.B == 1 && g.Hn >= 2 ? g.Hn / 2 : 0;
+  if (heads_a > 0) {
+    const int64_t per_head = p->pair_col ? lcsa::pair_count(g) / g.Hn : int64_t(g.nQB);
+    sb.k3_split = int(heads_a * per_head);
+    sb.k3_first_done = p->ev_k3a;
+  }
+  lcsa_status_t st = run_step(p, p->st_q, p->st_k, p->st_gq, p->st_gk, p->st_out, s, sb);
   if (st != LCSA_OK) return st;
-  if ((e = cudaMemcpyAsync(out, p->st_out, qb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+  const size_t pitch = size_t(g.C) * 2, head_bytes = size_t(g.D) * 2;
+  if (heads_a > 0) {
+    if ((e = cudaStreamWaitEvent(p->io_stream, p->ev_k3a, 0)) != cudaSuccess ||
+        (e = cudaMemcpy2DAsync(out, pitch, p->st_out, pitch, heads_a * head_bytes, size_t(g.Lq),
+                               cudaMemcpyDeviceToHost, p->io_stream)) != cudaSuccess ||
+        (e = cudaEventRecord(p->ev_outa, p->io_stream)) != cudaSuccess ||
+        (e = cudaMemcpy2DAsync(static_cast<char*>(out) + heads_a * head_bytes, pitch,
+                               static_cast<const char*>(static_cast<const void*>(p->st_out)) + heads_a * head_bytes,
+                               pitch, (g.Hn - heads_a) * head_bytes, size_t(g.Lq), cudaMemcpyDeviceToHost, s)) !=
+            cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, p->ev_outa, 0)) != cudaSuccess)
+      return cuda_fail(e, "device-to-host copy");
+  } else if ((e = cudaMemcpyAsync(out, p->st_out, qb, cudaMemcpyDeviceToHost, s)) != cudaSuccess) {
     return cuda_fail(e, "device-to-host copy");
+  }
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
   return take_device_error(p);
 }

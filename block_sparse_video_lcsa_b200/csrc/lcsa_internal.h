@@ -15,9 +15,10 @@ constexpr int kMaxHeadDim = 128;     // head sizes the kernels implement: 64 and
 constexpr int kMaxHeads = 16;
 constexpr int kMaxCandidates = 4096; // admissible blocks per query block (K2 sort)
 constexpr int kMaxK1Ctas = 256;      // K1 persistent grid cap (sizes its split-block buffers)
-// The plan's counter array: K1's kMaxK1Ctas merge counters, then K3's work
-// counter; K2 zeroes all of them (after K1 has used its own, before K3 starts).
-constexpr int kCounters = kMaxK1Ctas + 1;
+// The plan's counter array: K1's kMaxK1Ctas merge counters, then K3's two
+// work counters (a call may run K3 as two launches over halves of the work
+// items); K2 zeroes all of them (after K1 has used its own, before K3 starts).
+constexpr int kCounters = kMaxK1Ctas + 2;
 
 // Device error word codes (first word of the plan's error buffer).
 constexpr unsigned kDevErrNone = 0;
@@ -183,6 +184,9 @@ struct K3Params {
   const int* pair_len;
   int pair_cap;
   unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work items from it
+  // Work items item_lo .. item_hi - 1 (rows, or query-block pairs); both 0:
+  // all of them
+  int item_lo, item_hi;
 };
 
 // Sizes of one configuration (lcsa_config.cu), derived without touching the
