@@ -35,8 +35,13 @@
 //           with barrier waits in between was measured to issue at half the
 //           pipe's rate, and issuing from an elected lane instead of a lane-0
 //           branch measured 1.5-3.5 % faster. The two streams are ordered
-//           only through mbarriers: S of block j+3 waits until P.V of block
-//           j (which reads P_j from the same buffer) has completed.
+//           through mbarriers: S of block j+3 waits until P.V of block j
+//           (which reads P_j from the same buffer) has been issued, not until
+//           it has completed. The tensor pipe runs a CTA's products in the
+//           order they reach it, so P.V_j reads P_j before S_{j+3} writes
+//           the buffer, and completes before it; the issuing warp's
+//           tcgen05.fence::before_thread_sync, the mbarrier and the S
+//           issuer's fence::after_thread_sync order the two warps' issues.
 //   warps 3-10 softmax, two groups of four (one warp per TMEM lane quarter):
 //           the KV tiles of the CTA's work go to the groups in turn, and a
 //           group's warp handles all 128 keys of its quarter's 32 rows, so
@@ -62,7 +67,8 @@
 // thread has already read).
 // Shared memory: Q 32 KB, K^ ring 2 x 32 KB, V ring 3 x 32 KB, all in the
 // 128-byte swizzled layout that TMA writes and the MMA descriptors read. The
-// producer fetches K^ two blocks ahead of V (K^_{j+2} before V_j), matching
+// producer fetches K^ as many blocks ahead of V as the K^ ring has stages
+// (K^_{j+2} before V_j), matching
 // the order in which the issuers consume them.
 //
 // Every wait on an mbarrier is bounded (wall-clock limit); a wait that runs
@@ -123,7 +129,8 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[kSBufs], p_full[kSBufs], s_free[kSBufs];
+  uint64_t s_full[kSBufs], p_full[kSBufs];
+  uint64_t pv_issued[kSBufs];  // P.V of the buffer's tile issued (one arrival per tile)
   uint64_t o_done[2];  // o_done[g & 1]: P.V number g (counted per CTA) and all before it have completed
   uint64_t o_free, mma_drain[2];
   uint64_t pair[4];  // end-of-row sum exchange between the two softmax warps of a lane quarter
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(bars->s_full[s]), 1);
       mbar_init(bar(bars->p_full[s]), kSoftmaxWarps / 2);
-      mbar_init(bar(bars->s_free[s]), 1);
+      mbar_init(bar(bars->pv_issued[s]), 1);
     }
     mbar_init(bar(bars->o_done[0]), 1);
     mbar_init(bar(bars->o_done[1]), 1);
@@ -534,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           e.f0 = b * g.Tkv + slot * g.bt;
         }
       };
-      Entries ke, ve;  // cursors of the K loads (two steps ahead) and of the V loads
+      Entries ke, ve;  // cursors of the K loads (kKStages steps ahead) and of the V loads
       // entry of the selected block feeding sub-tile i of step st (an odd last
       // step repeats its block; the softmax masks the copy)
       auto entry = [&](Entries& e, int st, int i) -> int {
@@ -561,9 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         k_issued = kvj + 1;
         return true;
       };
-      for (int st = 0; st < 2 && st < steps && ok; ++st) ok = load_k(st);
+      for (int st = 0; st < kKStages && st < steps && ok; ++st) ok = load_k(st);
       for (int st = 0; st < steps && ok; ++st) {
-        if (st + 2 < steps && !(ok = load_k(st + 2))) break;
+        if (st + kKStages < steps && !(ok = load_k(st + kKStages))) break;
         const int kvj = kv + st, vs = kvj % kVStages, vu = kvj / kVStages;
         if (vu > 0 && !(ok = warp_wait(bar(bars->v_empty[vs]), (vu - 1) & 1, abort, p.err, 3))) break;
         const uint32_t vdst = base + L::v + vs * L::tile;
@@ -634,9 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
         const int kvj = kv + j, ks = kvj % kKStages;
-        // buffer sb last held P of block s_it - 3: its P.V must have completed
+        // buffer sb last held P of block s_it - 3: its P.V must have been
+        // issued (the pipe then reads P before this S overwrites it)
         if (s_it >= kSBufs &&
-            !(ok = warp_wait(bar(bars->s_free[sb]), ((s_it / kSBufs) - 1) & 1, abort, p.err, 11)))
+            !(ok = warp_wait(bar(bars->pv_issued[sb]), ((s_it / kSBufs) - 1) & 1, abort, p.err, 11)))
           break;
         if (!(ok = warp_wait(bar(bars->k_full[ks]), (kvj / kKStages) & 1, abort, p.err, 12))) break;
         tc_fence_after();
@@ -688,14 +696,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tmem + kColO, pa + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), sdesc(va + kk * 2048, kHalfBytes, 1024),
                    id_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
-          // o_done first: the softmax's parity waits on o_done rely on a
-          // product's o_done arrival having happened once its s_free arrival
-          // (which lets S of a later block start) has been seen
           mma_commit(bar(bars->o_done[pv_it & 1]));
-          mma_commit(bar(bars->s_free[pb]));
           mma_commit(bar(bars->v_empty[vs]));
         }
+        // the products above are issued: S of tile pv_it + 3 may go into
+        // this buffer (the fence orders them before the arrival)
+        tc_fence_before();
         __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->pv_issued[pb]));
         issued = true;
       }
       kv += n;
@@ -847,8 +855,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         l += rsum.x + rsum.y;
         // O is rescaled when this tile raised the maximum, once every earlier
         // P.V of the row has completed; the last of them is P.V number
-        // gp = s_it - 1, and P.V gp - 2 has completed (S of this tile was
-        // issued only after it), so the parity wait is unambiguous
+        // gp = s_it - 1, and P.V gp - 2 has completed (it was issued before
+        // S of this tile, which has completed, and products complete in
+        // issue order), so the parity wait is unambiguous
         if (j >= 1 && __any_sync(0xffffffffu, need)) {
           const float alpha = need ? exp2_mufu(m_prev - m_used) : 1.f;
           const int gp = s_it - 1;
@@ -886,8 +895,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // barrier is at most one phase short of the target: o_done[gp & 1]
         // last completed for P.V gp - 2, which nothing may have waited for.
         // So P.V gp - 1 is waited for first: its barrier's previous phase,
-        // P.V gp - 3, completed before S of tile gp was issued, and its
-        // completion implies gp - 2's.
+        // P.V gp - 3, was issued before S of tile gp and so has completed
+        // (this group saw S of tile gp complete, directly or through the
+        // other group's published maximum), and its completion implies
+        // gp - 2's.
         const int gp = s_last;
         if (gp >= 1 && !(ok = warp_wait(bar(bars->o_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, abort, p.err, 25)))
           break;
