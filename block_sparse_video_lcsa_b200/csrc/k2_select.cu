@@ -239,31 +239,78 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const K2Params p) {
   if (p.reuse && threadIdx.x == kThreads - 1) p.row_len[rr] = pos;  // the last thread's end is the row's count
 }
 
-// Union of the selections of two query blocks, ascending: a byte per KV
-// block marks which of the two kept it (bit 0 the first, bit 1 the second),
-// then a block scan emits the marked blocks with their marks.
+// Union of the selections of two query blocks, ascending. A byte per KV
+// block marks which candidate rows kept it (bit i for r[i]); in a 2 x 2
+// group the two CTAs of the group's pairs both mark all four rows, count the
+// unions of either split (columns: r0+r2, r1+r3; rows: r0+r1, r2+r3) and so
+// take the same decision; then a block scan emits this pair's union, each
+// entry marked with which of its two rows kept it (bit 0 the first, bit 1
+// the second), and the pair's rows are recorded for K3.
 __global__ void __launch_bounds__(kThreads) pair_union_kernel(const PairParams p) {
-  extern __shared__ unsigned char mark[];  // [nkb]
+  extern __shared__ unsigned mark_words[];  // [ceil(nkb / 4)]: byte c of the array is block c's mark
+  const unsigned char* mark = reinterpret_cast<const unsigned char*>(mark_words);
   __shared__ int warp_sum[kWarps];
+  __shared__ int split_sum[2][kWarps];
   const int pr = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = threadIdx.x; c < p.nkb; c += kThreads) mark[c] = 0;
+  for (int c = threadIdx.x; c < (p.nkb + 3) / 4; c += kThreads) mark_words[c] = 0u;
   __syncthreads();
-  int rows2[2];
-  pair_rows(p.g, pr, rows2[0], rows2[1]);
-#pragma unroll 1
-  for (int side = 0; side < 2; ++side) {
-    const int row = rows2[side];
+  int r[4], slot;
+  pair_candidates(p.g, pr, r, slot);
+  // the rows' entries all at once: each sets its own bit of the block's byte
+#pragma unroll
+  for (int side = 0; side < 4; ++side) {
+    const int row = r[side];
     if (row >= 0) {
       const int64_t beg = p.row_len ? int64_t(row) * p.pad_cap : int64_t(p.row_ptr[row]);
       const int n = p.row_len ? p.row_len[row] : p.row_ptr[row + 1] - p.row_ptr[row];
-      for (int i = threadIdx.x; i < n; i += kThreads) mark[p.col_idx[beg + i]] |= (unsigned char)(1u << side);
+      for (int i = threadIdx.x; i < n; i += kThreads) {
+        const int c = p.col_idx[beg + i];
+        atomicOr(&mark_words[c >> 2], 1u << ((c & 3) * 8 + side));
+      }
     }
-    __syncthreads();  // one side's blocks are distinct; the sides run one after the other
   }
+  __syncthreads();
   const int span = (p.nkb + kThreads - 1) / kThreads;
   const int c_beg = min(int(threadIdx.x) * span, p.nkb), c_end = min(c_beg + span, p.nkb);
+  // the pair's two rows as bits of mark[]
+  unsigned first = 1u, second = 2u;
+  int ra = r[0], rb = r[1];
+  if (slot >= 0) {
+    int by_cols = 0, by_rows = 0;
+    for (int c = c_beg; c < c_end; ++c) {
+      const unsigned m = mark[c];
+      by_cols += ((m & 5u) != 0) + ((m & 10u) != 0);
+      by_rows += ((m & 3u) != 0) + ((m & 12u) != 0);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      by_cols += __shfl_xor_sync(0xffffffffu, by_cols, o);
+      by_rows += __shfl_xor_sync(0xffffffffu, by_rows, o);
+    }
+    if (lane == 0) {
+      split_sum[0][warp] = by_cols;
+      split_sum[1][warp] = by_rows;
+    }
+    __syncthreads();
+    int tot_cols = 0, tot_rows = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      tot_cols += split_sum[0][w];
+      tot_rows += split_sum[1][w];
+    }
+    if (tot_rows < tot_cols) {  // left with right
+      first = slot ? 4u : 1u;
+      second = slot ? 8u : 2u;
+      ra = slot ? r[2] : r[0];
+      rb = slot ? r[3] : r[1];
+    } else {  // top with bottom
+      first = slot ? 2u : 1u;
+      second = slot ? 8u : 4u;
+      ra = slot ? r[1] : r[0];
+      rb = slot ? r[3] : r[2];
+    }
+  }
   int cnt = 0;
-  for (int c = c_beg; c < c_end; ++c) cnt += mark[c] != 0;
+  for (int c = c_beg; c < c_end; ++c) cnt += (mark[c] & (first | second)) != 0;
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -275,17 +322,23 @@ __global__ void __launch_bounds__(kThreads) pair_union_kernel(const PairParams p
   int pos = incl - cnt;
   for (int w = 0; w < warp; ++w) pos += warp_sum[w];
   int* dst = p.pair_col + int64_t(pr) * p.pair_cap;
-  for (int c = c_beg; c < c_end; ++c)
-    if (mark[c]) dst[pos++] = c | (int(mark[c]) << kPairShift);
-  if (threadIdx.x == kThreads - 1) p.pair_len[pr] = pos;
+  for (int c = c_beg; c < c_end; ++c) {
+    const unsigned m = mark[c];
+    const int two = ((m & first) ? 1 : 0) | ((m & second) ? 2 : 0);
+    if (two) dst[pos++] = c | (two << kPairShift);
+  }
+  if (threadIdx.x == kThreads - 1) {
+    p.pair_len[pr] = pos;
+    p.pair_rows[pr] = make_int2(ra, rb);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_pair_union(const PairParams& p, cudaStream_t s) {
   if (p.npairs <= 0) return cudaSuccess;
-  if (p.nkb > 48 * 1024) return cudaErrorInvalidValue;
-  pair_union_kernel<<<p.npairs, kThreads, size_t(p.nkb), s>>>(p);
+  if (p.nkb > 48 * 1024 - 256) return cudaErrorInvalidValue;  // marks + the kernel's static arrays in 48 KB
+  pair_union_kernel<<<p.npairs, kThreads, size_t((p.nkb + 3) / 4) * 4, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -155,6 +155,7 @@ struct TcParams {
   int pad_cap;
   const int* pair_col;  // paired 64-token query blocks: union lists (entries kb | marks << kPairShift)
   const int* pair_len;
+  const int2* pair_rows;  // each pair's two query blocks (second -1: a single block)
   int pair_cap;
   __nv_bfloat16* out;
   float scale_log2;
@@ -506,8 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = list_count<PAIR>(p, rr);
       int ra = rr, rb = rr;  // the query block(s) of this work item
       if constexpr (PAIR) {
-        pair_rows(g, rr, ra, rb);
-        if (rb < 0) rb = ra;  // a single block fills both halves; the second is not written out
+        const int2 two = p.pair_rows[rr];
+        ra = two.x;
+        rb = two.y < 0 ? two.x : two.y;  // a single block fills both halves; the second is not written out
       }
       const int bhh = ra / g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
@@ -916,12 +918,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int qrow = rr, m_tok = row_in_tile;  // query block (row) and token of this lane's row
       bool store = true;
       if constexpr (PAIR) {
-        int ra, rb;
-        pair_rows(g, rr, ra, rb);
-        qrow = sp < 2 ? ra : rb;
+        const int2 two = p.pair_rows[rr];
+        qrow = sp < 2 ? two.x : two.y;
         m_tok = row_in_tile & (NBLK - 1);
         store = qrow >= 0;  // a single block's second half is a copy
-        qrow = store ? qrow : ra;
+        qrow = store ? qrow : two.x;
       }
       const int bhh = qrow / g.nQB, qb = qrow % g.nQB;
       const int b = bhh / g.Hn, h = bhh % g.Hn;
@@ -1062,6 +1063,7 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   if (!tp.work_counter) return cudaErrorInvalidValue;
   tp.pair_col = p.pair_col;
   tp.pair_len = p.pair_len;
+  tp.pair_rows = p.pair_rows;
   tp.pair_cap = p.pair_cap;
   tp.ring_fb = p.ring_fb;
   tp.slot0_fb = p.slot0_fb;

@@ -98,7 +98,7 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   ws += size_t(rows) * (8 + size_t(wmax) * 4);                                    // threshold reuse
   if (nb == 64) {                                                                 // query-block pairs
     const size_t cap = size_t(2 * wmax < g.nKB ? 2 * wmax : g.nKB);
-    ws += size_t(lcsa::pair_count(g)) * (cap + 1) * 4;
+    ws += size_t(lcsa::pair_count(g)) * (cap + 3) * 4;                          // lists, counts, rows
   }
   ws += rope_n * sizeof(float2) + 256;
   ws += size_t(lcsa::kMaxK1Ctas) * 2 * size_t(g.C) * 4 + size_t(lcsa::kCounters) * 4;  // K1 split blocks, counters
@@ -142,6 +142,7 @@ struct lcsa_plan {
   // 64-token blocks: pairs of query blocks as one 128-row tile (union lists)
   int32_t* pair_col = nullptr;
   int32_t* pair_len = nullptr;
+  int2* pair_rows = nullptr;
   int npairs = 0, pair_cap = 0;
   bool reuse_mode = false;   // lcsa_plan_set_threshold_reuse
   bool have_thresh = false;  // a selecting call has recorded thresholds
@@ -176,7 +177,7 @@ void release(lcsa_plan* p) {
   void* ptrs[] = {p->v_ring, p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
                   p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
                   p->st_v,  p->st_out,  p->st_gq,    p->st_gk,    p->thresh,     p->row_len, p->col_pad,
-                  p->pair_col, p->pair_len};
+                  p->pair_col, p->pair_len,  p->pair_rows};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (auto& set : p->evsets)
@@ -261,6 +262,7 @@ lcsa_status_t alloc_pairs(lcsa_plan* p) {
   p->pair_cap = pair_capacity(p->res);
   lcsa_status_t st = dev_alloc(&p->pair_col, size_t(np) * size_t(p->pair_cap) * 4, "pair lists");
   if (st == LCSA_OK) st = dev_alloc(&p->pair_len, size_t(np) * 4, "pair counts");
+  if (st == LCSA_OK) st = dev_alloc(&p->pair_rows, size_t(np) * sizeof(int2), "pair rows");
   return st;
 }
 
@@ -516,6 +518,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k3.npairs = p->npairs;
   k3.pair_col = p->pair_col;
   k3.pair_len = p->pair_len;
+  k3.pair_rows = p->pair_rows;
   k3.pair_cap = p->pair_cap;
   k3.work_counter = p->split_cnt + lcsa::kMaxK1Ctas;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
@@ -555,6 +558,7 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     pp.nkb = g.nKB;
     pp.pair_col = p->pair_col;
     pp.pair_len = p->pair_len;
+    pp.pair_rows = p->pair_rows;
     pp.pair_cap = p->pair_cap;
     if (lcsa_status_t st = injected_launch_failure(p, kFaultPair, "pair union")) return st;
     if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return cuda_fail(e, "pair union launch");

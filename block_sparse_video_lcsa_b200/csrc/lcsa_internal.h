@@ -119,36 +119,56 @@ struct K2Params {
 // Pairs of neighbouring 64-token query blocks (same batch, head and frame
 // group) that K3 computes as one 128-row tile over the union of their
 // selected blocks, each entry kb | (which of the two selected it) <<
-// kPairShift. Within a frame group's nHb x nWb block grid, block rows 2i and
-// 2i+1 pair column by column; an odd last block row pairs columns 2j and
-// 2j+1; an odd last column of it stays single.
+// kPairShift. A frame group's nHb x nWb block grid is cut into 2 x 2 groups
+// of blocks; each group splits into two pairs either by columns (top with
+// bottom) or by rows (left with right), whichever gives the smaller total
+// union (the pair-union kernel decides from the selections and records each
+// pair's two rows; a tie keeps columns). An odd last column pairs its blocks
+// top with bottom, an odd last block row left with right, and a block left
+// over in both stays single.
 constexpr int kPairShift = 28;
 __host__ __device__ inline int pairs_per_group(const Grid& g) {
-  return (g.nHb / 2) * g.nWb + (g.nHb % 2) * ((g.nWb + 1) / 2);
+  return 2 * (g.nHb / 2) * (g.nWb / 2) + (g.nWb % 2) * (g.nHb / 2) + (g.nHb % 2) * ((g.nWb + 1) / 2);
 }
 __host__ __device__ inline int64_t pair_count(const Grid& g) {
   return int64_t(g.B) * g.Hn * (g.nQB / g.bpf) * pairs_per_group(g);
 }
-// rows (batch, head, query block) of pair pr; the second is -1 for a single block
-__host__ __device__ inline void pair_rows(const Grid& g, int64_t pr, int& ra, int& rb) {
+// The rows (batch, head, query block) pair pr is chosen from. In a 2 x 2
+// group: the group's four rows (top left, top right, bottom left, bottom
+// right) and slot = which of the group's two pairs pr is (0 or 1). Otherwise
+// the pair's own rows in r[0], r[1] (r[1] = -1 for a single block), r[2] =
+// r[3] = -1 and slot = -1.
+__host__ __device__ inline void pair_candidates(const Grid& g, int64_t pr, int r[4], int& slot) {
   const int pg = pairs_per_group(g);
   const int64_t per_bh = int64_t(g.nQB / g.bpf) * pg;
   const int bh = int(pr / per_bh);
-  const int rem = int(pr % per_bh), tb = rem / pg, k = rem % pg;
-  int ha, wa, hb, wb;
-  if (k < (g.nHb / 2) * g.nWb) {
-    ha = 2 * (k / g.nWb);
-    hb = ha + 1;
-    wa = wb = k % g.nWb;
-  } else {
-    const int k2 = k - (g.nHb / 2) * g.nWb;
-    ha = hb = g.nHb - 1;
-    wa = 2 * k2;
-    wb = wa + 1;
-  }
+  const int rem = int(pr % per_bh), tb = rem / pg;
+  int k = rem % pg;
   const int base = bh * g.nQB + tb * g.bpf;
-  ra = base + ha * g.nWb + wa;
-  rb = wb < g.nWb ? base + hb * g.nWb + wb : -1;
+  const int in_groups = 2 * (g.nHb / 2) * (g.nWb / 2);
+  r[2] = r[3] = -1;
+  slot = -1;
+  if (k < in_groups) {
+    const int gi = k >> 1, gw = g.nWb / 2;
+    const int h0 = 2 * (gi / gw), w0 = 2 * (gi % gw);
+    r[0] = base + h0 * g.nWb + w0;
+    r[1] = r[0] + 1;
+    r[2] = r[0] + g.nWb;
+    r[3] = r[2] + 1;
+    slot = k & 1;
+    return;
+  }
+  k -= in_groups;
+  if (g.nWb % 2 && k < g.nHb / 2) {  // odd last column: top with bottom
+    r[0] = base + 2 * k * g.nWb + g.nWb - 1;
+    r[1] = r[0] + g.nWb;
+    return;
+  }
+  if (g.nWb % 2) k -= g.nHb / 2;
+  // odd last block row: left with right (the last of an odd row alone)
+  const int w0 = 2 * k;
+  r[0] = base + (g.nHb - 1) * g.nWb + w0;
+  r[1] = w0 + 1 < g.nWb ? r[0] + 1 : -1;
 }
 struct PairParams {
   Grid g;
@@ -160,6 +180,7 @@ struct PairParams {
   int nkb;                // KV blocks per (batch, head): the range of block indices
   int* pair_col;          // [npairs][pair_cap]
   int* pair_len;          // [npairs]
+  int2* pair_rows;        // [npairs] the pair's two rows (second -1: a single block)
   int pair_cap;
 };
 
@@ -182,6 +203,7 @@ struct K3Params {
   int npairs;
   const int* pair_col;
   const int* pair_len;
+  const int2* pair_rows;
   int pair_cap;
   unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work items from it
   // Work items item_lo .. item_hi - 1 (rows, or query-block pairs); both 0:

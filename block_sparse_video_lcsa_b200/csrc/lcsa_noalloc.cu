@@ -188,12 +188,13 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   const size_t off_pk = off_pq + round256(size_t(g.B) * g.Hn * g.nQB * D * 4);
   const size_t off_qh = off_pk + round256(size_t(g.B) * g.Hn * g.nKB * D * 4);
   const size_t off_kh = off_qh + round256(size_t(g.B) * g.Lq * g.C * 2);
-  // 64-token blocks: query-block pairs as 128-row tiles (union lists and counts)
+  // 64-token blocks: query-block pairs as 128-row tiles (union lists, counts and rows)
   const int64_t npairs = g.nb == 64 ? lcsa::pair_count(g) : 0;
   const int pair_cap = 2 * core.max_window < g.nKB ? 2 * core.max_window : g.nKB;
   const size_t off_pc = off_kh + round256(size_t(g.B) * g.Lkv * g.C * 2);
   const size_t off_pl = off_pc + round256(size_t(npairs) * size_t(pair_cap) * 4);
-  const size_t need = off_pl + round256(size_t(npairs) * 4);
+  const size_t off_pr = off_pl + round256(size_t(npairs) * 4);
+  const size_t need = off_pr + round256(size_t(npairs) * sizeof(int2));
   if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES)) return LCSA_ERR_UNSUPPORTED;  // create a plan instead
 
   int dev = 0;
@@ -219,6 +220,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   __nv_bfloat16* khat = reinterpret_cast<__nv_bfloat16*>(ws + off_kh);
   int* pair_col = npairs ? reinterpret_cast<int*>(ws + off_pc) : nullptr;
   int* pair_len = npairs ? reinterpret_cast<int*>(ws + off_pl) : nullptr;
+  int2* pair_rows = npairs ? reinterpret_cast<int2*>(ws + off_pr) : nullptr;
 
   // the counters start at zero (an aborted call may have left them set)
   if ((e = cudaMemsetAsync(split_cnt, 0, kOffAfterCnt - kOffCnt, s)) != cudaSuccess) return LCSA_ERR_CUDA;
@@ -290,6 +292,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
     pp.nkb = g.nKB;
     pp.pair_col = pair_col;
     pp.pair_len = pair_len;
+    pp.pair_rows = pair_rows;
     pp.pair_cap = pair_cap;
     if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
@@ -310,6 +313,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.pad_cap = 0;
   k3.pair_col = pair_col;
   k3.pair_len = pair_len;
+  k3.pair_rows = pair_rows;
   k3.npairs = int(npairs);
   k3.pair_cap = pair_cap;
   k3.work_counter = split_cnt + lcsa::kMaxK1Ctas;
