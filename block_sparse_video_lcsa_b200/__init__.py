@@ -197,7 +197,7 @@ def lcsa_plan_create_stream(cfg: lcsa_config_t, device: int = 0) -> "Plan":
     return Plan(h, cfg, int(device))
 
 
-LCSA_NOALLOC_WORKSPACE_BYTES = 32 << 20
+LCSA_NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 
 def lcsa_forward_noalloc(cfg: lcsa_config_t, q, k, v, gamma_q, gamma_k, out, stream=None) -> int:

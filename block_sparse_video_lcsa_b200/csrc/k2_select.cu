@@ -254,6 +254,11 @@ __global__ void __launch_bounds__(kThreads) pair_union_kernel(const PairParams p
   const int pr = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = threadIdx.x; c < (p.nkb + 3) / 4; c += kThreads) mark_words[c] = 0u;
   __syncthreads();
+  // the attention's merge state of cut pairs starts at zero
+  for (int i = pr * kThreads + threadIdx.x; i < p.cut * 8 * (1 + kCutParts); i += p.npairs * kThreads) {
+    if (i < p.cut * 8) p.merge_cnt[i] = 0u;
+    else p.merge_ready[i - p.cut * 8] = 0u;
+  }
   int r[4], slot;
   pair_candidates(p.g, pr, r, slot);
   // the rows' entries all at once: each sets its own bit of the block's byte

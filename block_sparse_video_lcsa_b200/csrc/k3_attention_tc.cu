@@ -17,11 +17,18 @@
 // one thread issues the MMAs, and P goes back to tensor memory as the A
 // operand of the P.V product.
 //
-// Persistent: one CTA per SM takes work items (rows (batch, head, query
-// block), or pairs of 64-token query blocks) from a global counter: the
-// producer warp draws the next item and hands it to the other roles through
-// a four-slot queue in shared memory, so CTAs that drew short items take
-// more. Roles (352 threads):
+// Persistent: one CTA per SM takes work entries from a global counter: the
+// producer warp draws the next one and hands it to the other roles through a
+// four-slot queue in shared memory, so CTAs that drew short entries take
+// more. An entry is a work item (a row (batch, head, query block), or a pair
+// of 64-token query blocks) or, for the last few pairs, one part of one (up
+// to kCutParts equal shares of its KV tiles): long items handed out whole
+// leave SMs idle at the end when their count is not a multiple of the SM
+// count. The parts of a cut pair run on whatever CTAs drew them; the last to
+// finish combines them: the others leave their part's O, row maxima and row
+// sums in global memory, and the last adds all parts in part order (the
+// online-softmax merge), so the result does not depend on which CTA finishes
+// first. Roles (352 threads):
 //   warp 0  TMA producer: Q tile of the row, then K^ / V blocks of its CSR list
 //           (K^ from the block-major prologue output, V straight from the
 //           raster input through a 5-D tensor map: d, head, x, y, frame).
@@ -139,7 +146,7 @@ struct Bars {
   // the global counter and hands it to the other roles through item[]
   uint64_t item_full[kItemSlots], item_empty[kItemSlots];
   uint64_t never;  // test-only build: a barrier nothing arrives on
-  int item[kItemSlots];
+  alignas(16) int4 item[kItemSlots];  // segment: item, first tile, end tile, part | parts << 16
   uint32_t tmem_base;
   int abort;
 };
@@ -161,8 +168,17 @@ struct TcParams {
   float scale_log2;
   unsigned* err;
   int rows;
-  unsigned* work_counter;  // zero at launch; each CTA takes work items from it
-  int item_lo, item_hi;    // this launch's work items (rows or pairs item_lo .. item_hi - 1)
+  // Work entries: item i < rows - cut_items is entry i; the parts of the
+  // last cut_items items (up to kCutParts each) follow, one entry per part.
+  // This launch runs entries entry_lo .. entry_hi - 1 (those of its items),
+  // taken from work_counter (zero at launch); a cut item's parts merge
+  // through the counters, ready flags and partial-result slots.
+  unsigned* work_counter;
+  int entry_lo, entry_hi;
+  int cut_items;
+  unsigned* merge_cnt;
+  unsigned* merge_ready;
+  float* part_buf;
   int stall_site;          // test-only build: 0, or where the first work item stalls
 };
 
@@ -235,6 +251,33 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
         return false;
       }
     }
+  }
+}
+
+// Flags between the CTAs that share a split work item: a release store
+// after the part's slice is written, and a bounded acquire poll (returns
+// false if the CTA is aborting or the limit passed, then records the error).
+__device__ __forceinline__ void flag_release(unsigned* f) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(1u) : "memory");
+}
+__device__ __noinline__ bool flag_wait(const unsigned* f, volatile int* abort, unsigned* err, unsigned site) {
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v) return true;
+    if ((i & 15u) == 15u) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        if (atomicCAS(err, kDevErrNone, kDevErrTimeout) == kDevErrNone) {
+          err[1] = site;
+          err[2] = blockIdx.x;
+        }
+        return false;
+      }
+    }
+    __nanosleep(64);
   }
 }
 
@@ -416,31 +459,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int KB = kNB / NBLK;
 
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
-  // Work item number `it` of this CTA, as every role sees it: the producer
-  // takes it from the global counter and publishes it in item[it % slots];
-  // the other roles read it there (one arrival per reader frees the slot).
-  // An item >= p.rows ends the CTA's work.
-  auto take_item = [&](int it, bool& ok) -> int {
+  // Segment number `it` of this CTA, as every role sees it: the producer
+  // takes it (take_item, below) and publishes it in item[it % slots]; the
+  // other roles read it there (one arrival per reader frees the slot). An
+  // item >= p.rows ends the CTA's work.
+  auto read_item = [&](int it, bool& ok) -> int4 {
     const int slot = it % kItemSlots;
-    if (it >= kItemSlots &&
-        !(ok = warp_wait(bar(bars->item_empty[slot]), ((it / kItemSlots) - 1) & 1, abort, p.err, 4)))
-      return p.rows;
-    int rr = 0;
-    if (lane == 0) {
-      rr = p.item_lo + int(atomicAdd(p.work_counter, 1u));
-      if (rr >= p.item_hi) rr = p.rows;  // past this launch's items: the end
-      bars->item[slot] = rr;
-      mbar_arrive(bar(bars->item_full[slot]));
-    }
-    return __shfl_sync(0xffffffffu, rr, 0);
-  };
-  auto read_item = [&](int it, bool& ok) -> int {
-    const int slot = it % kItemSlots;
-    if (!(ok = warp_wait(bar(bars->item_full[slot]), (it / kItemSlots) & 1, abort, p.err, 5))) return p.rows;
-    const int rr = static_cast<volatile int*>(bars->item)[slot];
+    if (!(ok = warp_wait(bar(bars->item_full[slot]), (it / kItemSlots) & 1, abort, p.err, 5)))
+      return make_int4(p.rows, 0, 0, 0);
+    const volatile int* w = reinterpret_cast<const volatile int*>(&bars->item[slot]);
+    const int4 sg = make_int4(w[0], w[1], w[2], w[3]);
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(bars->item_empty[slot]));
-    return rr;
+    return sg;
   };
 
   if (threadIdx.x == 0) {
@@ -499,9 +530,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int kv = 0, row_it = 0;
     int q_issued = 0, k_issued = 0, v_issued = 0;  // tiles whose loads this warp has issued
+    // The next work entry of this launch, from the global counter: a whole
+    // item, or (the last cut_items items) one part of one, up to kCutParts
+    // equal shares of its KV tiles (fewer for an item of fewer tiles: the
+    // entries of the missing parts are skipped).
+    const int whole = p.rows - p.cut_items;
+    auto take_item = [&](int it, bool& ok) -> int4 {
+      const int slot = it % kItemSlots;
+      int4 sg = make_int4(p.rows, 0, 0, 0);
+      if (it >= kItemSlots &&
+          !(ok = warp_wait(bar(bars->item_empty[slot]), ((it / kItemSlots) - 1) & 1, abort, p.err, 4)))
+        return sg;
+      if (lane == 0) {
+        for (;;) {
+          const int e = p.entry_lo + int(atomicAdd(p.work_counter, 1u));
+          if (e >= p.entry_hi) break;  // past this launch's entries: the end
+          if (e < whole) {
+            sg = make_int4(e, 0, (list_count<PAIR>(p, e) + KB - 1) / KB, 1 << 16);
+            break;
+          }
+          const int item = whole + (e - whole) / kCutParts, part = (e - whole) % kCutParts;
+          const int n = (list_count<PAIR>(p, item) + KB - 1) / KB;
+          const int parts = n < kCutParts ? n : kCutParts;
+          if (part >= parts) continue;
+          sg = make_int4(item, part * n / parts, (part + 1) * n / parts, part | (parts << 16));
+          break;
+        }
+        bars->item[slot] = sg;
+        mbar_arrive(bar(bars->item_full[slot]));
+      }
+      sg.x = __shfl_sync(0xffffffffu, sg.x, 0);
+      sg.y = __shfl_sync(0xffffffffu, sg.y, 0);
+      sg.z = __shfl_sync(0xffffffffu, sg.z, 0);
+      sg.w = __shfl_sync(0xffffffffu, sg.w, 0);
+      return sg;
+    };
     bool ok = true;
     for (int it = 0; ok; ++it, ++row_it) {
-      const int rr = take_item(it, ok);
+      const int4 sg = take_item(it, ok);
+      const int rr = sg.x, t0 = sg.y;
       if (!ok || rr >= p.rows) break;
       const int64_t beg = list_begin<PAIR>(p, rr);
       const int n = list_count<PAIR>(p, rr);
@@ -528,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       q_issued = row_it + 1;
-      const int steps = (n + KB - 1) / KB;
+      const int steps = sg.z - t0;  // the segment's KV tiles t0 .. sg.z - 1 of the item
       auto fill = [&](Entries& e, int chunk) {
         e.chunk = chunk;
         const int j = chunk * 32 + lane;
@@ -544,10 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       Entries ke, ve;  // cursors of the K loads (kKStages steps ahead) and of the V loads
-      // entry of the selected block feeding sub-tile i of step st (an odd last
-      // step repeats its block; the softmax masks the copy)
+      // entry of the selected block feeding sub-tile i of step st (the item's
+      // tile t0 + st; an odd last tile repeats its block; the softmax masks
+      // the copy)
       auto entry = [&](Entries& e, int st, int i) -> int {
-        const int j = min(st * KB + i, n - 1);
+        const int j = min((t0 + st) * KB + i, n - 1);
         if (e.chunk != (j >> 5)) fill(e, j >> 5);  // warp-uniform
         return j & 31;
       };
@@ -636,9 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, s_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int it = 0; ok; ++it, ++row_it) {
-      const int rr = read_item(it, ok);
-      if (!ok || rr >= p.rows) break;
-      const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
+      const int4 sg = read_item(it, ok);
+      if (!ok || sg.x >= p.rows) break;
+      const int n = sg.z - sg.y;  // KV tiles of the segment
       if (!(ok = warp_wait(bar(bars->q_full), row_it & 1, abort, p.err, 10))) break;
       for (int j = 0; j < n; ++j, ++s_it) {
         const int sb = s_it % kSBufs;
@@ -679,9 +747,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kv = 0, pv_it = 0, row_it = 0;
     bool ok = true, issued = false;
     for (int it = 0; ok; ++it, ++row_it) {
-      const int rr = read_item(it, ok);
-      if (!ok || rr >= p.rows) break;
-      const int n = (list_count<PAIR>(p, rr) + KB - 1) / KB;  // KV tiles of the work item
+      const int4 sg = read_item(it, ok);
+      if (!ok || sg.x >= p.rows) break;
+      const int n = sg.z - sg.y;  // KV tiles of the segment
       for (int j = 0; j < n; ++j, ++pv_it) {
         const int pb = pv_it % kSBufs;
         if (!(ok = warp_wait(bar(bars->p_full[pb]), (pv_it / kSBufs) & 1, abort, p.err, 13))) break;
@@ -742,11 +810,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the maximum in use after tile s has been published
     auto wait_dec = [&](int s) { return warp_wait(bar(bars->dec[sp][s & 1]), (s >> 1) & 1, abort, p.err, 26); };
     for (int it = 0; ok; ++it) {
-      const int rr = read_item(it, ok);
+      const int4 sg = read_item(it, ok);
+      const int rr = sg.x, t0 = sg.y;
       if (!ok || rr >= p.rows) break;
       const int n_sel = list_count<PAIR>(p, rr);
-      const int n = (n_sel + KB - 1) / KB;  // KV tiles of the work item
-      const int* lst = PAIR ? p.pair_col + list_begin<PAIR>(p, rr) : nullptr;
+      const int n = sg.z - t0;  // KV tiles of the segment: the item's t0 .. t0 + n - 1
+      const int* lst = PAIR ? p.pair_col + list_begin<PAIR>(p, rr) + KB * t0 : nullptr;
+      const int sel_left = n_sel - KB * t0;  // list entries from the segment's first tile on
       float m_g = -INFINITY, l = 0.f;  // this group's partial row sum, scaled by 2^-m_g
       for (int j = 0; j < n && ok; ++j, ++s_it) {
         if ((s_it & 1) != grp) continue;
@@ -758,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (PAIR) {
           const int bit = sp < 2 ? 1 : 2;
           mask0 = !((__ldg(lst + KB * j) >> kPairShift) & bit);
-          mask1 = KB * j + 1 >= n_sel || !((__ldg(lst + KB * j + 1) >> kPairShift) & bit);
+          mask1 = KB * j + 1 >= sel_left || !((__ldg(lst + KB * j + 1) >> kPairShift) & bit);
         }
         const int sb = s_it % kSBufs;
 #ifdef LCSA_TEST_STALL
@@ -914,7 +984,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(bars->pair[sp]));
       if (!(ok = warp_wait(bar(bars->pair[sp]), xk & 1, abort, p.err, 24))) break;
       ++xk;
-      const float inv = 1.0f / (l + xs[(grp ^ 1) * 128 + row_in_tile]);
+      const float l_row = l + xs[(grp ^ 1) * 128 + row_in_tile];  // the segment's row sum at m_final
       int qrow = rr, m_tok = row_in_tile;  // query block (row) and token of this lane's row
       bool store = true;
       if constexpr (PAIR) {
@@ -931,20 +1001,129 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
       // this group's half of the row's D output channels, 32 at a time
       __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * D + grp * (D / 2);
+      // An item cut into parts (segments on consecutive CTAs): each warp
+      // counts its part's arrival; all but the last write their slice (this
+      // warp's 32 rows x D / 2 channels of O, with the rows' maxima and sums)
+      // and flag it; the last waits for those flags and combines every part,
+      // in part order, into the output.
+      const int parts = PAIR ? sg.w >> 16 : 1, part = sg.w & 0xFFFF;  // only pairs are cut
+      const int wsl = warp - 3;  // this warp's slice
+      constexpr int kSlice = 32 * (D / 2) + 64;
+      const int slot0 = parts > 1 ? (rr - (p.rows - p.cut_items)) * kCutParts : 0;
+      auto slot_of = [&](int j) { return slot0 + j; };
+      auto slice = [&](int j) { return p.part_buf + (int64_t(slot_of(j)) * 8 + wsl) * kSlice; };
+      bool last = true;
+      if (parts > 1) {
+        unsigned before = 0;
+        if (lane == 0) before = atomicAdd(p.merge_cnt + int64_t(rr - (p.rows - p.cut_items)) * 8 + wsl, 1u);
+        last = __shfl_sync(0xffffffffu, before, 0) + 1 == unsigned(parts);
+      }
+      if (!last) {
+        float* my = slice(part);
 #pragma unroll
-      for (int q2 = 0; q2 < D / 64; ++q2) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + kColO + grp * (D / 2) + q2 * 32, o);
-        tmem_wait_ld();
-        uint4 v[4];
-        uint32_t* w = reinterpret_cast<uint32_t*>(v);
+        for (int q2 = 0; q2 < D / 64; ++q2) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + kColO + grp * (D / 2) + q2 * 32, o);
+          tmem_wait_ld();
+          // channels 4 e .. 4 e + 3 of chunk q2, lane by lane (a warp's store is 512 contiguous bytes)
+          float4* d4 = reinterpret_cast<float4*>(my) + q2 * 8 * 32 + lane;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
-        if (store) {
+          for (int e = 0; e < 8; ++e)
+            d4[e * 32] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                     __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        }
+        my[32 * (D / 2) + lane] = m_final;
+        my[32 * (D / 2) + 32 + lane] = l_row;
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) flag_release(p.merge_ready + slot_of(part) * 8 + wsl);
+      } else {
+        float inv;
+        if (parts > 1) {
+          bool got = true;
+          if (lane == 0)
+            for (int j = 0; j < parts && got; ++j)
+              if (j != part) got = flag_wait(p.merge_ready + slot_of(j) * 8 + wsl, abort, p.err, 27);
+          if (!(ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0)) break;
+          __threadfence();
+          // the row's maximum over the parts, then the sum of their sums at it
+          // (every part's values read at once: at most kCutParts of them)
+          float mj[kCutParts], sj[kCutParts];
+          float mx = m_final;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = v[e];
+          for (int j = 0; j < kCutParts; ++j) {
+            mj[j] = j < parts && j != part ? slice(j)[32 * (D / 2) + lane] : m_final;
+            mx = fmaxf(mx, mj[j]);
+          }
+          float lsum = 0.f;
+#pragma unroll
+          for (int j = 0; j < kCutParts; ++j) {
+            sj[j] = j < parts && mj[j] != -INFINITY ? exp2_mufu(mj[j] - mx) : 0.f;
+            const float lj = j == part ? l_row : (j < parts ? slice(j)[32 * (D / 2) + 32 + lane] : 0.f);
+            if (j < parts) lsum = j == 0 ? lj * sj[j] : fmaf(lj, sj[j], lsum);
+          }
+          inv = 1.0f / lsum;
+#pragma unroll 1
+          for (int q2 = 0; q2 < D / 64; ++q2) {
+            uint32_t o[32];  // this part's O
+            tmem_ld32(lane_addr + kColO + grp * (D / 2) + q2 * 32, o);
+            tmem_wait_ld();
+            uint4 v[4];
+            uint32_t* w = reinterpret_cast<uint32_t*>(v);
+            // two groups of four channels at a time: the other parts' values
+            // are loaded together, then added in part order at the common maximum
+            constexpr int kGroup = 2;
+#pragma unroll
+            for (int e0 = 0; e0 < 8; e0 += kGroup) {
+              float4 x[kCutParts][kGroup];
+#pragma unroll
+              for (int j = 0; j < kCutParts; ++j)
+#pragma unroll
+                for (int e = 0; e < kGroup; ++e)
+                  x[j][e] = j < parts && j != part
+                                ? reinterpret_cast<const float4*>(slice(j))[(q2 * 8 + e0 + e) * 32 + lane]
+                                : make_float4(__uint_as_float(o[4 * (e0 + e)]), __uint_as_float(o[4 * (e0 + e) + 1]),
+                                              __uint_as_float(o[4 * (e0 + e) + 2]),
+                                              __uint_as_float(o[4 * (e0 + e) + 3]));
+#pragma unroll
+              for (int e = 0; e < kGroup; ++e) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < kCutParts; ++j) {
+                  if (j >= parts) break;
+                  acc[0] = j == 0 ? x[j][e].x * sj[j] : fmaf(x[j][e].x, sj[j], acc[0]);
+                  acc[1] = j == 0 ? x[j][e].y * sj[j] : fmaf(x[j][e].y, sj[j], acc[1]);
+                  acc[2] = j == 0 ? x[j][e].z * sj[j] : fmaf(x[j][e].z, sj[j], acc[2]);
+                  acc[3] = j == 0 ? x[j][e].w * sj[j] : fmaf(x[j][e].w, sj[j], acc[3]);
+                }
+                w[2 * (e0 + e)] = pack_bf16(acc[0] * inv, acc[1] * inv);
+                w[2 * (e0 + e) + 1] = pack_bf16(acc[2] * inv, acc[3] * inv);
+              }
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
+            if (store) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d4[e] = v[e];
+            }
+          }
+        } else {
+          inv = 1.0f / l_row;
+#pragma unroll
+          for (int q2 = 0; q2 < D / 64; ++q2) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + kColO + grp * (D / 2) + q2 * 32, o);
+            tmem_wait_ld();
+            uint4 v[4];
+            uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + q2 * 32);
+            if (store) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d4[e] = v[e];
+            }
+          }
         }
       }
       tc_fence_before();
@@ -1056,11 +1235,21 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.scale_log2 = p.scale_log2;
   tp.err = p.err;
   tp.rows = paired ? p.npairs : p.g.B * p.g.Hn * p.g.nQB;
-  tp.item_lo = p.item_lo;
-  tp.item_hi = p.item_hi > 0 ? p.item_hi : tp.rows;
-  if (tp.item_lo < 0 || tp.item_hi > tp.rows || tp.item_lo >= tp.item_hi) return cudaErrorInvalidValue;
+  const int item_lo = p.item_lo, item_hi = p.item_hi > 0 ? p.item_hi : tp.rows;
+  if (item_lo < 0 || item_hi > tp.rows || item_lo >= item_hi) return cudaErrorInvalidValue;
   tp.work_counter = p.work_counter;
   if (!tp.work_counter) return cudaErrorInvalidValue;
+  // cut items (64-token pairs only): the entries of items lo .. hi - 1
+  tp.cut_items = paired ? p.cut_items : 0;
+  if (tp.cut_items < 0 || tp.cut_items > tp.rows) return cudaErrorInvalidValue;
+  if (tp.cut_items > 0 && (!p.merge_cnt || !p.merge_ready || !p.part_buf)) return cudaErrorInvalidValue;
+  tp.merge_cnt = p.merge_cnt;
+  tp.merge_ready = p.merge_ready;
+  tp.part_buf = p.part_buf;
+  const int whole = tp.rows - tp.cut_items;
+  auto entry_of = [&](int i) { return i <= whole ? i : whole + (i - whole) * kCutParts; };
+  tp.entry_lo = entry_of(item_lo);
+  tp.entry_hi = entry_of(item_hi);
   tp.pair_col = p.pair_col;
   tp.pair_len = p.pair_len;
   tp.pair_rows = p.pair_rows;
@@ -1071,8 +1260,8 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
   tp.stall_site = g_stall_site;
   g_stall_site = 0;
 #endif
-  const int items = tp.item_hi - tp.item_lo;
-  const int grid = items < num_sms ? items : num_sms;
+  const int entries = tp.entry_hi - tp.entry_lo;
+  const int grid = entries < num_sms ? entries : num_sms;
   kern<<<grid, kThreads, smem, s>>>(tm_q, tm_k, tm_v, tp);
   return cudaGetLastError();
 }

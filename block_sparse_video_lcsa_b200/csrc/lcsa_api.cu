@@ -102,6 +102,10 @@ lcsa_status_t resolve(const lcsa_config_t* c, Resolved* r, bool want_rows) {
   }
   ws += rope_n * sizeof(float2) + 256;
   ws += size_t(lcsa::kMaxK1Ctas) * 2 * size_t(g.C) * 4 + size_t(lcsa::kCounters) * 4;  // K1 split blocks, counters
+  if (nb == 64) {  // merge state of cut pairs, for up to kMaxK1Ctas SMs (the plan sizes it for the device's)
+    const size_t cut = size_t(lcsa::cut_items(int(lcsa::pair_count(g)), lcsa::kMaxK1Ctas));
+    ws += cut * 8 * 4 + cut * lcsa::kCutParts * 8 * 4 + lcsa::part_buf_floats(int(cut), c->head_dim) * 4;
+  }
   if (c->host_io)
     ws += size_t(g.B) * (2 * g.Lq + 2 * g.Lkv) * g.C * 2 + size_t(2) * g.C * 4;
   o.workspace_bytes = ws;
@@ -144,6 +148,11 @@ struct lcsa_plan {
   int32_t* pair_len = nullptr;
   int2* pair_rows = nullptr;
   int npairs = 0, pair_cap = 0;
+  // 64-token pairs: merge state of the last pairs, cut into parts
+  unsigned* merge_cnt = nullptr;
+  unsigned* merge_ready = nullptr;
+  float* part_buf = nullptr;
+  int cut = 0;
   bool reuse_mode = false;   // lcsa_plan_set_threshold_reuse
   bool have_thresh = false;  // a selecting call has recorded thresholds
   bool last_reuse = false;   // the last call kept blocks by threshold
@@ -177,7 +186,7 @@ void release(lcsa_plan* p) {
   void* ptrs[] = {p->v_ring, p->qhat,  p->khat,    p->pooled_q, p->pooled_k, p->split_part, p->split_cnt,
                   p->row_ptr, p->col_idx, p->rope,     p->err,      p->st_q,       p->st_k,
                   p->st_v,  p->st_out,  p->st_gq,    p->st_gk,    p->thresh,     p->row_len, p->col_pad,
-                  p->pair_col, p->pair_len,  p->pair_rows};
+                  p->pair_col, p->pair_len,  p->pair_rows, p->merge_cnt, p->merge_ready, p->part_buf};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (auto& set : p->evsets)
@@ -263,6 +272,12 @@ lcsa_status_t alloc_pairs(lcsa_plan* p) {
   lcsa_status_t st = dev_alloc(&p->pair_col, size_t(np) * size_t(p->pair_cap) * 4, "pair lists");
   if (st == LCSA_OK) st = dev_alloc(&p->pair_len, size_t(np) * 4, "pair counts");
   if (st == LCSA_OK) st = dev_alloc(&p->pair_rows, size_t(np) * sizeof(int2), "pair rows");
+  // the last pairs are cut into parts: the attention's merge state
+  p->cut = lcsa::cut_items(p->npairs, p->num_sms);
+  const size_t cut = size_t(p->cut);
+  if (st == LCSA_OK) st = dev_alloc(&p->merge_cnt, cut * 8 * 4, "cut pairs' counters");
+  if (st == LCSA_OK) st = dev_alloc(&p->merge_ready, cut * lcsa::kCutParts * 8 * 4, "cut pairs' ready flags");
+  if (st == LCSA_OK) st = dev_alloc(&p->part_buf, lcsa::part_buf_floats(p->cut, p->res.grid.D) * 4, "cut pairs' partials");
   return st;
 }
 
@@ -345,6 +360,10 @@ lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Fault
   p->rope_w_off = p->rope_h_off + g.gh * rs.pairs_h;
   const size_t rows = size_t(p->res.geo.rows), nnz = size_t(p->res.geo.nnz);
   const size_t D = size_t(cfg->head_dim);
+  if ((e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, cuda_device)) != cudaSuccess) {
+    delete p;
+    return cuda_fail(e, "device attributes");
+  }
   if ((st = dev_alloc(&p->qhat, size_t(g.B) * g.Lq * g.C * 2, "q^")) ||
       (st = dev_alloc(&p->khat, size_t(g.B) * g.Lkv * g.C * 2, "k^")) ||
       (st = dev_alloc(&p->pooled_q, size_t(g.B) * g.Hn * g.nQB * D * 4, "pooled q")) ||
@@ -393,11 +412,6 @@ lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Fault
     release(p);
     delete p;
     return cuda_fail(e, "plan set-up");
-  }
-  if ((e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, cuda_device)) != cudaSuccess) {
-    release(p);
-    delete p;
-    return cuda_fail(e, "device attributes");
   }
   {
     if ((e = lcsa::make_block_map(&p->tm_q, p->qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb, g.D)) != cudaSuccess ||
@@ -521,6 +535,10 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
   k3.pair_rows = p->pair_rows;
   k3.pair_cap = p->pair_cap;
   k3.work_counter = p->split_cnt + lcsa::kMaxK1Ctas;
+  k3.cut_items = p->cut;
+  k3.merge_cnt = p->merge_cnt;
+  k3.merge_ready = p->merge_ready;
+  k3.part_buf = p->part_buf;
   k3.scale_log2 = p->res.scale * 1.4426950408889634f;
   k3.err = p->err;
   k3.ring_fb = g.Tkv / g.bt;
@@ -560,6 +578,9 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
     pp.pair_len = p->pair_len;
     pp.pair_rows = p->pair_rows;
     pp.pair_cap = p->pair_cap;
+    pp.merge_cnt = p->merge_cnt;
+    pp.merge_ready = p->merge_ready;
+    pp.cut = p->cut;
     if (lcsa_status_t st = injected_launch_failure(p, kFaultPair, "pair union")) return st;
     if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return cuda_fail(e, "pair union launch");
   }

@@ -182,6 +182,10 @@ struct PairParams {
   int* pair_len;          // [npairs]
   int2* pair_rows;        // [npairs] the pair's two rows (second -1: a single block)
   int pair_cap;
+  // the attention's merge state of cut pairs, cleared here for the call that follows
+  unsigned* merge_cnt;    // [cut][8]
+  unsigned* merge_ready;  // [cut * kCutParts][8]
+  int cut;                // cut_items(npairs, SMs)
 };
 
 struct K3Params {
@@ -205,7 +209,14 @@ struct K3Params {
   const int* pair_len;
   const int2* pair_rows;
   int pair_cap;
-  unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work items from it
+  unsigned* work_counter;   // zero at launch (K2 clears it); K3's CTAs take work entries from it
+  // The last cut_items work items (64-token pairs) are cut into up to
+  // kCutParts parts of their KV tiles, each its own work entry; the last
+  // part to finish merges them (merge state: cut_state, see CutState).
+  int cut_items;
+  unsigned* merge_cnt;      // [cut_items][8] arrivals per softmax warp slice
+  unsigned* merge_ready;    // [cut_items * kCutParts][8] a part's partial result written
+  float* part_buf;          // [cut_items * kCutParts][8][32 * (head_dim / 2) + 64]
   // Work items item_lo .. item_hi - 1 (rows, or query-block pairs); both 0:
   // all of them
   int item_lo, item_hi;
@@ -267,5 +278,19 @@ cudaError_t make_xhat_row_map(CUtensorMap* map, void* base, const Grid& g, int n
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, int num_sms, cudaStream_t s);
+
+// Cut work items of the attention (64-token pairs): a persistent kernel that
+// hands out whole items leaves SMs idle at the end when the item count is
+// not a multiple of the SM count and the items are long, so the last
+// cut_items(items, ctas) items are cut into up to kCutParts parts (of their
+// KV tiles), each handed out on its own; the parts of an item are merged by
+// the last of them to finish.
+constexpr int kCutParts = 4;
+inline int cut_items(int items, int ctas) { return items < ctas / 2 ? items : ctas / 2; }
+// floats of part_buf for n cut items: per part and softmax warp, 32 rows x
+// (head_dim / 2) of O, then the rows' maxima and sums
+inline size_t part_buf_floats(int n, int head_dim) {
+  return size_t(n) * kCutParts * 8 * (32 * size_t(head_dim / 2) + 64);
+}
 
 }  // namespace lcsa

@@ -194,12 +194,21 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   const size_t off_pc = off_kh + round256(size_t(g.B) * g.Lkv * g.C * 2);
   const size_t off_pl = off_pc + round256(size_t(npairs) * size_t(pair_cap) * 4);
   const size_t off_pr = off_pl + round256(size_t(npairs) * 4);
-  const size_t need = off_pr + round256(size_t(npairs) * sizeof(int2));
-  if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES)) return LCSA_ERR_UNSUPPORTED;  // create a plan instead
-
-  int dev = 0;
+  const size_t off_sg = off_pr + round256(size_t(npairs) * sizeof(int2));
+  // the problem's own buffers must fit before any device is asked anything
+  if (off_sg > size_t(LCSA_NOALLOC_WORKSPACE_BYTES)) return LCSA_ERR_UNSUPPORTED;  // create a plan instead
+  int dev = 0, num_sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return LCSA_ERR_CUDA;
+  if ((e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return LCSA_ERR_CUDA;
+  // 64-token pairs: the attention's merge state of the last pairs, cut into parts
+  const int cut = npairs ? lcsa::cut_items(int(npairs), num_sms) : 0;
+  const size_t off_mc = off_sg;
+  const size_t off_mr = off_mc + round256(size_t(cut) * 8 * 4);
+  const size_t off_pb = off_mr + round256(size_t(cut) * lcsa::kCutParts * 8 * 4);
+  const size_t need = off_pb + round256(lcsa::part_buf_floats(cut, D) * 4);
+  if (need > size_t(LCSA_NOALLOC_WORKSPACE_BYTES)) return LCSA_ERR_UNSUPPORTED;  // create a plan instead
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* ws = nullptr;
   {
@@ -221,6 +230,9 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   int* pair_col = npairs ? reinterpret_cast<int*>(ws + off_pc) : nullptr;
   int* pair_len = npairs ? reinterpret_cast<int*>(ws + off_pl) : nullptr;
   int2* pair_rows = npairs ? reinterpret_cast<int2*>(ws + off_pr) : nullptr;
+  unsigned* merge_cnt = reinterpret_cast<unsigned*>(ws + off_mc);
+  unsigned* merge_ready = reinterpret_cast<unsigned*>(ws + off_mr);
+  float* part_buf = reinterpret_cast<float*>(ws + off_pb);
 
   // the counters start at zero (an aborted call may have left them set)
   if ((e = cudaMemsetAsync(split_cnt, 0, kOffAfterCnt - kOffCnt, s)) != cudaSuccess) return LCSA_ERR_CUDA;
@@ -253,8 +265,7 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k1.ss_ext = nullptr;
   k1.norm_inv_c = 1.0f / float(g.C);
   lcsa::k1_all_blocks(k1);
-  if ((e = cudaDeviceGetAttribute(&k1.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return LCSA_ERR_CUDA;
+  k1.num_sms = num_sms;
   {
     LCSA_RANGE("lcsa K1 prologue");
     if ((e = lcsa::launch_prologue(k1, s)) != cudaSuccess) return LCSA_ERR_CUDA;
@@ -294,6 +305,9 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
     pp.pair_len = pair_len;
     pp.pair_rows = pair_rows;
     pp.pair_cap = pair_cap;
+    pp.merge_cnt = merge_cnt;
+    pp.merge_ready = merge_ready;
+    pp.cut = cut;
     if ((e = lcsa::launch_pair_union(pp, s)) != cudaSuccess) return LCSA_ERR_CUDA;
   }
 
@@ -317,10 +331,13 @@ extern "C" lcsa_status_t lcsa_forward_noalloc(const lcsa_config_t* cfg, const vo
   k3.npairs = int(npairs);
   k3.pair_cap = pair_cap;
   k3.work_counter = split_cnt + lcsa::kMaxK1Ctas;
+  k3.cut_items = cut;
+  k3.merge_cnt = merge_cnt;
+  k3.merge_ready = merge_ready;
+  k3.part_buf = part_buf;
   {
     LCSA_RANGE("lcsa K3 attention");
     CUtensorMap tm_q, tm_k, tm_v;  // encoded on the host stack: no allocation
-    const int num_sms = k1.num_sms;
     if ((e = lcsa::make_block_map(&tm_q, qhat, int64_t(g.B) * g.Hn * g.nQB * g.nb, g.nb, g.D)) != cudaSuccess ||
         (e = lcsa::make_block_map(&tm_k, khat, int64_t(g.B) * g.Hn * g.nKB * g.nb, g.nb, g.D)) != cudaSuccess ||
         (e = lcsa::make_raster_map(&tm_v, v, g)) != cudaSuccess)

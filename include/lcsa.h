@@ -127,7 +127,7 @@ typedef struct lcsa_geometry {
   double selected_flops;             /* sum over rows of kept * 4 * n_b^2 * head_dim */
   double prologue_bytes;             /* bytes the prologue must move (q,k in; q^,k^ out) */
   double attention_min_bytes;        /* q^ + out + each touched k^/v block once */
-  size_t workspace_bytes;            /* device bytes the plan allocates */
+  size_t workspace_bytes;            /* device bytes the plan allocates (at most) */
 } lcsa_geometry_t;
 
 typedef struct lcsa_plan* lcsa_plan_t;
@@ -240,10 +240,10 @@ LCSA_API lcsa_status_t lcsa_forward_sharded(lcsa_plan_t plan, const void* q, con
 LCSA_API lcsa_status_t lcsa_plan_set_threshold_reuse(lcsa_plan_t plan, int on);
 LCSA_API lcsa_status_t lcsa_selection_nnz(lcsa_plan_t plan, int64_t* nnz);
 
-/* Size of the static device workspace used by lcsa_forward_noalloc (32 MiB).
+/* Size of the static device workspace used by lcsa_forward_noalloc (64 MiB).
    A GPU holds this array from the first lcsa_forward_noalloc call made on it
    (when the CUDA module that holds it is loaded) until the process exits. */
-#define LCSA_NOALLOC_WORKSPACE_BYTES (32u << 20)
+#define LCSA_NOALLOC_WORKSPACE_BYTES (64u << 20)
 
 /* The LCSA call without a plan and without any allocation, for callers that
    may not allocate device memory once running (for instance a real-time
