@@ -281,12 +281,13 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
 
 // Cut work items of the attention (64-token pairs): a persistent kernel that
 // hands out whole items leaves SMs idle at the end when the item count is
-// not a multiple of the SM count and the items are long, so the last
-// cut_items(items, ctas) items are cut into up to kCutParts parts (of their
-// KV tiles), each handed out on its own; the parts of an item are merged by
-// the last of them to finish.
+// not a multiple of the SM count and the items are long, so when there are
+// at least as many items as CTAs the last ctas / 2 are cut into up to
+// kCutParts parts (of their KV tiles), each handed out on its own; the parts
+// of an item are merged by the last of them to finish. Fewer items than CTAs
+// leave no tail to even out, and are not cut.
 constexpr int kCutParts = 4;
-inline int cut_items(int items, int ctas) { return items < ctas / 2 ? items : ctas / 2; }
+inline int cut_items(int items, int ctas) { return items >= ctas ? ctas / 2 : 0; }
 // floats of part_buf for n cut items: per part and softmax warp, 32 rows x
 // (head_dim / 2) of O, then the rows' maxima and sums
 inline size_t part_buf_floats(int n, int head_dim) {
