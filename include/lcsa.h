@@ -158,7 +158,11 @@ LCSA_API void lcsa_plan_destroy(lcsa_plan_t plan);
 /* One LCSA call: prologue, block selection and block-sparse attention,
    launched on `stream` (a cudaStream_t; null = legacy default stream).
    q, k, v, out: device bf16 as laid out above, 16-byte aligned. gamma_q,
-   gamma_k: device fp32 [heads*head_dim], 16-byte aligned. Asynchronous. */
+   gamma_k: device fp32 [heads*head_dim], 16-byte aligned. Asynchronous.
+   Deterministic: the same inputs give the same output bits on every call,
+   however the attention's work is spread over the SMs (with 64-token blocks
+   and at least as many query-block pairs as SMs, the last pairs are cut into
+   parts run by different CTAs and merged in a fixed part order). */
 LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void* k, const void* v,
                            const float* gamma_q, const float* gamma_k, void* out, void* stream);
 
