@@ -32,6 +32,9 @@ CASES = {
     "batch2": _T.replace(batch=2, heads=2, topk=3, field=True, unit_gain=False, seed=6),
     "d64_split": _T.replace(head_dim=64, heads=4, q_frames=1, kv_frames=3, grid_h=24, grid_w=48, block_w=16,
                             local_range=3, topk=5, field=True, unit_gain=False, seed=7),
+    # 160 query-block pairs, at least as many as the SMs: the last pairs are cut and merged
+    "cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                            field=True, unit_gain=False, seed=22),
 }
 
 

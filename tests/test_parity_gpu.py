@@ -47,6 +47,11 @@ SMALL = {
     "d64_k1_split_blocks": _T.replace(head_dim=64, heads=2, q_frames=1, kv_frames=2, grid_h=64, grid_w=128,
                                       block_w=16, local_range=3, topk=4, kv_frame_offset=1, field=True,
                                       unit_gain=False, seed=11),
+    # 160 query-block pairs (8 heads x 2 frame groups x 10 pairs of a 4 x 5
+    # block grid): at least as many as the B200's 148 SMs, so the last pairs
+    # are cut into parts and merged
+    "blocks64_cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                                     field=True, unit_gain=False, seed=21),
 }
 OVERRIDES = {"tiny_head_scope": dict(norm_scope=1), "d64_head_scope": dict(norm_scope=1)}
 

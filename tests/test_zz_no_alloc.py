@@ -28,6 +28,9 @@ CASES = {
                                topk=5, kv_frame_offset=2, field=True, unit_gain=False),
     "blocks64_d64": _T.replace(head_dim=64, heads=4, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5,
                                topk=9, field=True, unit_gain=False, seed=13),
+    # 160 query-block pairs, at least as many as the SMs: the last pairs are cut and merged
+    "cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                            field=True, unit_gain=False, seed=22),
 }
 
 
