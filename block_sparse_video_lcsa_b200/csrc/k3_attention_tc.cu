@@ -1001,7 +1001,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tok = (int64_t(tb * g.bt + tt) * g.gh + (rem / g.nWb) * g.bh + yy) * g.gw + (rem % g.nWb) * g.bw + xx;
       // this group's half of the row's D output channels, 32 at a time
       __nv_bfloat16* dst = p.out + (int64_t(b) * g.Lq + tok) * g.C + h * D + grp * (D / 2);
-      // An item cut into parts (segments on consecutive CTAs): each warp
+      // An item cut into parts (run by whatever CTAs drew them): each warp
       // counts its part's arrival; all but the last write their slice (this
       // warp's 32 rows x D / 2 channels of O, with the rows' maxima and sums)
       // and flag it; the last waits for those flags and combines every part,
