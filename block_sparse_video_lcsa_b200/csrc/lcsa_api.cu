@@ -170,10 +170,11 @@ struct lcsa_plan {
   CUtensorMap tm_q, tm_k;
   int num_sms = 0;
   // host-IO plans: a copy stream and the events that order it against the
-  // call's stream (q/k uploaded, V uploaded, first attention half done,
-  // first half of the output downloaded)
+  // call's stream (q/k uploaded, V (or its first half of the heads)
+  // uploaded, V's second half uploaded, first attention half done, first
+  // half of the output downloaded)
   cudaStream_t io_stream = nullptr;
-  cudaEvent_t ev_qk = nullptr, ev_v = nullptr, ev_k3a = nullptr, ev_outa = nullptr;
+  cudaEvent_t ev_qk = nullptr, ev_v = nullptr, ev_v2 = nullptr, ev_k3a = nullptr, ev_outa = nullptr;
   unsigned fault_launch = 0;                       // LCSA_FAULT launch:K (kFault* bits)
   bool fault_copy = false;                         // LCSA_FAULT copy
   std::vector<std::array<cudaEvent_t, 4>> evsets;  // timing ring
@@ -193,7 +194,7 @@ void release(lcsa_plan* p) {
     for (auto e : set)
       if (e) cudaEventDestroy(e);
   p->evsets.clear();
-  for (cudaEvent_t e : {p->ev_qk, p->ev_v, p->ev_k3a, p->ev_outa})
+  for (cudaEvent_t e : {p->ev_qk, p->ev_v, p->ev_v2, p->ev_k3a, p->ev_outa})
     if (e) cudaEventDestroy(e);
   if (p->io_stream) cudaStreamDestroy(p->io_stream);
 }
@@ -396,6 +397,7 @@ lcsa_status_t create_plan(const lcsa_config_t* cfg, int cuda_device, const Fault
     if ((e = cudaStreamCreateWithFlags(&p->io_stream, cudaStreamNonBlocking)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&p->ev_qk, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&p->ev_v, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&p->ev_v2, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&p->ev_k3a, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&p->ev_outa, cudaEventDisableTiming)) != cudaSuccess) {
       release(p);
@@ -465,6 +467,7 @@ struct StepBlocks {
   cudaEvent_t k3_wait = nullptr; // an event K3 waits for (the host-IO call's V upload)
   int k3_split = 0;              // > 0: K3 as two launches, work items [0, k3_split) and the rest,
   cudaEvent_t k3_first_done = nullptr;  // recorded between them
+  cudaEvent_t k3_wait_b = nullptr;      // an event the second of them also waits for (V's second half)
 };
 
 lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float* gamma_q, const float* gamma_k,
@@ -605,6 +608,8 @@ lcsa_status_t run_step(lcsa_plan_t p, const void* q, const void* k, const float*
       k3.item_lo = sb.k3_split;
       k3.item_hi = 0;  // to the end
       k3.work_counter += 1;
+      if (sb.k3_wait_b && (e = cudaStreamWaitEvent(s, sb.k3_wait_b, 0)) != cudaSuccess)
+        return cuda_fail(e, "wait for V");
     }
     if ((e = lcsa::launch_attention_tc(k3, p->tm_q, p->tm_k, tm_v, p->num_sms, s)) != cudaSuccess)
       return cuda_fail(e, "attention launch");
@@ -794,6 +799,15 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
   const lcsa::Grid& g = p->res.grid;
   const size_t qb = size_t(g.B) * g.Lq * g.C * 2, kb = size_t(g.B) * g.Lkv * g.C * 2, gb = size_t(g.C) * 4;
   if (p->fault_copy) return fail(LCSA_ERR_CUDA, "host-to-device copy: injected failure (LCSA_FAULT)");
+  // With one batch element and at least two heads K3 runs as two launches
+  // over the first and the second half of the heads (rows, or query-block
+  // pairs, are numbered head-major): each reads only its heads' channels of
+  // v, so v goes up in those two halves (strided copies, a token's channels
+  // being head-major) and each launch waits only for its own; the first
+  // half's output channels go back on the copy stream while the second half
+  // computes.
+  const int heads_a = g.B == 1 && g.Hn >= 2 ? g.Hn / 2 : 0;
+  const size_t pitch = size_t(g.C) * 2, head_bytes = size_t(g.D) * 2;
   // The copies share one link, so they go in the order the kernels need
   // them: gains, q and k on the call's stream (K1 and K2 start as soon as
   // they are in), then v on the plan's copy stream while K1 and K2 run.
@@ -802,27 +816,35 @@ lcsa_status_t lcsa_forward_host(lcsa_plan_t p, const void* q, const void* k, con
       (e = cudaMemcpyAsync(p->st_q, q, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
       (e = cudaMemcpyAsync(p->st_k, k, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
       (e = cudaEventRecord(p->ev_qk, s)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(p->io_stream, p->ev_qk, 0)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, p->io_stream)) != cudaSuccess ||
-      (e = cudaEventRecord(p->ev_v, p->io_stream)) != cudaSuccess)
+      (e = cudaStreamWaitEvent(p->io_stream, p->ev_qk, 0)) != cudaSuccess)
     return cuda_fail(e, "host-to-device copy");
-  // K3 waits for v. With one batch element and at least two heads it runs as
-  // two launches over the first and the second half of the heads (rows, or
-  // query-block pairs, are numbered head-major), and the first half's output
-  // channels go back on the copy stream while the second half computes.
+  if (heads_a > 0) {
+    char* dv = static_cast<char*>(p->st_v);
+    const char* hv = static_cast<const char*>(v);
+    if ((e = cudaMemcpy2DAsync(dv, pitch, hv, pitch, heads_a * head_bytes, size_t(g.Lkv), cudaMemcpyHostToDevice,
+                               p->io_stream)) != cudaSuccess ||
+        (e = cudaEventRecord(p->ev_v, p->io_stream)) != cudaSuccess ||
+        (e = cudaMemcpy2DAsync(dv + heads_a * head_bytes, pitch, hv + heads_a * head_bytes, pitch,
+                               (g.Hn - heads_a) * head_bytes, size_t(g.Lkv), cudaMemcpyHostToDevice,
+                               p->io_stream)) != cudaSuccess ||
+        (e = cudaEventRecord(p->ev_v2, p->io_stream)) != cudaSuccess)
+      return cuda_fail(e, "host-to-device copy");
+  } else if ((e = cudaMemcpyAsync(p->st_v, v, kb, cudaMemcpyHostToDevice, p->io_stream)) != cudaSuccess ||
+             (e = cudaEventRecord(p->ev_v, p->io_stream)) != cudaSuccess) {
+    return cuda_fail(e, "host-to-device copy");
+  }
   StepBlocks sb;
   sb.k_in_fb = g.Tkv / g.bt;
   sb.v_attn = p->st_v;
   sb.k3_wait = p->ev_v;
-  const int heads_a = g.B == 1 && g.Hn >= 2 ? g.Hn / 2 : 0;
   if (heads_a > 0) {
     const int64_t per_head = p->pair_col ? lcsa::pair_count(g) / g.Hn : int64_t(g.nQB);
     sb.k3_split = int(heads_a * per_head);
     sb.k3_first_done = p->ev_k3a;
+    sb.k3_wait_b = p->ev_v2;
   }
   lcsa_status_t st = run_step(p, p->st_q, p->st_k, p->st_gq, p->st_gk, p->st_out, s, sb);
   if (st != LCSA_OK) return st;
-  const size_t pitch = size_t(g.C) * 2, head_bytes = size_t(g.D) * 2;
   if (heads_a > 0) {
     if ((e = cudaStreamWaitEvent(p->io_stream, p->ev_k3a, 0)) != cudaSuccess ||
         (e = cudaMemcpy2DAsync(out, pitch, p->st_out, pitch, heads_a * head_bytes, size_t(g.Lq),

@@ -168,12 +168,14 @@ LCSA_API lcsa_status_t lcsa_forward(lcsa_plan_t plan, const void* q, const void*
 
 /* Same call from HOST buffers: copies q, k, v and the gains into plan-owned
    device staging, runs the call and copies out back. Needs a plan created
-   with host_io = 1 (which also creates a plan-owned copy stream and four
+   with host_io = 1 (which also creates a plan-owned copy stream and five
    events). The gains, q and k go up on `stream`, v on the copy stream once
    they are in, so the prologue and the selection run while v uploads; with
    batch 1 and at least two heads the attention runs as two launches over
-   the first and the second half of the heads, and the first half's output
-   channels come back on the copy stream while the second half computes.
+   the first and the second half of the heads, v goes up in those two halves
+   of its channels (each launch waits only for its own), and the first
+   half's output channels come back on the copy stream while the second half
+   computes.
    The result equals lcsa_forward's bit for bit. Host buffers should be pinned
    for asynchronous copies; the call returns once `out` holds the result,
    after reading the plan's device error word as lcsa_check_device_error does
