@@ -22,6 +22,9 @@ WL = {
                             topk=5, kv_frame_offset=2, field=True, unit_gain=False),
     "blocks64": _T.replace(heads=2, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
                            field=True, unit_gain=False),
+    # 160 query-block pairs: the last pairs are cut and merged inside the graph
+    "blocks64_cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                                     field=True, unit_gain=False, seed=25),
 }
 LAYERS = 3
 

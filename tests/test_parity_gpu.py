@@ -52,6 +52,8 @@ SMALL = {
     # are cut into parts and merged
     "blocks64_cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
                                      field=True, unit_gain=False, seed=21),
+    "d64_blocks64_cut_pairs": _T.replace(head_dim=64, heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40,
+                                         local_range=5, topk=9, field=True, unit_gain=False, seed=23),
 }
 OVERRIDES = {"tiny_head_scope": dict(norm_scope=1), "d64_head_scope": dict(norm_scope=1)}
 

@@ -25,6 +25,9 @@ CASES = {
                                topk=5, kv_frame_offset=2, field=True, unit_gain=False),
     "blocks64_odd_heads": _T.replace(heads=5, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
                                      field=True, unit_gain=False, seed=1),
+    # 160 query-block pairs: cut and merged, over reused thresholds
+    "blocks64_cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                                     field=True, unit_gain=False, seed=26),
     "stream_768x1280": synth.WORKLOADS["stream_768x1280"],
 }
 

@@ -31,6 +31,9 @@ STREAMS = {
     # head_dim 64
     "stream128_d64": _T.replace(head_dim=64, heads=4, q_frames=2, kv_frames=6, grid_h=24, grid_w=48, block_w=16,
                                 local_range=3, topk=5, field=True, unit_gain=False, seed=12),
+    # 160 query-block pairs, at least as many as the SMs: the last pairs are cut and merged
+    "stream64_cut_pairs": _T.replace(heads=8, q_frames=2, kv_frames=6, grid_h=32, grid_w=40, local_range=5, topk=7,
+                                     field=True, unit_gain=False, seed=24),
 }
 TOTAL_FRAMES = 10   # 4 pushed to fill the window, then three chunks of 2
 
