@@ -1013,10 +1013,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto slot_of = [&](int j) { return slot0 + j; };
       auto slice = [&](int j) { return p.part_buf + (int64_t(slot_of(j)) * 8 + wsl) * kSlice; };
       bool last = true;
+      unsigned before = 0;  // parts of this slice that arrived before this one
       if (parts > 1) {
-        unsigned before = 0;
         if (lane == 0) before = atomicAdd(p.merge_cnt + int64_t(rr - (p.rows - p.cut_items)) * 8 + wsl, 1u);
-        last = __shfl_sync(0xffffffffu, before, 0) + 1 == unsigned(parts);
+        before = __shfl_sync(0xffffffffu, before, 0);
+        last = before + 1 == unsigned(parts);
       }
       if (!last) {
         float* my = slice(part);
@@ -1036,7 +1037,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         my[32 * (D / 2) + 32 + lane] = l_row;
         __threadfence();
         __syncwarp();
-        if (lane == 0) flag_release(p.merge_ready + slot_of(part) * 8 + wsl);
+        bool flag = true;
+#ifdef LCSA_TEST_STALL
+        // the first part of the first cut pair to arrive, in slice 0, leaves
+        // its flag unset: the last part's wait for it runs out
+        if (p.stall_site == 3 && rr == p.rows - p.cut_items && before == 0 && wsl == 0) flag = false;
+#endif
+        if (lane == 0 && flag) flag_release(p.merge_ready + slot_of(part) * 8 + wsl);
       } else {
         float inv;
         if (parts > 1) {
@@ -1269,10 +1276,12 @@ cudaError_t launch_attention_tc(const K3Params& p, const CUtensorMap& tm_q, cons
 }  // namespace lcsa
 
 #ifdef LCSA_TEST_STALL
-// Test-only build: make the next attention launch give up a wait in its
-// first work item. site 1: the TMA producer aborts right after issuing the
-// item's first loads (they are still in flight); site 2: a softmax warp waits
-// on a barrier nothing arrives on until the (100 ms) limit. Either records
-// LCSA_ERR_DEVICE_TIMEOUT (error sites 91 / 92) and the kernel winds down.
+// Test-only build: make the next attention launch give up a wait. site 1:
+// the TMA producer aborts right after issuing its first work item's loads
+// (they are still in flight); site 2: a softmax warp waits on a barrier
+// nothing arrives on until the (100 ms) limit; site 3 (cut 64-token pairs):
+// one part of the first cut pair never flags its partial result, so the last
+// part's wait for it runs out. Each records LCSA_ERR_DEVICE_TIMEOUT (error
+// sites 91, 92 or the waiter's own, 27 for site 3) and the kernel winds down.
 extern "C" LCSA_API void lcsa_test_arm_stall(int site) { lcsa::g_stall_site = site; }
 #endif

@@ -7,13 +7,17 @@ status, and the same context and plan go on to compute correct results.
 It runs the test-only build liblcsa_stalltest.so (-DLCSA_TEST_STALL: waits
 give up after 100 ms; lcsa_test_arm_stall makes the next attention launch
 give up on purpose) in a child process, so the product library is never
-loaded beside it. Two ways to give up, each on 128-token blocks and on the
+loaded beside it. Ways to give up, each on 128-token blocks and on the
 paired 64-token path:
   site 1: the TMA producer gives up right after issuing its first work item's
           loads, while they are still in flight;
   site 2: a softmax warp waits on a barrier nothing arrives on, until the
           limit (the waits held up behind it run out at the same time, and
-          the first to give up records its site).
+          the first to give up records its site);
+  site 3 (with at least as many 64-token pairs as SMs, so the last pairs are
+          cut into parts): one part of the first cut pair never flags its
+          partial result, and the part that merges waits for it until the
+          limit (site 27, the merge's wait).
 Then lcsa_check_device_error must return LCSA_ERR_DEVICE_TIMEOUT, and the next
 call on the same plan must match the fp64 oracle. The same holds for the
 allocation-free entry point and its status call.
@@ -51,6 +55,9 @@ CASES = {{
                            topk=5, kv_frame_offset=2, field=True, unit_gain=False),
     "blocks64": T.replace(heads=2, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
                           field=True, unit_gain=False, seed=3),
+    # 160 pairs: the last are cut into parts and merged
+    "blocks64_cut_pairs": T.replace(heads=8, q_frames=2, kv_frames=4, grid_h=32, grid_w=40, local_range=5, topk=9,
+                                    field=True, unit_gain=False, seed=27),
 }}
 
 def err_vs_oracle(wl, inp, out):
@@ -67,7 +74,7 @@ for name, wl in CASES.items():
     inp = synth.make_inputs(wl)
     q, k, v, gq, gk = torch_inputs(inp)
     plan = L.lcsa_plan_create(L.config_from_workload(wl), 0)
-    for site in (1, 2):
+    for site in ((1, 2, 3) if "cut" in name else (1, 2)):
         out = torch.full_like(q, float("nan"))
         arm(site)
         plan.lcsa_forward(q, k, v, gq, gk, out)
@@ -77,7 +84,7 @@ for name, wl in CASES.items():
         # site 1 records at once; at site 2 the waits held up behind the
         # stalled warp (the P.V issuer's, a partner's exchange) run out at the
         # same limit, and whichever is first records its own site
-        assert ("site 91" in msg) if site == 1 else ("site " in msg), msg
+        assert {{1: "site 91", 2: "site ", 3: "site 27"}}[site] in msg, msg
         # the next call on the same plan and context is correct
         out = torch.full_like(q, float("nan"))
         plan.lcsa_forward(q, k, v, gq, gk, out)
